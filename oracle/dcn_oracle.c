@@ -1,0 +1,369 @@
+/*
+ * Float64 CPU oracle for the modulated deformable convolution (DCNv2).
+ *
+ * TEST INFRASTRUCTURE. Only tests/, __graft_entry__.smoke() and the CPU-baseline
+ * leg of bench.py may load this library. The product (the CUDA library under
+ * deformable_convolution_dcn_b200/) never calls it and shares no code with it.
+ *
+ * What is computed (all sums in float64, in the order written below):
+ *
+ *   y(p0) = bias + sum_{k in R} w(p_k) * m_k * x(p0 + p_k + dp_k)
+ *
+ *   - the plain convolution over the regular grid R and its deformable form with
+ *     a learned offset dp_k per tap ("Deformable ConvNets" notes, section
+ *     "可变形卷积", the two y(p0) equations);
+ *   - the DCNv2 modulation scalar m_k that multiplies each sampled value
+ *     ("DCNv2", section 3.2 "添加幅值参数"; the tutorial's mask argument, table in
+ *     section 2.1, default all ones);
+ *   - x(p) at a fractional p is bilinear interpolation over the four integer
+ *     neighbours, each weighted by the area of the opposite sub-rectangle
+ *     (notes, "双线性插值" equation S1..S4);
+ *   - channels are split into G deformable groups, every channel of a group
+ *     sharing one offset field (notes, "Deformable Group");
+ *   - torchvision deform_conv2d conventions for layout and borders (tutorial,
+ *     section 2 "解剖torchvision.ops.deform_conv2d"): offsets carry 2*G*K*K
+ *     channels with channel g*2K^2 + 2k = dy (row) and +1 = dx (column); a
+ *     neighbour that lies outside the map contributes zero (no clamping).
+ *
+ * Layouts (row-major, innermost last):
+ *   x       [B, H, W, Cin]                  channel-contiguous (NHWC)
+ *   offset  [B, 2*G*K*K, Ho, Wo]
+ *   mask    [B, G*K*K, Ho, Wo]              NULL means m = 1 everywhere (DCNv1)
+ *   weight  [Cout, K, K, Cin]
+ *   bias    [Cout]                          NULL means no bias
+ *   y       [B, Ho, Wo, Cout]
+ *   Ho = (H + 2*pad - dil*(K-1) - 1) / stride + 1, likewise Wo.
+ *
+ * Tap k = i*K + j (i = kernel row, j = kernel column) samples at
+ *   py = ho*stride - pad + i*dil + dy,   px = wo*stride - pad + j*dil + dx.
+ *
+ * Backward: the chain rule through the same expression. The offset gradient is
+ * the page's d y(p0) / d dp_n = sum w(p_n) * sum_q dG(q, p)/d dp_n * x(q)
+ * (notes, "计算梯度"), with dG taken through floor(p): at an exact integer
+ * coordinate the derivative uses the neighbours floor(p) and floor(p)+1, i.e. the
+ * right-hand derivative (the tutorial, section 3.2, notes the kink there).
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+typedef struct {
+    int B, H, W, Cin, Cout, K, stride, pad, dil, G;
+} dcn_oracle_shape;
+
+int dcn_oracle_out_h(const dcn_oracle_shape* s) {
+    return (s->H + 2 * s->pad - s->dil * (s->K - 1) - 1) / s->stride + 1;
+}
+int dcn_oracle_out_w(const dcn_oracle_shape* s) {
+    return (s->W + 2 * s->pad - s->dil * (s->K - 1) - 1) / s->stride + 1;
+}
+
+void dcn_oracle_set_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+int dcn_oracle_max_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* ---------------------------------------------------------------- sampling -- */
+
+/* Value of channel c of image b at integer (r, q); zero outside the map. */
+static double pixel_or_zero(const double* x, const dcn_oracle_shape* s, int b, int r, int q, int c) {
+    if (r < 0 || r >= s->H || q < 0 || q >= s->W) return 0.0;
+    return x[(((size_t)b * s->H + r) * s->W + q) * s->Cin + c];
+}
+
+/* Bilinear interpolation at fractional (py, px): the four integer neighbours
+ * (floor(py) + a, floor(px) + e), a, e in {0, 1}, weighted by
+ * (1 - |py - row|) * (1 - |px - col|). */
+static double bilinear(const double* x, const dcn_oracle_shape* s, int b, int c, double py, double px) {
+    double y0 = floor(py), x0 = floor(px);
+    double v = 0.0;
+    for (int a = 0; a < 2; ++a)
+        for (int e = 0; e < 2; ++e) {
+            double r = y0 + a, q = x0 + e;
+            double g = (1.0 - fabs(py - r)) * (1.0 - fabs(px - q));
+            v += g * pixel_or_zero(x, s, b, (int)r, (int)q, c);
+        }
+    return v;
+}
+
+/* d bilinear / d py and d bilinear / d px, taken through floor(): the row
+ * factor of neighbour row y0 is (1 - (py - y0)) with derivative -1, that of
+ * row y0 + 1 is (py - y0) with derivative +1; likewise for columns. */
+static void bilinear_grad(const double* x, const dcn_oracle_shape* s, int b, int c, double py, double px,
+                          double* dpy, double* dpx) {
+    double y0 = floor(py), x0 = floor(px);
+    double ly = py - y0, lx = px - x0;
+    double v00 = pixel_or_zero(x, s, b, (int)y0, (int)x0, c);
+    double v01 = pixel_or_zero(x, s, b, (int)y0, (int)x0 + 1, c);
+    double v10 = pixel_or_zero(x, s, b, (int)y0 + 1, (int)x0, c);
+    double v11 = pixel_or_zero(x, s, b, (int)y0 + 1, (int)x0 + 1, c);
+    *dpy = (1.0 - lx) * (v10 - v00) + lx * (v11 - v01);
+    *dpx = (1.0 - ly) * (v01 - v00) + ly * (v11 - v10);
+}
+
+/* Sampling position, modulation scalar for tap k = i*K + j of group g at output
+ * pixel (b, ho, wo). */
+static void tap_position(const dcn_oracle_shape* s, const double* off, const double* mask, int b, int ho, int wo,
+                         int g, int i, int j, double* py, double* px, double* m) {
+    int Ho = dcn_oracle_out_h(s), Wo = dcn_oracle_out_w(s);
+    int K2 = s->K * s->K, k = i * s->K + j;
+    size_t plane = (size_t)Ho * Wo, pix = (size_t)ho * Wo + wo;
+    double dy = off[((size_t)b * 2 * s->G * K2 + (size_t)g * 2 * K2 + 2 * k) * plane + pix];
+    double dx = off[((size_t)b * 2 * s->G * K2 + (size_t)g * 2 * K2 + 2 * k + 1) * plane + pix];
+    *py = (double)(ho * s->stride - s->pad + i * s->dil) + dy;
+    *px = (double)(wo * s->stride - s->pad + j * s->dil) + dx;
+    *m = mask ? mask[((size_t)b * s->G * K2 + (size_t)g * K2 + k) * plane + pix] : 1.0;
+}
+
+static size_t weight_index(const dcn_oracle_shape* s, int o, int i, int j, int c) {
+    return (((size_t)o * s->K + i) * s->K + j) * s->Cin + c;
+}
+
+/* ----------------------------------------------------------------- forward -- */
+
+/* y for one output pixel p (flat index into B*Ho*Wo), all Cout channels. */
+static void forward_pixel(const dcn_oracle_shape* s, const double* x, const double* off, const double* mask,
+                          const double* w, const double* bias, long p, double* yrow) {
+    int Ho = dcn_oracle_out_h(s), Wo = dcn_oracle_out_w(s);
+    int b = (int)(p / ((long)Ho * Wo)), ho = (int)((p / Wo) % Ho), wo = (int)(p % Wo);
+    int Cg = s->Cin / s->G;
+    for (int o = 0; o < s->Cout; ++o) yrow[o] = bias ? bias[o] : 0.0;
+    for (int g = 0; g < s->G; ++g)
+        for (int i = 0; i < s->K; ++i)
+            for (int j = 0; j < s->K; ++j) {
+                double py, px, m;
+                tap_position(s, off, mask, b, ho, wo, g, i, j, &py, &px, &m);
+                for (int c = g * Cg; c < (g + 1) * Cg; ++c) {
+                    double v = m * bilinear(x, s, b, c, py, px);
+                    for (int o = 0; o < s->Cout; ++o) yrow[o] += w[weight_index(s, o, i, j, c)] * v;
+                }
+            }
+}
+
+/* Forward at a list of output pixels (pix == NULL: every pixel in order).
+ * y receives npix rows of Cout values. */
+int dcn_oracle_forward_pixels(const dcn_oracle_shape* s, const double* x, const double* off, const double* mask,
+                              const double* w, const double* bias, long npix, const long* pix, double* y) {
+    if (s->G <= 0 || s->Cin % s->G) return -1;
+    long n;
+#pragma omp parallel for schedule(dynamic, 16)
+    for (n = 0; n < npix; ++n) forward_pixel(s, x, off, mask, w, bias, pix ? pix[n] : n, y + (size_t)n * s->Cout);
+    return 0;
+}
+
+int dcn_oracle_forward(const dcn_oracle_shape* s, const double* x, const double* off, const double* mask,
+                       const double* w, const double* bias, double* y) {
+    long P = (long)s->B * dcn_oracle_out_h(s) * dcn_oracle_out_w(s);
+    return dcn_oracle_forward_pixels(s, x, off, mask, w, bias, P, NULL, y);
+}
+
+/* Single bilinear sample of a [H, W, C] image at (py, px), C values. */
+void dcn_oracle_bilinear(int H, int W, int C, const double* img, double py, double px, double* out) {
+    dcn_oracle_shape s = {1, H, W, C, 1, 1, 1, 0, 1, 1};
+    for (int c = 0; c < C; ++c) out[c] = bilinear(img, &s, 0, c, py, px);
+}
+
+/* ---------------------------------------------------------------- backward -- */
+
+/* Upstream gradient propagated to the sampled column: gcol = sum_o gy[o] * w[o, i, j, c]. */
+static double column_grad(const dcn_oracle_shape* s, const double* w, const double* gyrow, int i, int j, int c) {
+    double acc = 0.0;
+    for (int o = 0; o < s->Cout; ++o) acc += gyrow[o] * w[weight_index(s, o, i, j, c)];
+    return acc;
+}
+
+/* Full backward. Any output pointer may be NULL. Outputs are overwritten.
+ *   gx [B,H,W,Cin], goff [B,2GK^2,Ho,Wo], gmask [B,GK^2,Ho,Wo] (needs mask),
+ *   gw [Cout,K,K,Cin], gb [Cout].
+ * Parallel over the batch: image b's pixels only touch gx[b]; gw and gb are
+ * accumulated per image and summed over b in order afterwards. */
+int dcn_oracle_backward(const dcn_oracle_shape* s, const double* x, const double* off, const double* mask,
+                        const double* w, const double* gy, double* gx, double* goff, double* gmask, double* gw,
+                        double* gb) {
+    if (s->G <= 0 || s->Cin % s->G) return -1;
+    int Ho = dcn_oracle_out_h(s), Wo = dcn_oracle_out_w(s);
+    int K2 = s->K * s->K, Cg = s->Cin / s->G;
+    size_t nw = (size_t)s->Cout * K2 * s->Cin, plane = (size_t)Ho * Wo;
+    double* gw_b = (double*)calloc(nw * s->B, sizeof(double));
+    double* gb_b = (double*)calloc((size_t)s->Cout * s->B, sizeof(double));
+    if (!gw_b || !gb_b) {
+        free(gw_b);
+        free(gb_b);
+        return -2;
+    }
+    if (gx) memset(gx, 0, sizeof(double) * (size_t)s->B * s->H * s->W * s->Cin);
+    int b;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (b = 0; b < s->B; ++b) {
+        double* gwb = gw_b + nw * b;
+        double* gbb = gb_b + (size_t)s->Cout * b;
+        for (int ho = 0; ho < Ho; ++ho)
+            for (int wo = 0; wo < Wo; ++wo) {
+                size_t p = ((size_t)b * Ho + ho) * Wo + wo;
+                const double* gyrow = gy + p * s->Cout;
+                for (int o = 0; o < s->Cout; ++o) gbb[o] += gyrow[o];
+                for (int g = 0; g < s->G; ++g)
+                    for (int i = 0; i < s->K; ++i)
+                        for (int j = 0; j < s->K; ++j) {
+                            int k = i * s->K + j;
+                            double py, px, m;
+                            tap_position(s, off, mask, b, ho, wo, g, i, j, &py, &px, &m);
+                            double y0 = floor(py), x0 = floor(px);
+                            double gdy = 0.0, gdx = 0.0, gm = 0.0;
+                            for (int c = g * Cg; c < (g + 1) * Cg; ++c) {
+                                double gcol = column_grad(s, w, gyrow, i, j, c);
+                                double v = bilinear(x, s, b, c, py, px);
+                                double dpy, dpx;
+                                bilinear_grad(x, s, b, c, py, px, &dpy, &dpx);
+                                gm += gcol * v;
+                                gdy += gcol * m * dpy;
+                                gdx += gcol * m * dpx;
+                                for (int o = 0; o < s->Cout; ++o) gwb[weight_index(s, o, i, j, c)] += gyrow[o] * m * v;
+                                if (gx)
+                                    for (int a = 0; a < 2; ++a)
+                                        for (int e = 0; e < 2; ++e) {
+                                            int r = (int)y0 + a, q = (int)x0 + e;
+                                            if (r < 0 || r >= s->H || q < 0 || q >= s->W) continue;
+                                            double gq = (1.0 - fabs(py - r)) * (1.0 - fabs(px - q));
+                                            gx[(((size_t)b * s->H + r) * s->W + q) * s->Cin + c] += gcol * m * gq;
+                                        }
+                            }
+                            size_t ob = (size_t)b * 2 * s->G * K2 + (size_t)g * 2 * K2 + 2 * k;
+                            if (goff) {
+                                goff[ob * plane + (size_t)ho * Wo + wo] = gdy;
+                                goff[(ob + 1) * plane + (size_t)ho * Wo + wo] = gdx;
+                            }
+                            if (gmask && mask) gmask[((size_t)b * s->G * K2 + (size_t)g * K2 + k) * plane + (size_t)ho * Wo + wo] = gm;
+                        }
+            }
+    }
+    if (gw) {
+        memset(gw, 0, sizeof(double) * nw);
+        for (int bb = 0; bb < s->B; ++bb)
+            for (size_t t = 0; t < nw; ++t) gw[t] += gw_b[nw * bb + t];
+    }
+    if (gb) {
+        memset(gb, 0, sizeof(double) * s->Cout);
+        for (int bb = 0; bb < s->B; ++bb)
+            for (int o = 0; o < s->Cout; ++o) gb[o] += gb_b[(size_t)s->Cout * bb + o];
+    }
+    free(gw_b);
+    free(gb_b);
+    return 0;
+}
+
+/* --------------------------------------------- backward at sampled entries -- */
+/* These compute single gradient entries straight from their definitions, so that
+ * full-size problems can be checked at sampled positions. */
+
+/* grad_offset (2GK^2 values) and grad_mask (GK^2 values) for listed output pixels. */
+int dcn_oracle_grad_offset_mask_pixels(const dcn_oracle_shape* s, const double* x, const double* off,
+                                       const double* mask, const double* w, const double* gy, long npix,
+                                       const long* pix, double* goff, double* gmask) {
+    if (s->G <= 0 || s->Cin % s->G) return -1;
+    int Ho = dcn_oracle_out_h(s), Wo = dcn_oracle_out_w(s);
+    int K2 = s->K * s->K, Cg = s->Cin / s->G;
+    long n;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (n = 0; n < npix; ++n) {
+        long p = pix[n];
+        int b = (int)(p / ((long)Ho * Wo)), ho = (int)((p / Wo) % Ho), wo = (int)(p % Wo);
+        const double* gyrow = gy + (size_t)p * s->Cout;
+        for (int g = 0; g < s->G; ++g)
+            for (int i = 0; i < s->K; ++i)
+                for (int j = 0; j < s->K; ++j) {
+                    int k = i * s->K + j;
+                    double py, px, m;
+                    tap_position(s, off, mask, b, ho, wo, g, i, j, &py, &px, &m);
+                    double gdy = 0.0, gdx = 0.0, gm = 0.0;
+                    for (int c = g * Cg; c < (g + 1) * Cg; ++c) {
+                        double gcol = column_grad(s, w, gyrow, i, j, c);
+                        double dpy, dpx;
+                        bilinear_grad(x, s, b, c, py, px, &dpy, &dpx);
+                        gm += gcol * bilinear(x, s, b, c, py, px);
+                        gdy += gcol * m * dpy;
+                        gdx += gcol * m * dpx;
+                    }
+                    goff[(size_t)n * 2 * s->G * K2 + (size_t)g * 2 * K2 + 2 * k] = gdy;
+                    goff[(size_t)n * 2 * s->G * K2 + (size_t)g * 2 * K2 + 2 * k + 1] = gdx;
+                    if (gmask) gmask[(size_t)n * s->G * K2 + (size_t)g * K2 + k] = gm;
+                }
+    }
+    return 0;
+}
+
+/* grad_weight at listed flat indices into [Cout, K, K, Cin]:
+ * sum over every output pixel of gy[p, o] * m * x(sample). */
+int dcn_oracle_grad_weight_entries(const dcn_oracle_shape* s, const double* x, const double* off, const double* mask,
+                                   const double* gy, long n_ent, const long* idx, double* out) {
+    if (s->G <= 0 || s->Cin % s->G) return -1;
+    int Ho = dcn_oracle_out_h(s), Wo = dcn_oracle_out_w(s);
+    int Cg = s->Cin / s->G;
+    long n;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (n = 0; n < n_ent; ++n) {
+        long t = idx[n];
+        int c = (int)(t % s->Cin), j = (int)((t / s->Cin) % s->K), i = (int)((t / ((long)s->Cin * s->K)) % s->K);
+        int o = (int)(t / ((long)s->Cin * s->K * s->K));
+        int g = c / Cg;
+        double acc = 0.0;
+        for (int b = 0; b < s->B; ++b)
+            for (int ho = 0; ho < Ho; ++ho)
+                for (int wo = 0; wo < Wo; ++wo) {
+                    double py, px, m;
+                    tap_position(s, off, mask, b, ho, wo, g, i, j, &py, &px, &m);
+                    size_t p = ((size_t)b * Ho + ho) * Wo + wo;
+                    acc += gy[p * s->Cout + o] * m * bilinear(x, s, b, c, py, px);
+                }
+        out[n] = acc;
+    }
+    return 0;
+}
+
+/* grad_x at listed flat indices into [B, H, W, Cin]: every (output pixel, tap)
+ * of image b whose bilinear neighbourhood contains the input pixel adds
+ * gcol * m * (its bilinear weight). */
+int dcn_oracle_grad_x_entries(const dcn_oracle_shape* s, const double* off, const double* mask, const double* w,
+                              const double* gy, long n_ent, const long* idx, double* out) {
+    if (s->G <= 0 || s->Cin % s->G) return -1;
+    int Ho = dcn_oracle_out_h(s), Wo = dcn_oracle_out_w(s);
+    int Cg = s->Cin / s->G;
+    long n;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (n = 0; n < n_ent; ++n) {
+        long t = idx[n];
+        int c = (int)(t % s->Cin), q = (int)((t / s->Cin) % s->W), r = (int)((t / ((long)s->Cin * s->W)) % s->H);
+        int b = (int)(t / ((long)s->Cin * s->W * s->H));
+        int g = c / Cg;
+        double acc = 0.0;
+        for (int ho = 0; ho < Ho; ++ho)
+            for (int wo = 0; wo < Wo; ++wo) {
+                const double* gyrow = gy + (((size_t)b * Ho + ho) * Wo + wo) * s->Cout;
+                for (int i = 0; i < s->K; ++i)
+                    for (int j = 0; j < s->K; ++j) {
+                        double py, px, m;
+                        tap_position(s, off, mask, b, ho, wo, g, i, j, &py, &px, &m);
+                        double y0 = floor(py), x0 = floor(px);
+                        if (!(r == (int)y0 || r == (int)y0 + 1) || !(q == (int)x0 || q == (int)x0 + 1)) continue;
+                        double gq = (1.0 - fabs(py - r)) * (1.0 - fabs(px - q));
+                        acc += column_grad(s, w, gyrow, i, j, c) * m * gq;
+                    }
+            }
+        out[n] = acc;
+    }
+    return 0;
+}
