@@ -1,0 +1,470 @@
+#!/usr/bin/env python
+"""Benchmark of the DCNv2 layer on B200: forward TFLOP/s and % of roofline.
+
+One step is one pass of the whole hot path over one batch of synthetic input:
+the forward (sampling coordinates, bilinear x mask, gather, tensor-core
+contraction, epilogue) and the full backward (grad_x, grad_offset, grad_mask in
+one data pass; grad_weight and grad_bias in one weight pass), on the ResNet-50
+conv4 3x3 DCNv2 layer (B=8, Cin=Cout=256, 50x50, K=3, stride 1, pad 1, G=1,
+bfloat16 in / float32 accumulate). ``value`` is the forward's TFLOP/s (the
+metric), from CUDA events around the forward launches inside the timed steps;
+``ms_per_step`` covers the whole step. Inputs rotate over enough independent
+sets that every step reads from HBM, not from a warm L2.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload conv4] [--impl ours|reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own independent
+layer instance (weak scaling, no collective on the data path); the time is the
+max over ranks, the value the sum of all ranks' work over that time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "DCNv2 forward TFLOP/s and % of roofline (bf16, B200) per layer shape"
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks --
+
+class ClockSampler:
+    """nvidia-smi sampled every 100 ms while the timed region runs."""
+
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        time.sleep(0.25)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx.append(float(f[1]))
+                power.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(power) if power else None, "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------ distributed --
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def dist_init(backend, timeout_s=120):
+    import datetime
+
+    import torch.distributed as dist
+    rank, world, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
+    return rank, world
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a float over all ranks (identity with one rank)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# -------------------------------------------------------------- work model --
+
+def work_model(s, elem=2):
+    """Algorithmic FLOPs and minimal HBM bytes per launch of each pass."""
+    nx = s.B * s.H * s.W * s.Cin
+    noff = s.P * 2 * s.G * s.K * s.K
+    nm = s.P * s.G * s.K * s.K
+    nw = s.Cout * s.K * s.K * s.Cin
+    ny = s.P * s.Cout
+    f = s.flops()
+    return {
+        "forward": {"flops": f, "bytes": elem * (nx + noff + nm + nw + ny)},
+        "backward_data": {"flops": f, "bytes": elem * (nx + noff + nm + nw + ny) + 4 * (nx + noff + nm)},
+        "backward_weight": {"flops": f, "bytes": elem * (nx + noff + nm + ny) + 4 * (nw + s.Cout)},
+    }
+
+
+def roofline_entry(work, seconds, pk, sustained):
+    tflop = pk["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    t_flop = work["flops"] / (tflop * 1e12)
+    t_hbm = work["bytes"] / (pk["hbm_gbs"] * 1e9)
+    if t_flop >= t_hbm:
+        ach = work["flops"] / seconds / 1e12
+        return {"bound": "tensor", "achieved": round(ach, 2), "peak": tflop, "unit": "TFLOP/s",
+                "frac": round(ach / tflop, 4), "roofline_frac": round(max(t_flop, t_hbm) / seconds, 4)}
+    ach = work["bytes"] / seconds / 1e9
+    return {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": round(ach / pk["hbm_gbs"], 4), "roofline_frac": round(max(t_flop, t_hbm) / seconds, 4)}
+
+
+# ---------------------------------------------------------------- our arm --
+
+def run_ours(args):
+    import torch
+
+    import deformable_convolution_dcn_b200 as dcn
+    from deformable_convolution_dcn_b200 import inputs as gen
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist_init("nccl")
+    w = gen.WORKLOADS[args.workload]
+    s = w.shape
+    do_bwd = not args.forward_only
+    elem = 2 if w.dtype == "bf16" else 4
+    wm = work_model(s, elem)
+    pk, pk_src = peaks()
+
+    # rotating input sets so that every step reads its inputs from HBM
+    host = gen.make_inputs(w if do_bwd else w, seed=w.seed)
+    if do_bwd and "grad_y" not in host:
+        g = torch.Generator().manual_seed(w.seed + 99)
+        host["grad_y"] = torch.randn((s.B, s.Ho, s.Wo, s.Cout), generator=g).to(host["x"].dtype)
+    set_bytes = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
+    out_bytes = wm["forward"]["bytes"] - elem * (s.B * s.H * s.W * s.Cin)  # rough; only sizes the rotation
+    n_sets = max(2, min(64, math.ceil(3 * L2_BYTES / max(1, set_bytes + out_bytes)) + 1))
+    sets = []
+    for k in range(n_sets):
+        d = {}
+        for name, t in host.items():
+            if t is None:
+                d[name] = None
+            elif k == 0:
+                d[name] = t.to(device)
+            else:  # an independent copy in its own memory
+                d[name] = t.to(device) if name == "weight" and k % 2 == 0 else t.to(device).clone()
+        sets.append(d)
+    f32 = dict(dtype=torch.float32, device=device)
+    outs = []
+    for k in range(n_sets):
+        o = {"y": torch.empty((s.B, s.Ho, s.Wo, s.Cout), dtype=host["x"].dtype, device=device)}
+        if do_bwd:
+            o["grad_x"] = torch.empty((s.B, s.H, s.W, s.Cin), **f32)
+            o["grad_offset"] = torch.empty(tuple(host["offset"].shape), **f32)
+            o["grad_mask"] = torch.empty(tuple(host["mask"].shape), **f32) if host["mask"] is not None else None
+            o["grad_weight"] = torch.empty(tuple(host["weight"].shape), **f32)
+            o["grad_bias"] = torch.empty((s.Cout,), **f32)
+        outs.append(o)
+    p = dcn._params(sets[0]["x"], sets[0]["weight"], sets[0]["offset"], s.stride, s.pad, s.dil, False)
+    ws = {op: (torch.empty(max(1, dcn.workspace_size(p, op)), dtype=torch.uint8, device=device))
+          for op in (dcn.OP_FORWARD, dcn.OP_BACKWARD_DATA, dcn.OP_BACKWARD_WEIGHT)}
+
+    def step(k, ev=None):
+        d, o = sets[k % n_sets], outs[k % n_sets]
+        if ev is not None:
+            ev[0].record()
+        dcn.forward(d["x"], d["offset"], d["mask"], d["weight"], d["bias"], s.stride, s.pad, s.dil, out=o["y"],
+                    workspace=ws[dcn.OP_FORWARD])
+        if ev is not None:
+            ev[1].record()
+        if do_bwd:
+            dcn.backward_data(d["x"], d["offset"], d["mask"], d["weight"], d["grad_y"], s.stride, s.pad, s.dil,
+                              out=(o["grad_x"], o["grad_offset"], o["grad_mask"]),
+                              workspace=ws[dcn.OP_BACKWARD_DATA])
+            if ev is not None:
+                ev[2].record()
+            dcn.backward_weight(d["x"], d["offset"], d["mask"], d["grad_y"], tuple(d["weight"].shape), s.stride,
+                                s.pad, s.dil, out=(o["grad_weight"], o["grad_bias"]),
+                                workspace=ws[dcn.OP_BACKWARD_WEIGHT])
+            if ev is not None:
+                ev[3].record()
+
+    for k in range(args.warmup):
+        step(k)
+    torch.cuda.synchronize()
+    dcn.check_status()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(device)
+    torch.cuda.synchronize()
+    launches0 = dcn.launch_count()
+    t0.record()
+    for k in range(args.steps):
+        step(args.warmup + k, evs[k])
+    t1.record()
+    torch.cuda.synchronize()
+    launches = dcn.launch_count() - launches0
+    barrier(device)
+    clk = clocks.stop()
+    dcn.check_status()
+    total_ms = t0.elapsed_time(t1)
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    bd_ms = [e[1].elapsed_time(e[2]) for e in evs] if do_bwd else []
+    bw_ms = [e[2].elapsed_time(e[3]) for e in evs] if do_bwd else []
+
+    total_ms_max = max_over_ranks(total_ms, device)
+    fwd_sum_max = max_over_ranks(sum(fwd_ms), device)
+    value = world * args.steps * wm["forward"]["flops"] / (fwd_sum_max / 1e3) / 1e12
+
+    per = {"forward": statistics.mean(fwd_ms) / 1e3}
+    if do_bwd:
+        per["backward_data"] = statistics.mean(bd_ms) / 1e3
+        per["backward_weight"] = statistics.mean(bw_ms) / 1e3
+    rl = {k: roofline_entry(wm[k], t, pk, sustained=True) for k, t in per.items()}
+    dominant = max(per, key=per.get)
+    traffic = load_traffic(args.workload, dominant)
+    roof = dict(rl[dominant])
+    roof.update({"kernel": dominant, "traffic": traffic, "peak_source": pk_src + " (sustained bf16, HBM copy)",
+                 "share_of_step": round(per[dominant] / (total_ms / args.steps / 1e3), 3)})
+
+    e2e = measure_e2e(args, s, host, device, wm) if rank == 0 else None
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, host, args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(total_ms_max / args.steps, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.description, "name": w.name, "B": s.B, "Cin": s.Cin, "Cout": s.Cout,
+                       "H": s.H, "W": s.W, "K": s.K, "stride": s.stride, "pad": s.pad, "dil": s.dil, "G": s.G,
+                       "step": "forward + backward_data + backward_weight" if do_bwd else "forward",
+                       "l2": "inputs and outputs rotate over %d independent sets (%.0f MB each) so each step "
+                             "reads from HBM" % (n_sets, (set_bytes + out_bytes) / 1e6),
+                       "parallelism": "1 GPU" if world == 1 else "%d independent replicas" % world,
+                       "forward_path": dcn.forward_path(p)},
+            "roofline": roof,
+            "kernels": {k: dict(rl[k], us=round(per[k] * 1e6, 2)) for k in per},
+            "forward": {"us": round(per["forward"] * 1e6, 2), "tflops": round(wm["forward"]["flops"] /
+                                                                             per["forward"] / 1e12, 2),
+                        "roofline_frac": rl["forward"]["roofline_frac"]},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+
+
+def load_traffic(workload, kernel):
+    """DRAM bytes per launch from a committed ncu summary, or None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        return json.load(open(path))[workload][kernel]
+    except Exception:
+        return None
+
+
+def measure_e2e(args, s, host, device, wm):
+    """Forward through the public API with host buffers: pinned H2D of the
+    inputs, the forward, D2H of y, all inside the timed region."""
+    import torch
+
+    import deformable_convolution_dcn_b200 as dcn
+    pin = {k: (None if v is None else v.pin_memory()) for k, v in host.items() if k != "grad_y"}
+    dev = {k: (None if v is None else torch.empty_like(v, device=device)) for k, v in pin.items()}
+    y_dev = torch.empty((s.B, s.Ho, s.Wo, s.Cout), dtype=host["x"].dtype, device=device)
+    y_host = torch.empty(y_dev.shape, dtype=y_dev.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pin.values() if v is not None)
+    d2h = y_host.numel() * y_host.element_size()
+    n = max(3, min(args.steps, 20))
+
+    def one():
+        for k, v in pin.items():
+            if v is not None:
+                dev[k].copy_(v, non_blocking=True)
+        dcn.forward(dev["x"], dev["offset"], dev["mask"], dev["weight"], dev["bias"], s.stride, s.pad, s.dil,
+                    out=y_dev)
+        y_host.copy_(y_dev, non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(n):
+        one()
+    b.record()
+    torch.cuda.synchronize()
+    sec = a.elapsed_time(b) / 1e3 / n
+    return {"value": round(wm["forward"]["flops"] / sec / 1e12, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": round(sec * 1e3, 4)}
+
+
+# ---------------------------------------------------------- CPU baseline --
+
+def _oracle_arrays(host):
+    from deformable_convolution_dcn_b200 import inputs as gen
+    return {k: gen.as_f64(v) for k, v in host.items()}
+
+
+def cpu_baseline(w, host, seconds=10.0):
+    """The float64 oracle, as it stands, on the host cores: the forward over a
+    growing sample of output pixels until it runs for about `seconds`."""
+    import numpy as np
+
+    import oracle
+    s = w.shape
+    a = _oracle_arrays(host)
+    cores = len(os.sched_getaffinity(0))
+    oracle.set_threads(cores)
+    n = 64
+    while True:
+        pix = np.linspace(0, s.P - 1, min(n, s.P)).astype(np.int64)
+        t = time.perf_counter()
+        oracle.forward(a["x"], a["offset"], a["mask"], a["weight"], a["bias"], s.stride, s.pad, s.dil, s.G,
+                       pixels=pix)
+        dt = time.perf_counter() - t
+        if dt >= seconds / 3 or len(pix) >= s.P:
+            break
+        n = int(n * min(8.0, max(2.0, seconds / 3 / max(dt, 1e-3))))
+    flops = s.flops() * len(pix) / s.P
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.max_threads(),
+            "kind": "oracle", "sample": "forward at %d of %d output pixels (all %d output channels), %.2f s" %
+                                        (len(pix), s.P, s.Cout, dt)}
+
+
+# ---------------------------------------------------------- reference arm --
+
+def run_reference(args):
+    """The oracle as the reference arm: each step is the float64 forward over a
+    bounded sample of the same workload's output pixels, on the host cores."""
+    import numpy as np
+
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    from deformable_convolution_dcn_b200 import inputs as gen
+    w = gen.WORKLOADS[args.workload]
+    s = w.shape
+    host = gen.make_inputs(w)
+    a = _oracle_arrays(host)
+    cores = len(os.sched_getaffinity(0))
+    oracle.set_threads(cores)
+    budget = float(os.environ.get("DCN_REFERENCE_STEP_SECONDS", "1.0"))
+    npix = 32
+    while npix < s.P:   # size one step to about `budget` seconds
+        pix = np.linspace(0, s.P - 1, npix).astype(np.int64)
+        t = time.perf_counter()
+        oracle.forward(a["x"], a["offset"], a["mask"], a["weight"], a["bias"], s.stride, s.pad, s.dil, s.G,
+                       pixels=pix)
+        dt = time.perf_counter() - t
+        if dt >= budget / 2:
+            break
+        npix = min(s.P, npix * 2)
+    pix = np.linspace(0, s.P - 1, npix).astype(np.int64)
+    for _ in range(args.warmup):
+        oracle.forward(a["x"], a["offset"], a["mask"], a["weight"], a["bias"], s.stride, s.pad, s.dil, s.G,
+                       pixels=pix)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.forward(a["x"], a["offset"], a["mask"], a["weight"], a["bias"], s.stride, s.pad, s.dil, s.G,
+                       pixels=pix)
+    dt = (time.perf_counter() - t) / args.steps
+    flops = s.flops() * npix / s.P
+    value = flops / dt / 1e12
+    sample = "forward at %d of %d output pixels per step (all %d output channels)" % (npix, s.P, s.Cout)
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.description, "name": w.name, "reference": "float64 CPU oracle (oracle/)"},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "kind": "oracle",
+                             "cores": oracle.max_threads(), "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="conv4", help="conv4 | conv3_s2 | conv5_d2g4 | stem | tiny | conv4_bwd")
+    ap.add_argument("--forward-only", action="store_true", help="time the forward alone (not the default step)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("at least 3 warm-up steps")
+    if args.workload == "conv4_bwd":
+        args.workload = "conv4"
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,250 @@
+// C ABI of libdcn_b200 (declared in include/dcn.h): argument checks, workspace
+// sizing and dispatch to the kernels. Nothing here computes the convolution;
+// every step runs in the CUDA kernels.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <atomic>
+#include <string>
+
+#include "dcn.h"
+#include "kernels.h"
+
+namespace {
+
+thread_local std::string g_err;
+std::atomic<unsigned long long> g_launches{0};
+
+int fail(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return code;
+}
+
+int ok() {
+    g_err.clear();
+    return DCN_OK;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+    return fail(DCN_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
+}
+
+const long long kMaxElems = (1LL << 31) - 1;
+
+// Validates params and fills the kernel-side shape. Returns DCN_OK or an error code (message set).
+int make_shape(const dcn_params_t* p, dcn::Shape& s) {
+    if (!p) return fail(DCN_ERR_INVALID_ARG, "params is NULL");
+    if (p->B < 1 || p->H < 1 || p->W < 1 || p->Cin < 1 || p->Cout < 1 || p->K < 1 || p->stride < 1 || p->dil < 1 ||
+        p->G < 1 || p->pad < 0)
+        return fail(DCN_ERR_INVALID_ARG,
+                    "sizes must be positive (B=%d H=%d W=%d Cin=%d Cout=%d K=%d stride=%d dil=%d G=%d) and pad >= 0 "
+                    "(pad=%d)",
+                    p->B, p->H, p->W, p->Cin, p->Cout, p->K, p->stride, p->dil, p->G, p->pad);
+    if (p->Cin % p->G) return fail(DCN_ERR_INVALID_ARG, "Cin=%d is not a multiple of G=%d", p->Cin, p->G);
+    if (p->dtype != DCN_F32 && p->dtype != DCN_BF16) return fail(DCN_ERR_UNSUPPORTED, "unknown dtype %d", p->dtype);
+    if (p->H > (1 << 19) || p->W > (1 << 19) || p->K > 64 || p->pad > (1 << 19) || p->dil > (1 << 16) ||
+        p->stride > (1 << 16))
+        return fail(DCN_ERR_UNSUPPORTED, "H, W, pad up to 2^19, K up to 64, stride and dil up to 2^16");
+    long long Ho = ((long long)p->H + 2LL * p->pad - (long long)p->dil * (p->K - 1) - 1) / p->stride + 1;
+    long long Wo = ((long long)p->W + 2LL * p->pad - (long long)p->dil * (p->K - 1) - 1) / p->stride + 1;
+    if ((long long)p->H + 2LL * p->pad - (long long)p->dil * (p->K - 1) - 1 < 0 ||
+        (long long)p->W + 2LL * p->pad - (long long)p->dil * (p->K - 1) - 1 < 0 || Ho < 1 || Wo < 1)
+        return fail(DCN_ERR_INVALID_ARG, "output would be empty: the dilated kernel does not fit the padded input");
+    long long K2 = (long long)p->K * p->K;
+    long long P = (long long)p->B * Ho * Wo;
+    long long nx = (long long)p->B * p->H * p->W * p->Cin;
+    long long noff = P * 2 * p->G * K2;
+    long long ny = P * p->Cout;
+    long long nw = (long long)p->Cout * K2 * p->Cin;
+    if (nx > kMaxElems || noff > kMaxElems || ny > kMaxElems || nw > kMaxElems)
+        return fail(DCN_ERR_UNSUPPORTED, "a tensor exceeds 2^31-1 elements");
+    s.B = p->B;
+    s.H = p->H;
+    s.W = p->W;
+    s.Cin = p->Cin;
+    s.Cout = p->Cout;
+    s.K = p->K;
+    s.stride = p->stride;
+    s.pad = p->pad;
+    s.dil = p->dil;
+    s.G = p->G;
+    s.Ho = (int)Ho;
+    s.Wo = (int)Wo;
+    s.K2 = (int)K2;
+    s.Cg = p->Cin / p->G;
+    s.P = (int)P;
+    s.KC = (int)(K2 * p->Cin);
+    return DCN_OK;
+}
+
+size_t elem_size(int dtype) { return dtype == DCN_F32 ? 4 : 2; }
+
+int check_ptr(const void* ptr, const char* name, size_t align, bool required) {
+    if (!ptr) return required ? fail(DCN_ERR_INVALID_ARG, "%s is NULL", name) : DCN_OK;
+    if ((uintptr_t)ptr % align)
+        return fail(DCN_ERR_UNSUPPORTED, "%s is not aligned to %zu bytes", name, align);
+    return DCN_OK;
+}
+
+#define TRY(expr)                    \
+    do {                             \
+        int _rc = (expr);            \
+        if (_rc != DCN_OK) return _rc; \
+    } while (0)
+
+}  // namespace
+
+extern "C" {
+
+int dcn_abi_version(void) { return DCN_ABI_VERSION; }
+
+int dcn_output_size(const dcn_params_t* params, int* Ho, int* Wo) {
+    dcn::Shape s;
+    TRY(make_shape(params, s));
+    if (Ho) *Ho = s.Ho;
+    if (Wo) *Wo = s.Wo;
+    return ok();
+}
+
+size_t dcn_workspace_size(const dcn_params_t* params, int op) {
+    dcn::Shape s;
+    std::string keep = g_err;
+    if (make_shape(params, s) != DCN_OK) {
+        g_err = keep;
+        return 0;
+    }
+    (void)op;
+    return 0;
+}
+
+const char* dcn_forward_path(const dcn_params_t* params) {
+    dcn::Shape s;
+    std::string keep = g_err;
+    if (make_shape(params, s) != DCN_OK) {
+        g_err = keep;
+        return "invalid";
+    }
+    return "generic";
+}
+
+int dcn_forward(const dcn_params_t* params, const void* x, const void* offset, const void* mask, const void* weight,
+                const void* bias, void* y, void* workspace, size_t workspace_bytes, void* stream) {
+    dcn::Shape s;
+    TRY(make_shape(params, s));
+    size_t es = elem_size(params->dtype);
+    TRY(check_ptr(x, "x", es, true));
+    TRY(check_ptr(offset, "offset", es, true));
+    TRY(check_ptr(mask, "mask", es, false));
+    TRY(check_ptr(weight, "weight", es, true));
+    TRY(check_ptr(bias, "bias", es, false));
+    TRY(check_ptr(y, "y", es, true));
+    (void)workspace;
+    (void)workspace_bytes;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = dcn::generic_forward(s, params->dtype, x, offset, mask, weight, bias, y, st);
+    g_launches += 1;
+    if (e != cudaSuccess) return cuda_fail(e, "forward launch");
+    return ok();
+}
+
+int dcn_backward_data(const dcn_params_t* params, const void* x, const void* offset, const void* mask,
+                      const void* weight, const void* grad_y, float* grad_x, float* grad_offset, float* grad_mask,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+    dcn::Shape s;
+    TRY(make_shape(params, s));
+    size_t es = elem_size(params->dtype);
+    TRY(check_ptr(x, "x", es, true));
+    TRY(check_ptr(offset, "offset", es, true));
+    TRY(check_ptr(mask, "mask", es, false));
+    TRY(check_ptr(weight, "weight", es, true));
+    TRY(check_ptr(grad_y, "grad_y", es, true));
+    TRY(check_ptr(grad_x, "grad_x", 4, false));
+    TRY(check_ptr(grad_offset, "grad_offset", 4, false));
+    TRY(check_ptr(grad_mask, "grad_mask", 4, false));
+    if (grad_mask && !mask) return fail(DCN_ERR_INVALID_ARG, "grad_mask requested but mask is NULL");
+    (void)workspace;
+    (void)workspace_bytes;
+    if (!grad_x && !grad_offset && !grad_mask) return ok();
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e;
+    if (grad_x) {
+        e = cudaMemsetAsync(grad_x, 0, sizeof(float) * (size_t)s.B * s.H * s.W * s.Cin, st);
+        g_launches += 1;
+        if (e != cudaSuccess) return cuda_fail(e, "zeroing grad_x");
+    }
+    e = dcn::generic_backward_data(s, params->dtype, x, offset, mask, weight, grad_y, grad_x, grad_offset, grad_mask,
+                                   st);
+    g_launches += 1;
+    if (e != cudaSuccess) return cuda_fail(e, "backward-data launch");
+    return ok();
+}
+
+int dcn_backward_input(const dcn_params_t* params, const void* x, const void* offset, const void* mask,
+                       const void* weight, const void* grad_y, float* grad_x, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+    if (!grad_x) return fail(DCN_ERR_INVALID_ARG, "grad_x is NULL");
+    return dcn_backward_data(params, x, offset, mask, weight, grad_y, grad_x, nullptr, nullptr, workspace,
+                             workspace_bytes, stream);
+}
+
+int dcn_backward_offset_mask(const dcn_params_t* params, const void* x, const void* offset, const void* mask,
+                             const void* weight, const void* grad_y, float* grad_offset, float* grad_mask,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+    if (!grad_offset) return fail(DCN_ERR_INVALID_ARG, "grad_offset is NULL");
+    return dcn_backward_data(params, x, offset, mask, weight, grad_y, nullptr, grad_offset, grad_mask, workspace,
+                             workspace_bytes, stream);
+}
+
+int dcn_backward_weight(const dcn_params_t* params, const void* x, const void* offset, const void* mask,
+                        const void* grad_y, float* grad_weight, float* grad_bias, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+    dcn::Shape s;
+    TRY(make_shape(params, s));
+    size_t es = elem_size(params->dtype);
+    TRY(check_ptr(x, "x", es, true));
+    TRY(check_ptr(offset, "offset", es, true));
+    TRY(check_ptr(mask, "mask", es, false));
+    TRY(check_ptr(grad_y, "grad_y", es, true));
+    TRY(check_ptr(grad_weight, "grad_weight", 4, true));
+    TRY(check_ptr(grad_bias, "grad_bias", 4, false));
+    (void)workspace;
+    (void)workspace_bytes;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cudaMemsetAsync(grad_weight, 0, sizeof(float) * (size_t)s.Cout * s.KC, st);
+    g_launches += 1;
+    if (e != cudaSuccess) return cuda_fail(e, "zeroing grad_weight");
+    e = dcn::generic_backward_weight(s, params->dtype, x, offset, mask, grad_y, grad_weight, st);
+    g_launches += 1;
+    if (e != cudaSuccess) return cuda_fail(e, "backward-weight launch");
+    if (grad_bias) {
+        e = cudaMemsetAsync(grad_bias, 0, sizeof(float) * (size_t)s.Cout, st);
+        g_launches += 1;
+        if (e != cudaSuccess) return cuda_fail(e, "zeroing grad_bias");
+        e = dcn::bias_grad(s, params->dtype, grad_y, grad_bias, st);
+        g_launches += 1;
+        if (e != cudaSuccess) return cuda_fail(e, "bias-gradient launch");
+    }
+    return ok();
+}
+
+const char* dcn_last_error_string(void) { return g_err.c_str(); }
+
+int dcn_check_status(void) {
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "synchronising before the status read");
+    unsigned int st = 0;
+    e = dcn::read_and_clear_status(&st);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+    if (st) return fail(DCN_ERR_TIMEOUT, "a kernel gave up a bounded wait (status 0x%x)", st);
+    return ok();
+}
+
+unsigned long long dcn_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

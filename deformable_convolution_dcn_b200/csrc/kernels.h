@@ -1,0 +1,25 @@
+// Internal launchers of libdcn_b200 (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "common.cuh"
+
+namespace dcn {
+
+// generic.cu — CUDA-core kernels for every shape; dtype 0 = float, 1 = bfloat16.
+cudaError_t generic_forward(const Shape& s, int dtype, const void* x, const void* off, const void* mask,
+                            const void* w, const void* bias, void* y, cudaStream_t st);
+cudaError_t generic_backward_data(const Shape& s, int dtype, const void* x, const void* off, const void* mask,
+                                  const void* w, const void* gy, float* gx, float* goff, float* gmask,
+                                  cudaStream_t st);
+cudaError_t generic_backward_weight(const Shape& s, int dtype, const void* x, const void* off, const void* mask,
+                                    const void* gy, float* gw, cudaStream_t st);
+cudaError_t bias_grad(const Shape& s, int dtype, const void* gy, float* gb, cudaStream_t st);
+
+// status.cu — the device status word that bounded waits report to.
+cudaError_t status_word_ptr(unsigned int** ptr);
+cudaError_t read_and_clear_status(unsigned int* out);
+
+}  // namespace dcn

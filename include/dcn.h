@@ -1,0 +1,168 @@
+/*
+ * dcn.h — C ABI of libdcn_b200, a CUDA library (sm_100a, NVIDIA B200) for the
+ * modulated deformable convolution (DCNv2) with torchvision deform_conv2d
+ * semantics.
+ *
+ * The operation ("Deformable ConvNets" notes, section "可变形卷积": the plain
+ * convolution y(p0) = sum_{p_n in R} w(p_n) x(p0 + p_n) and its deformable form
+ * with a learned offset dp_n per tap; DCNv2 section 3.2 adds a modulation
+ * scalar m_k per tap):
+ *
+ *   y[b,ho,wo,o] = bias[o] + sum_{g<G} sum_{i,j<K} m * sum_{c in group g}
+ *                  w[o,i,j,c] * bilinear(x[b,:,:,c], py, px)
+ *   k  = i*K + j
+ *   py = ho*stride - pad + i*dil + offset[b, g*2K^2 + 2k,     ho, wo]   (row,    "dy")
+ *   px = wo*stride - pad + j*dil + offset[b, g*2K^2 + 2k + 1, ho, wo]   (column, "dx")
+ *   m  = mask[b, g*K^2 + k, ho, wo]   (mask == NULL: m = 1, i.e. DCNv1)
+ *
+ * bilinear() weights the four integer neighbours of (py, px) by the areas of
+ * the opposite sub-rectangles (notes, "双线性插值" S1..S4); a neighbour outside
+ * [0,H) x [0,W) contributes zero (no clamping). Channels are split into G
+ * deformable groups of Cin/G channels sharing one offset field (notes,
+ * "Deformable Group"). Output size: Ho = (H + 2*pad - dil*(K-1) - 1)/stride + 1,
+ * likewise Wo.
+ *
+ * Layouts (row-major, innermost dimension last; every tensor dense):
+ *   x        [B, H, W, Cin]        channel-contiguous (NHWC)
+ *   offset   [B, 2*G*K*K, Ho, Wo]
+ *   mask     [B, G*K*K, Ho, Wo]
+ *   weight   [Cout, K, K, Cin]     i.e. [Cout, K*K*Cin], tap-major then channel
+ *   bias     [Cout]
+ *   y        [B, Ho, Wo, Cout]
+ *   grad_*   float32, laid out like the tensor they differentiate
+ *
+ * Element types: x, offset, mask, weight, bias, y and grad_y all have the type
+ * given by dcn_params_t.dtype (DCN_F32: float, DCN_BF16: bfloat16). Gradients
+ * are always float32. Arithmetic is float32 (coordinates, bilinear weights,
+ * accumulation); on the bfloat16 path the modulated samples are rounded to
+ * bfloat16 once, as tensor-core operands.
+ *
+ * Ownership and streams: every pointer except `params` is a DEVICE pointer
+ * owned by the caller. The library never allocates device memory and never
+ * synchronises: all work is enqueued on `stream` (a cudaStream_t; NULL is the
+ * legacy default stream) of the current device, and returns as soon as it is
+ * enqueued. Some calls need a caller-provided device workspace of
+ * dcn_workspace_size() bytes (may be NULL when that size is 0). Outputs are
+ * overwritten, never accumulated into.
+ *
+ * Errors: every entry point returns DCN_OK (0) or a negative code, and checks
+ * its arguments before enqueueing anything. dcn_last_error_string() gives the
+ * calling thread's last message. Device-side waits are bounded; a wait that
+ * runs out records DCN_ERR_TIMEOUT in a device status word that
+ * dcn_check_status() reads.
+ */
+#ifndef DCN_B200_H
+#define DCN_B200_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DCN_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define DCN_API __attribute__((visibility("default")))
+#else
+#define DCN_API
+#endif
+
+typedef enum {
+    DCN_F32 = 0,  /* float32 inputs and y */
+    DCN_BF16 = 1  /* bfloat16 inputs and y */
+} dcn_dtype_t;
+
+/* Status codes. */
+#define DCN_OK 0
+#define DCN_ERR_INVALID_ARG (-1) /* a size is non-positive, Cin % G != 0, Ho or Wo <= 0, a required pointer is NULL */
+#define DCN_ERR_UNSUPPORTED (-2) /* unknown dtype, pointer not aligned to its element size, size beyond int32 indexing */
+#define DCN_ERR_CUDA (-3)        /* a CUDA call or launch failed; the message names it */
+#define DCN_ERR_TIMEOUT (-4)     /* a bounded device wait ran out (reported by dcn_check_status) */
+#define DCN_ERR_WORKSPACE (-5)   /* workspace NULL or smaller than dcn_workspace_size() */
+
+/* dcn_params_t.flags */
+#define DCN_FLAG_GENERIC 0x1u    /* use the generic CUDA-core kernels even where a specialised kernel exists */
+
+typedef struct dcn_params {
+    int B, H, W;     /* batch, input height and width */
+    int Cin, Cout;   /* input / output channels; Cin % G == 0 */
+    int K;           /* square kernel size */
+    int stride, pad, dil;
+    int G;           /* deformable groups */
+    int dtype;       /* dcn_dtype_t */
+    unsigned flags;  /* DCN_FLAG_* */
+} dcn_params_t;
+
+/* Operation selectors for dcn_workspace_size(). */
+#define DCN_OP_FORWARD 0
+#define DCN_OP_BACKWARD_DATA 1   /* dcn_backward_data, dcn_backward_input, dcn_backward_offset_mask */
+#define DCN_OP_BACKWARD_WEIGHT 2
+
+/* Library ABI version (DCN_ABI_VERSION). */
+DCN_API int dcn_abi_version(void);
+
+/* Output size of the layer (the standard convolution formula above).
+ * Returns DCN_ERR_INVALID_ARG when a size is invalid or Ho/Wo would be <= 0. */
+DCN_API int dcn_output_size(const dcn_params_t* params, int* Ho, int* Wo);
+
+/* Bytes of device workspace that the operation `op` (DCN_OP_*) needs for these
+ * params; 0 when none. Returns 0 for invalid params as well (the call itself
+ * then reports the error). */
+DCN_API size_t dcn_workspace_size(const dcn_params_t* params, int op);
+
+/* Forward pass: y = DCNv2(x, offset, mask, weight, bias).
+ * mask and bias may be NULL. Writes y. */
+DCN_API int dcn_forward(const dcn_params_t* params, const void* x, const void* offset, const void* mask,
+                const void* weight, const void* bias, void* y, void* workspace, size_t workspace_bytes,
+                void* stream);
+
+/* Data-side backward in one pass: the gradients with respect to the input, the
+ * offsets and the mask, given grad_y = dL/dy. Any of grad_x, grad_offset,
+ * grad_mask may be NULL (not computed); grad_mask must be NULL when mask is
+ * NULL. The offset gradient is taken through floor(): at an exact integer
+ * sampling coordinate it is the right-hand derivative (the pages note the
+ * bilinear kink there: the torchvision tutorial, section 3.2). */
+DCN_API int dcn_backward_data(const dcn_params_t* params, const void* x, const void* offset, const void* mask,
+                      const void* weight, const void* grad_y, float* grad_x, float* grad_offset, float* grad_mask,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* grad_x only (dcn_backward_data with grad_offset = grad_mask = NULL). */
+DCN_API int dcn_backward_input(const dcn_params_t* params, const void* x, const void* offset, const void* mask,
+                       const void* weight, const void* grad_y, float* grad_x, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/* grad_offset and grad_mask (dcn_backward_data with grad_x = NULL). grad_mask may
+ * be NULL; it must be NULL when mask is NULL. */
+DCN_API int dcn_backward_offset_mask(const dcn_params_t* params, const void* x, const void* offset, const void* mask,
+                             const void* weight, const void* grad_y, float* grad_offset, float* grad_mask,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Weight-side backward: grad_weight [Cout, K, K, Cin] = sum over output pixels of
+ * grad_y[p, o] * m * bilinear sample, and grad_bias [Cout] = sum_p grad_y[p, o]
+ * (grad_bias may be NULL). */
+DCN_API int dcn_backward_weight(const dcn_params_t* params, const void* x, const void* offset, const void* mask,
+                        const void* grad_y, float* grad_weight, float* grad_bias, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/* The calling thread's last error message ("" after success). */
+DCN_API const char* dcn_last_error_string(void);
+
+/* Reads and clears the device status word of the current device (synchronises
+ * the device). Returns DCN_OK, or DCN_ERR_TIMEOUT if a kernel gave up a bounded
+ * wait since the last check. */
+DCN_API int dcn_check_status(void);
+
+/* Number of kernels (and memsets) this library has enqueued since the process
+ * started, summed over threads. */
+DCN_API unsigned long long dcn_launch_count(void);
+
+/* Name of the kernel path the forward would take for these params (static
+ * string), e.g. "tcgen05_gather" or "generic"; "invalid" for bad params. */
+DCN_API const char* dcn_forward_path(const dcn_params_t* params);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DCN_B200_H */

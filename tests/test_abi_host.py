@@ -1,0 +1,95 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point that include/dcn.h declares, and rejects bad arguments with
+the documented codes before anything reaches the device. No call here passes
+valid device pointers, so nothing is launched."""
+import ctypes
+
+import pytest
+
+import deformable_convolution_dcn_b200 as dcn
+
+OK, EINVAL, EUNSUP, ECUDA, ETIMEOUT, EWS = 0, -1, -2, -3, -4, -5
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from deformable_convolution_dcn_b200 import build
+    build.build()
+    return dcn._load()
+
+
+def P(**kw):
+    d = dict(B=2, H=9, W=8, Cin=8, Cout=4, K=3, stride=1, pad=1, dil=1, G=2, dtype=0, flags=0)
+    d.update(kw)
+    return dcn.make_params(**d)
+
+
+def test_exports_every_header_symbol(lib):
+    names = dcn.header_symbols()
+    assert {"dcn_forward", "dcn_backward_input", "dcn_backward_weight", "dcn_backward_offset_mask",
+            "dcn_backward_data", "dcn_workspace_size", "dcn_last_error_string"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert lib.dcn_abi_version() == 1
+
+
+@pytest.mark.parametrize("H,W,K,stride,pad,dil,expect", [
+    (224, 224, 3, 1, 1, 1, (224, 224)), (200, 200, 3, 2, 1, 1, (100, 100)), (25, 25, 3, 1, 2, 2, (25, 25)),
+    (50, 50, 3, 1, 1, 1, (50, 50)), (7, 5, 5, 2, 0, 1, (2, 1)), (1, 1, 3, 1, 1, 1, (1, 1)), (6, 6, 2, 1, 0, 1, (5, 5)),
+])
+def test_output_size(lib, H, W, K, stride, pad, dil, expect):
+    assert dcn.output_size(P(H=H, W=W, K=K, stride=stride, pad=pad, dil=dil)) == expect
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(B=0), EINVAL), (dict(H=-1), EINVAL), (dict(Cin=7, G=2), EINVAL), (dict(K=0), EINVAL),
+    (dict(stride=0), EINVAL), (dict(pad=-1), EINVAL), (dict(dil=0), EINVAL), (dict(G=0), EINVAL),
+    (dict(H=2, W=2, K=5, pad=0), EINVAL), (dict(dtype=7), EUNSUP),
+    (dict(B=4096, H=1024, W=1024, Cin=8), EUNSUP),
+])
+def test_invalid_params_rejected(lib, bad, code):
+    p = P(**bad)
+    ho, wo = ctypes.c_int(), ctypes.c_int()
+    assert lib.dcn_output_size(ctypes.byref(p), ctypes.byref(ho), ctypes.byref(wo)) == code
+    assert lib.dcn_last_error_string().decode() != ""
+    fake = ctypes.c_void_p(1 << 20)
+    rc = lib.dcn_forward(ctypes.byref(p), fake, fake, None, fake, None, fake, None, 0, None)
+    assert rc == code
+    assert lib.dcn_workspace_size(ctypes.byref(p), 0) == 0
+    assert dcn.forward_path(p) == "invalid"
+
+
+def test_null_required_pointers(lib):
+    p = P()
+    f = ctypes.c_void_p(1 << 20)
+    assert lib.dcn_forward(ctypes.byref(p), None, f, None, f, None, f, None, 0, None) == EINVAL
+    assert "x is NULL" in lib.dcn_last_error_string().decode()
+    assert lib.dcn_forward(ctypes.byref(p), f, None, None, f, None, f, None, 0, None) == EINVAL
+    assert lib.dcn_forward(ctypes.byref(p), f, f, None, None, None, f, None, 0, None) == EINVAL
+    assert lib.dcn_forward(ctypes.byref(p), f, f, None, f, None, None, None, 0, None) == EINVAL
+    assert lib.dcn_backward_input(ctypes.byref(p), f, f, None, f, f, None, None, 0, None) == EINVAL
+    assert lib.dcn_backward_offset_mask(ctypes.byref(p), f, f, None, f, f, None, None, None, 0, None) == EINVAL
+    assert lib.dcn_backward_weight(ctypes.byref(p), f, f, None, f, None, None, None, 0, None) == EINVAL
+    # grad_mask without a mask
+    assert lib.dcn_backward_data(ctypes.byref(p), f, f, None, f, f, None, None, f, None, 0, None) == EINVAL
+    assert lib.dcn_forward(None, f, f, None, f, None, f, None, 0, None) == EINVAL
+
+
+def test_misaligned_pointers(lib):
+    f = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 2)
+    p32 = P(dtype=0)
+    assert lib.dcn_forward(ctypes.byref(p32), odd, f, None, f, None, f, None, 0, None) == EUNSUP
+    assert "aligned" in lib.dcn_last_error_string().decode()
+    one = ctypes.c_void_p((1 << 20) + 1)
+    p16 = P(dtype=1)
+    assert lib.dcn_forward(ctypes.byref(p16), f, f, one, f, None, f, None, 0, None) == EUNSUP
+    assert lib.dcn_backward_weight(ctypes.byref(p16), f, f, None, f, odd, None, None, 0, None) == EUNSUP
+
+
+def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    import importlib
+    monkeypatch.setattr(dcn, "_lib", None)
+    monkeypatch.setattr(dcn, "_LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        dcn._load()
