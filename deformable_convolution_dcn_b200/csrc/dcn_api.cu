@@ -92,6 +92,15 @@ int check_ptr(const void* ptr, const char* name, size_t align, bool required) {
     return DCN_OK;
 }
 
+bool aligned16(const void* p) { return p == nullptr || ((uintptr_t)p & 15) == 0; }
+
+// The tensor-core forward takes bfloat16 layers whose channel counts are
+// multiples of 8 (16-byte vectors) and at most 25 taps; pointers are checked
+// separately at the call.
+bool use_fwd_tc(const dcn_params_t* p, const dcn::Shape& s) {
+    return p->dtype == DCN_BF16 && !(p->flags & DCN_FLAG_GENERIC) && dcn::fwd_tc_supported(s);
+}
+
 #define TRY(expr)                    \
     do {                             \
         int _rc = (expr);            \
@@ -119,7 +128,7 @@ size_t dcn_workspace_size(const dcn_params_t* params, int op) {
         g_err = keep;
         return 0;
     }
-    (void)op;
+    if (op == DCN_OP_FORWARD && use_fwd_tc(params, s)) return dcn::fwd_tc_workspace(s);
     return 0;
 }
 
@@ -130,7 +139,7 @@ const char* dcn_forward_path(const dcn_params_t* params) {
         g_err = keep;
         return "invalid";
     }
-    return "generic";
+    return use_fwd_tc(params, s) ? "tcgen05_gather" : "generic";
 }
 
 int dcn_forward(const dcn_params_t* params, const void* x, const void* offset, const void* mask, const void* weight,
@@ -144,9 +153,21 @@ int dcn_forward(const dcn_params_t* params, const void* x, const void* offset, c
     TRY(check_ptr(weight, "weight", es, true));
     TRY(check_ptr(bias, "bias", es, false));
     TRY(check_ptr(y, "y", es, true));
-    (void)workspace;
-    (void)workspace_bytes;
     cudaStream_t st = (cudaStream_t)stream;
+    if (use_fwd_tc(params, s) && aligned16(x) && aligned16(weight) && aligned16(y)) {
+        size_t need = dcn::fwd_tc_workspace(s);
+        if (!workspace || workspace_bytes < need)
+            return fail(DCN_ERR_WORKSPACE, "forward needs %zu bytes of workspace, got %zu", need,
+                        workspace ? workspace_bytes : (size_t)0);
+        unsigned* status = nullptr;
+        cudaError_t e = dcn::status_word_ptr(&status);
+        if (e != cudaSuccess) return cuda_fail(e, "status word");
+        int n = 0;
+        e = dcn::fwd_tc(s, x, offset, mask, weight, bias, y, workspace, workspace_bytes, status, st, &n);
+        g_launches += n;
+        if (e != cudaSuccess) return cuda_fail(e, "tensor-core forward launch");
+        return ok();
+    }
     cudaError_t e = dcn::generic_forward(s, params->dtype, x, offset, mask, weight, bias, y, st);
     g_launches += 1;
     if (e != cudaSuccess) return cuda_fail(e, "forward launch");

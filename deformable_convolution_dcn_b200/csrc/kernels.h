@@ -18,6 +18,12 @@ cudaError_t generic_backward_weight(const Shape& s, int dtype, const void* x, co
                                     const void* gy, float* gw, cudaStream_t st);
 cudaError_t bias_grad(const Shape& s, int dtype, const void* gy, float* gb, cudaStream_t st);
 
+// fwd_tc.cu — bfloat16 forward on tcgen05 tensor cores with the fused deformable gather.
+bool fwd_tc_supported(const Shape& s);
+size_t fwd_tc_workspace(const Shape& s);
+cudaError_t fwd_tc(const Shape& s, const void* x, const void* off, const void* mask, const void* w, const void* bias,
+                   void* y, void* ws, size_t ws_bytes, unsigned* status, cudaStream_t st, int* launches);
+
 // status.cu — the device status word that bounded waits report to.
 cudaError_t status_word_ptr(unsigned int** ptr);
 cudaError_t read_and_clear_status(unsigned int* out);
