@@ -34,8 +34,8 @@ def _headers():
         glob.glob(os.path.join(INCLUDE, "*.h"))
 
 
-def _compile(src: str, force: bool, verbose: bool, extra=()) -> str:
-    obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+def _compile(src: str, force: bool, verbose: bool, extra=(), build_dir=BUILD) -> str:
+    obj = os.path.join(build_dir, os.path.basename(src) + ".o")
     newest = max([os.path.getmtime(src)] + [os.path.getmtime(h) for h in _headers()])
     if not force and os.path.exists(obj) and os.path.getmtime(obj) >= newest:
         return obj
@@ -50,24 +50,31 @@ def _compile(src: str, force: bool, verbose: bool, extra=()) -> str:
     return obj
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False) -> str:
-    """Compile every CUDA source for sm_100a and link libdcn_b200.so; returns its path."""
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False, defines=(), out: str = LIB,
+          build_dir: str = BUILD) -> str:
+    """Compile every CUDA source for sm_100a and link libdcn_b200.so; returns its path.
+
+    ``defines`` (e.g. ["DCN_FWD_MAX_STAGES=3"]) override compile-time tuning
+    constants; use them with a separate ``out`` and ``build_dir``.
+    """
+    os.makedirs(build_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
-    extra = ["-Xptxas", "-v"] if ptxas_verbose else []
+    extra = (["-Xptxas", "-v"] if ptxas_verbose else []) + ["-D" + d for d in defines]
     with concurrent.futures.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        objs = list(ex.map(lambda s: _compile(s, force or ptxas_verbose, verbose or ptxas_verbose, extra), srcs))
+        objs = list(ex.map(lambda s: _compile(s, force or ptxas_verbose, verbose or ptxas_verbose, extra, build_dir),
+                           srcs))
     newest_obj = max(os.path.getmtime(o) for o in objs)
-    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < newest_obj:
-        tmp = LIB + ".tmp%d" % os.getpid()
+    LIBOUT = out
+    if force or not os.path.exists(LIBOUT) or os.path.getmtime(LIBOUT) < newest_obj:
+        tmp = LIBOUT + ".tmp%d" % os.getpid()
         cmd = [NVCC, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
         if verbose:
             print(" ".join(cmd), flush=True)
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError("link failed:\n%s%s" % (r.stdout, r.stderr))
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, LIBOUT)
+    return LIBOUT
 
 
 if __name__ == "__main__":

@@ -181,6 +181,41 @@ __device__ __forceinline__ uint4 ldg_v4(const void* p) {
     return v;
 }
 
+// Four predicated 16-byte read-only loads issued back to back (a disabled load
+// leaves zeros). Volatile so that every row's loads are in flight before the
+// first of them is consumed.
+__device__ __forceinline__ void ldg4_pred(uint4 (&v)[4], const void* p0, const void* p1, const void* p2,
+                                          const void* p3, uint32_t mask) {
+    asm volatile(
+        "{\n\t.reg .pred q0, q1, q2, q3;\n\t.reg .b32 t;\n\t"
+        "and.b32 t, %16, 1;\n\tsetp.ne.b32 q0, t, 0;\n\t"
+        "and.b32 t, %16, 2;\n\tsetp.ne.b32 q1, t, 0;\n\t"
+        "and.b32 t, %16, 4;\n\tsetp.ne.b32 q2, t, 0;\n\t"
+        "and.b32 t, %16, 8;\n\tsetp.ne.b32 q3, t, 0;\n\t"
+        "mov.b32 %0, 0;\n\tmov.b32 %1, 0;\n\tmov.b32 %2, 0;\n\tmov.b32 %3, 0;\n\t"
+        "mov.b32 %4, 0;\n\tmov.b32 %5, 0;\n\tmov.b32 %6, 0;\n\tmov.b32 %7, 0;\n\t"
+        "mov.b32 %8, 0;\n\tmov.b32 %9, 0;\n\tmov.b32 %10, 0;\n\tmov.b32 %11, 0;\n\t"
+        "mov.b32 %12, 0;\n\tmov.b32 %13, 0;\n\tmov.b32 %14, 0;\n\tmov.b32 %15, 0;\n\t"
+        "@q0 ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%17];\n\t"
+        "@q1 ld.global.nc.v4.u32 {%4, %5, %6, %7}, [%18];\n\t"
+        "@q2 ld.global.nc.v4.u32 {%8, %9, %10, %11}, [%19];\n\t"
+        "@q3 ld.global.nc.v4.u32 {%12, %13, %14, %15}, [%20];\n\t}"
+        : "=&r"(v[0].x), "=&r"(v[0].y), "=&r"(v[0].z), "=&r"(v[0].w), "=&r"(v[1].x), "=&r"(v[1].y), "=&r"(v[1].z),
+          "=&r"(v[1].w), "=&r"(v[2].x), "=&r"(v[2].y), "=&r"(v[2].z), "=&r"(v[2].w), "=&r"(v[3].x), "=&r"(v[3].y),
+          "=&r"(v[3].z), "=&r"(v[3].w)
+        : "r"(mask), "l"(p0), "l"(p1), "l"(p2), "l"(p3));
+}
+
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+    asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ float4 ldcg_f4(const float* p) {
     float4 v;
     asm volatile("ld.global.cg.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(p));
