@@ -101,6 +101,11 @@ bool use_fwd_tc(const dcn_params_t* p, const dcn::Shape& s) {
     return p->dtype == DCN_BF16 && !(p->flags & DCN_FLAG_GENERIC) && dcn::fwd_tc_supported(s);
 }
 
+// The small-channel float32 forward: Cin <= 8, Cout a multiple of 32.
+bool use_fwd_small(const dcn_params_t* p, const dcn::Shape& s) {
+    return p->dtype == DCN_F32 && !(p->flags & DCN_FLAG_GENERIC) && dcn::fwd_f32_small_supported(s);
+}
+
 #define TRY(expr)                    \
     do {                             \
         int _rc = (expr);            \
@@ -139,7 +144,9 @@ const char* dcn_forward_path(const dcn_params_t* params) {
         g_err = keep;
         return "invalid";
     }
-    return use_fwd_tc(params, s) ? "tcgen05_gather" : "generic";
+    if (use_fwd_tc(params, s)) return "tcgen05_gather";
+    if (use_fwd_small(params, s)) return "f32_small_channels";
+    return "generic";
 }
 
 int dcn_forward(const dcn_params_t* params, const void* x, const void* offset, const void* mask, const void* weight,
@@ -166,6 +173,12 @@ int dcn_forward(const dcn_params_t* params, const void* x, const void* offset, c
         e = dcn::fwd_tc(s, x, offset, mask, weight, bias, y, workspace, workspace_bytes, status, st, &n);
         g_launches += n;
         if (e != cudaSuccess) return cuda_fail(e, "tensor-core forward launch");
+        return ok();
+    }
+    if (use_fwd_small(params, s) && aligned16(y)) {
+        cudaError_t e = dcn::fwd_f32_small(s, x, offset, mask, weight, bias, y, st);
+        g_launches += 1;
+        if (e != cudaSuccess) return cuda_fail(e, "small-channel forward launch");
         return ok();
     }
     cudaError_t e = dcn::generic_forward(s, params->dtype, x, offset, mask, weight, bias, y, st);

@@ -208,3 +208,21 @@ def test_full_size_backward_sampled():
     for gname, prim in (("grad_x", "x"), ("grad_weight", "weight"), ("grad_mask", "mask")):
         rhs = float((g[gname].double() * dd[prim].double()).sum())
         assert abs(lhs - rhs) <= 2e-2 * abs(lhs), (gname, lhs, rhs)
+
+
+@pytest.mark.parametrize("shape", [
+    gen.LayerShape(B=1, Cin=3, H=23, W=19, Cout=64, K=3, stride=1, pad=1),
+    gen.LayerShape(B=2, Cin=1, H=9, W=12, Cout=32, K=5, stride=2, pad=2),
+    gen.LayerShape(B=1, Cin=8, H=10, W=7, Cout=128, K=3, stride=1, pad=2, dil=2, G=2),
+    gen.LayerShape(B=2, Cin=2, H=6, W=9, Cout=16, K=3, stride=1, pad=1, G=2),
+    gen.LayerShape(B=3, Cin=6, H=8, W=8, Cout=128, K=1, stride=1, pad=0, G=3),
+    gen.LayerShape(B=1, Cin=4, H=31, W=17, Cout=64, K=3, stride=2, pad=0),
+], ids=lambda s: "C%dx%dK%ds%dd%dG%d" % (s.Cin, s.Cout, s.K, s.stride, s.dil, s.G))
+def test_small_channel_f32_layers(shape):
+    """Float32 layers with few input channels (the stem-style kernel), compared in full."""
+    w = gen.Workload("smallc", shape, "f32", seed=9, offset_dist="normal1.5_edges", bias=True)
+    d = gen.make_inputs(w)
+    p = dcn._params(d["x"], d["weight"], d["offset"], shape.stride, shape.pad, shape.dil, False)
+    assert dcn.forward_path(p) == "f32_small_channels"
+    y = run_forward(shape, to_dev(d))
+    assert_close(_cpu(y), _oracle_forward(shape, f64(d)), "f32", "y")
