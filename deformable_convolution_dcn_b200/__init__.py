@@ -23,7 +23,7 @@ import threading
 import torch
 
 __all__ = [
-    "forward", "backward_data", "backward_input", "backward_offset_mask", "backward_weight", "output_size",
+    "forward", "forward_noalloc", "backward_data", "backward_input", "backward_offset_mask", "backward_weight", "output_size",
     "workspace_size", "forward_path", "check_status", "launch_count", "library_path", "DeformConv2dFunction",
     "deform_conv2d", "DcnError",
 ]
@@ -71,6 +71,7 @@ def _load():
         lib.dcn_workspace_size.argtypes = [P, ctypes.c_int]
         lib.dcn_workspace_size.restype = sz
         lib.dcn_forward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.dcn_forward_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
         lib.dcn_backward_data.argtypes = [P, vp, vp, vp, vp, vp, fp, fp, fp, vp, sz, vp]
         lib.dcn_backward_input.argtypes = [P, vp, vp, vp, vp, vp, fp, vp, sz, vp]
         lib.dcn_backward_offset_mask.argtypes = [P, vp, vp, vp, vp, vp, fp, fp, vp, sz, vp]
@@ -177,6 +178,19 @@ def forward(x, offset, mask, weight, bias=None, stride=1, padding=0, dilation=1,
     ws, nws = _workspace(p, OP_FORWARD, x.device, workspace)
     _check(lib.dcn_forward(ctypes.byref(p), _ptr(x), _ptr(offset), _ptr(mask), _ptr(weight), _ptr(bias), _ptr(out),
                            _ptr(ws), nws, _stream(x.device)))
+    return out
+
+
+def forward_noalloc(x, offset, mask, weight, bias=None, stride=1, padding=0, dilation=1, *, out=None):
+    """Forward through dcn_forward_noalloc: no workspace, scratch in the library's static device array."""
+    lib = _load()
+    p = _params(x, weight, offset, stride, padding, dilation, False)
+    _check_tensors(x.dtype, x.device, x=x, offset=offset, mask=mask, weight=weight, bias=bias, out=out)
+    Ho, Wo = output_size(p)
+    if out is None:
+        out = torch.empty((p.B, Ho, Wo, p.Cout), dtype=x.dtype, device=x.device)
+    _check(lib.dcn_forward_noalloc(ctypes.byref(p), _ptr(x), _ptr(offset), _ptr(mask), _ptr(weight), _ptr(bias),
+                                   _ptr(out), _stream(x.device)))
     return out
 
 

@@ -187,6 +187,36 @@ int dcn_forward(const dcn_params_t* params, const void* x, const void* offset, c
     return ok();
 }
 
+int dcn_forward_noalloc(const dcn_params_t* params, const void* x, const void* offset, const void* mask,
+                        const void* weight, const void* bias, void* y, void* stream) {
+    dcn::Shape s;
+    TRY(make_shape(params, s));
+    size_t es = elem_size(params->dtype);
+    TRY(check_ptr(x, "x", es, true));
+    TRY(check_ptr(offset, "offset", es, true));
+    TRY(check_ptr(mask, "mask", es, false));
+    TRY(check_ptr(weight, "weight", es, true));
+    TRY(check_ptr(bias, "bias", es, false));
+    TRY(check_ptr(y, "y", es, true));
+    if (use_fwd_tc(params, s) && aligned16(x) && aligned16(weight) && aligned16(y)) {
+        const size_t need = dcn::fwd_tc_workspace(s), have = dcn::fwd_tc_static_scratch_bytes();
+        if (need > have)
+            return fail(DCN_ERR_WORKSPACE,
+                        "forward without allocation needs %zu bytes of scratch; the static array holds %zu", need,
+                        have);
+        unsigned* status = nullptr;
+        cudaError_t e = dcn::status_word_ptr(&status);
+        if (e != cudaSuccess) return cuda_fail(e, "status word");
+        int n = 0;
+        e = dcn::fwd_tc_noalloc(s, x, offset, mask, weight, bias, y, status, (cudaStream_t)stream, &n);
+        g_launches += n;
+        if (e != cudaSuccess) return cuda_fail(e, "tensor-core forward (static scratch) launch");
+        return ok();
+    }
+    // every other forward kernel needs no scratch
+    return dcn_forward(params, x, offset, mask, weight, bias, y, nullptr, 0, stream);
+}
+
 int dcn_backward_data(const dcn_params_t* params, const void* x, const void* offset, const void* mask,
                       const void* weight, const void* grad_y, float* grad_x, float* grad_offset, float* grad_mask,
                       void* workspace, size_t workspace_bytes, void* stream) {

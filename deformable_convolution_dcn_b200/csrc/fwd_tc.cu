@@ -868,4 +868,50 @@ cudaError_t fwd_tc(const Shape& s, const void* x, const void* off, const void* m
     return cudaGetLastError();
 }
 
+
+// ------------------------------------------------- forward without allocation --
+// Scratch for callers that cannot allocate device memory themselves (see
+// dcn_forward_noalloc in include/dcn.h). The array lives in this module's
+// device image, so every GPU that loads the library holds it until the
+// process exits; all calls share it.
+namespace {
+
+constexpr size_t kStaticScratchBytes = 40ull << 20;  // 40 MiB
+static __device__ __align__(256) unsigned char g_fwd_scratch[kStaticScratchBytes];
+
+// Device address of g_fwd_scratch on the current device, looked up once per
+// device. In host code the symbol itself is only a host-side handle, never a
+// device address, so kernels must get this pointer instead.
+cudaError_t static_scratch_ptr(void** out) {
+    static void* cache[64] = {nullptr};
+    static std::mutex mu;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!cache[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_fwd_scratch);
+        if (e != cudaSuccess) return e;
+        cache[dev] = p;
+    }
+    *out = cache[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+size_t fwd_tc_static_scratch_bytes() { return kStaticScratchBytes; }
+
+cudaError_t fwd_tc_noalloc(const Shape& s, const void* x, const void* off, const void* mask, const void* w,
+                           const void* bias, void* y, unsigned* status, cudaStream_t st, int* launches) {
+    if (fwd_tc_workspace(s) > kStaticScratchBytes) return cudaErrorInvalidValue;
+    void* scratch = nullptr;
+    cudaError_t e = static_scratch_ptr(&scratch);
+    if (e != cudaSuccess) return e;
+    // fwd_tc clears the tile counters in the scratch before its kernel runs
+    return fwd_tc(s, x, off, mask, w, bias, y, scratch, kStaticScratchBytes, status, st, launches);
+}
+
 }  // namespace dcn

@@ -24,6 +24,11 @@ size_t fwd_tc_workspace(const Shape& s);
 cudaError_t fwd_tc(const Shape& s, const void* x, const void* off, const void* mask, const void* w, const void* bias,
                    void* y, void* ws, size_t ws_bytes, unsigned* status, cudaStream_t st, int* launches);
 
+// Same forward with its scratch in a static device array instead of a caller workspace.
+size_t fwd_tc_static_scratch_bytes();
+cudaError_t fwd_tc_noalloc(const Shape& s, const void* x, const void* off, const void* mask, const void* w,
+                           const void* bias, void* y, unsigned* status, cudaStream_t st, int* launches);
+
 // fwd_f32_small.cu — float32 forward for layers with Cin <= 8 (CUDA cores, HBM-bound).
 bool fwd_f32_small_supported(const Shape& s);
 cudaError_t fwd_f32_small(const Shape& s, const void* x, const void* off, const void* mask, const void* w,

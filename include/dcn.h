@@ -145,6 +145,27 @@ DCN_API int dcn_backward_weight(const dcn_params_t* params, const void* x, const
                         const void* grad_y, float* grad_weight, float* grad_bias, void* workspace,
                         size_t workspace_bytes, void* stream);
 
+/* Forward pass that allocates nothing and takes no workspace. The pages have
+ * no counterpart to this entry point; it exists for callers that cannot
+ * allocate device memory themselves: code whose device memory is owned by
+ * another allocator it cannot reach, and code that must not call cudaMalloc
+ * during steady-state work because cudaMalloc can synchronize the device.
+ *
+ * Same arguments, layouts and results as dcn_forward, without workspace. Where
+ * the forward needs scratch (the tensor-core path keeps float32 partial tiles
+ * and per-tile counters there), it uses one static device array of
+ * 40 MiB (41943040 bytes) compiled into the library; every GPU that loads the
+ * library holds that array until the process exits. Shapes whose scratch
+ * would exceed it are rejected with DCN_ERR_WORKSPACE and a message giving
+ * both sizes, before anything is enqueued. The tile counters are cleared on
+ * `stream` before each kernel runs. All calls on a device share the one
+ * array, so calls whose work can overlap on the GPU (different streams, or
+ * different host threads) race and may produce wrong results: issue them in
+ * one stream order. The first call on each device looks up the array's
+ * device address; make that first call before any stream capture. */
+DCN_API int dcn_forward_noalloc(const dcn_params_t* params, const void* x, const void* offset, const void* mask,
+                                const void* weight, const void* bias, void* y, void* stream);
+
 /* The calling thread's last error message ("" after success). */
 DCN_API const char* dcn_last_error_string(void);
 
