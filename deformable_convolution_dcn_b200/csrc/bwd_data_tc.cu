@@ -1,0 +1,461 @@
+// Data-side backward of DCNv2 on sm_100a tensor cores (bfloat16 in, float32
+// gradients): in one pass, grad_x, grad_offset and grad_mask.
+//
+// The column gradient G[p, (tap, c)] = sum_o grad_y[p, o] * w[o, tap, c] (the
+// transpose of the forward's contraction, the col2im side of the im2col view in
+// the "Deformable ConvNets" notes) is computed on tcgen05 tensor cores into TMEM,
+// 128 output pixels x 256 channels of one (group, tap) per unit, K = Cout:
+//   A = grad_y [P, Cout]                 TMA, 128-byte swizzle, K-major
+//   B = w^T [K*K*Cin, Cout] (transposed once per call into the workspace)
+// G never reaches HBM. Eight epilogue warps (two per TMEM lane quarter, each on
+// half of the 256 channels) read it back and, per pixel, tap and channel, load
+// the four bilinear neighbours of the sample and
+//   * scatter G * m * (neighbour weight) into grad_x with 16-byte vector atomics,
+//   * accumulate m * G * d(sample)/dy and d/dx (the offset gradient of the
+//     notes' gradient equation, taken through floor()) and G * sample (the mask
+//     gradient), added into grad_offset / grad_mask with one atomic per value.
+// grad_x, grad_offset and grad_mask are zeroed first. Units (pixel tile,
+// group-tap block) are split evenly over one CTA per SM; the TMEM accumulator
+// is double-buffered so the epilogue of one unit overlaps the MMAs of the next.
+// All waits are bounded.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "kernels.h"
+#include "tc_ptx.cuh"
+
+namespace dcn {
+namespace {
+
+constexpr int BM = 128;     // pixels per unit (UMMA M)
+constexpr int NT = 256;     // channels per unit (UMMA N)
+constexpr int BK = 64;      // output channels per K chunk
+constexpr int EPI_WARPS = 8;
+constexpr int TMA_WARP = 8, MMA_WARP = 9;
+constexpr int NUM_THREADS = 10 * 32;
+constexpr long long WAIT_LIMIT = 2000000000LL;
+constexpr int MAX_STAGES = 4;
+constexpr uint32_t A_BYTES = BM * BK * 2;   // 16 KB
+constexpr uint32_t B_BYTES = NT * BK * 2;   // 32 KB
+
+struct BdArgs {
+    Shape s;
+    const bf16* x;
+    const float4* rec;   // [G*K2][Ppad]: {ly, lx, m, ((y0+1) << 16) | (x0+1)} or yx = ~0 when all neighbours are outside
+    float* gx;
+    float* goff;
+    float* gmask;
+    unsigned* status;
+    int nblk, units_per_tile, m_tiles, ppad, ctas, stages, kchunks;
+    long long total_units;
+};
+
+__device__ __forceinline__ long long unit_begin(int c, const BdArgs& a) { return a.total_units * c / a.ctas; }
+
+__device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    dcn_bwd_data_tc_kernel(const __grid_constant__ CUtensorMap tmap_dy, const __grid_constant__ CUtensorMap tmap_wt,
+                           const BdArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Shape& s = a.s;
+    const uint32_t stage_bytes = A_BYTES + B_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + a.stages * stage_bytes);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + MAX_STAGES;
+    uint64_t* acc_full = bars + 2 * MAX_STAGES;
+    uint64_t* acc_empty = acc_full + 2;
+    uint64_t* drain = acc_empty + 2;
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < a.stages; ++i) {
+            ptx::mbar_init(ptx::smem_u32(&full[i]), 1);
+            ptx::mbar_init(ptx::smem_u32(&empty[i]), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(ptx::smem_u32(&acc_full[i]), 1);
+            ptx::mbar_init(ptx::smem_u32(&acc_empty[i]), EPI_WARPS);
+        }
+        ptx::mbar_init(ptx::smem_u32(drain), 1);
+        *s_abort = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == MMA_WARP) {
+        ptx::tmem_alloc(ptx::smem_u32(s_tmem), 512);
+        ptx::tmem_relinquish();
+    }
+    if (warp == TMA_WARP && lane == 0) {
+        ptx::prefetch_tmap(&tmap_dy);
+        ptx::prefetch_tmap(&tmap_wt);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = *s_tmem;
+    const long long ubeg = unit_begin(blockIdx.x, a), uend = unit_begin(blockIdx.x + 1, a);
+
+    if (warp == TMA_WARP) {
+        // ------------------------------------------------- grad_y and w^T --
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0, issued = 0, issued_par = 0;
+            bool ok = true;
+            for (long long u = ubeg; u < uend && ok; ++u) {
+                const int mt = (int)(u / a.units_per_tile), r = (int)(u - (long long)mt * a.units_per_tile);
+                const int gtap = r / a.nblk, cb = r - gtap * a.nblk;
+                const int g = gtap / s.K2, tap = gtap - g * s.K2;
+                const int row0 = tap * s.Cin + g * s.Cg + cb * NT;  // first w^T row (input channel) of the unit
+                for (int kc = 0; kc < a.kchunks; ++kc) {
+                    if (!ptx::mbar_wait(ptx::smem_u32(&empty[stage]), phase ^ 1, s_abort, a.status, WAIT_LIMIT)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* st = smem + stage * stage_bytes;
+                    const uint32_t fb = ptx::smem_u32(&full[stage]);
+                    ptx::mbar_arrive_expect_tx(fb, A_BYTES + B_BYTES);
+                    ptx::tma_load_2d(ptx::smem_u32(st), &tmap_dy, fb, kc * BK, mt * BM);
+                    ptx::tma_load_2d(ptx::smem_u32(st + A_BYTES), &tmap_wt, fb, kc * BK, row0);
+                    issued |= 1u << stage;
+                    issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+                    if (++stage == a.stages) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+            if (*s_abort) {
+                volatile int dummy = 0;
+                for (int i = 0; i < a.stages; ++i)
+                    if ((issued >> i) & 1u)
+                        ptx::mbar_wait(ptx::smem_u32(&full[i]), (issued_par >> i) & 1u, &dummy, nullptr, WAIT_LIMIT);
+            }
+        }
+        __syncwarp();
+    } else if (warp == MMA_WARP) {
+        // ----------------------------------------------------------- MMA --
+        if (lane == 0) {
+            int stage = 0, seg = 0;
+            uint32_t phase = 0;
+            const uint32_t idesc = ptx::idesc_bf16_f32(BM, NT);
+            const uint32_t s0 = ptx::smem_u32(smem);
+            bool ok = true;
+            for (long long u = ubeg; u < uend && ok; ++u, ++seg) {
+                const int abuf = seg & 1;
+                const uint32_t aphase = (seg >> 1) & 1;
+                if (!ptx::mbar_wait(ptx::smem_u32(&acc_empty[abuf]), aphase ^ 1, s_abort, a.status, WAIT_LIMIT)) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                const uint32_t d = tmem_base + (uint32_t)(abuf * NT);
+                for (int kc = 0; kc < a.kchunks; ++kc) {
+                    if (!ptx::mbar_wait(ptx::smem_u32(&full[stage]), phase, s_abort, a.status, WAIT_LIMIT)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t st = s0 + stage * stage_bytes;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        ptx::mma_bf16(d, ptx::sw128_desc(st + kk * 32), ptx::sw128_desc(st + A_BYTES + kk * 32), idesc,
+                                      (kc > 0 || kk > 0) ? 1u : 0u);
+                    ptx::mma_commit(ptx::smem_u32(&empty[stage]));
+                    if (++stage == a.stages) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+                if (!ok) break;
+                ptx::mma_commit(ptx::smem_u32(&acc_full[abuf]));
+            }
+            ptx::mma_commit(ptx::smem_u32(drain));
+            volatile int dummy = 0;
+            ptx::mbar_wait(ptx::smem_u32(drain), 0, &dummy, a.status, WAIT_LIMIT);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------ epilogue --
+        const int quarter = warp & 3, half = warp >> 2;  // lane quarter of TMEM, channel half
+        const int row = quarter * 32 + lane;
+        const int plane = s.Ho * s.Wo;
+        int seg = 0;
+        bool ok = true;
+        for (long long u = ubeg; u < uend && ok; ++u, ++seg) {
+            const int abuf = seg & 1;
+            const uint32_t aphase = (seg >> 1) & 1;
+            if (!ptx::mbar_wait(ptx::smem_u32(&acc_full[abuf]), aphase, s_abort, a.status, WAIT_LIMIT)) {
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after();
+            const int mt = (int)(u / a.units_per_tile), r = (int)(u - (long long)mt * a.units_per_tile);
+            const int gtap = r / a.nblk, cb = r - gtap * a.nblk;
+            const int g = gtap / s.K2, tap = gtap - g * s.K2;
+            const int p = mt * BM + row;
+            const int c_lo = cb * NT + half * (NT / 2);               // channel within the group
+            const int nch = max(0, min(NT / 2, s.Cg - c_lo));
+            const uint32_t taddr = tmem_base + (uint32_t)(abuf * NT + half * (NT / 2)) + ((uint32_t)(quarter * 32) << 16);
+            // sample of (p, tap, g)
+            const float4 rc = (p < s.P) ? a.rec[(size_t)gtap * a.ppad + p] : make_float4(0.f, 0.f, 0.f, 0.f);
+            const uint32_t yx = __float_as_uint(rc.w);
+            const bool any = (p < s.P) && yx != 0xFFFFFFFFu;
+            const int y0 = (int)(yx >> 16) - 1, x0 = (int)(yx & 0xFFFFu) - 1;
+            const int b = p / plane;
+            const float ly = rc.x, lx = rc.y, m = rc.z;
+            const bool i00 = any && inside(s, y0, x0), i01 = any && inside(s, y0, x0 + 1);
+            const bool i10 = any && inside(s, y0 + 1, x0), i11 = any && inside(s, y0 + 1, x0 + 1);
+            const float w00 = (1.f - ly) * (1.f - lx), w01 = (1.f - ly) * lx, w10 = ly * (1.f - lx), w11 = ly * lx;
+            const size_t a00 = (((size_t)b * s.H + y0) * s.W + x0) * s.Cin + g * s.Cg + c_lo;
+            const size_t a01 = a00 + s.Cin, a10 = a00 + (size_t)s.W * s.Cin, a11 = a10 + s.Cin;
+            float gdy = 0.f, gdx = 0.f, gm = 0.f;
+            for (int cc = 0; cc < NT / 2; cc += 32) {
+                float G[32];
+                ptx::tmem_ld32(taddr + cc, G);
+                if (!any || cc >= nch) continue;
+                // neighbours of 32 channels (zero outside the map), 4 x 64 bytes
+                uint4 v[4][4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 z = make_uint4(0, 0, 0, 0);
+                    const bool cv = cc + 8 * q < nch;  // 8-channel vectors inside the group (Cin/G % 8 == 0)
+                    v[0][q] = (cv && i00) ? ptx::ldg_v4(a.x + a00 + cc + 8 * q) : z;
+                    v[1][q] = (cv && i01) ? ptx::ldg_v4(a.x + a01 + cc + 8 * q) : z;
+                    v[2][q] = (cv && i10) ? ptx::ldg_v4(a.x + a10 + cc + 8 * q) : z;
+                    v[3][q] = (cv && i11) ? ptx::ldg_v4(a.x + a11 + cc + 8 * q) : z;
+                }
+                float g00[32], g01[32], g10[32], g11[32];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t* p00 = reinterpret_cast<const uint32_t*>(&v[0][q]);
+                    const uint32_t* p01 = reinterpret_cast<const uint32_t*>(&v[1][q]);
+                    const uint32_t* p10 = reinterpret_cast<const uint32_t*>(&v[2][q]);
+                    const uint32_t* p11 = reinterpret_cast<const uint32_t*>(&v[3][q]);
+#pragma unroll
+                    for (int h = 0; h < 8; ++h) {
+                        const int c = 8 * q + h;
+                        const uint32_t w = h >> 1;
+                        const float x00 = (h & 1) ? bf_hi(p00[w]) : bf_lo(p00[w]);
+                        const float x01 = (h & 1) ? bf_hi(p01[w]) : bf_lo(p01[w]);
+                        const float x10 = (h & 1) ? bf_hi(p10[w]) : bf_lo(p10[w]);
+                        const float x11 = (h & 1) ? bf_hi(p11[w]) : bf_lo(p11[w]);
+                        const float Gc = (cc + c < nch) ? G[c] : 0.f;
+                        gm = fmaf(Gc, w00 * x00 + w01 * x01 + w10 * x10 + w11 * x11, gm);
+                        gdy = fmaf(Gc, (1.f - lx) * (x10 - x00) + lx * (x11 - x01), gdy);
+                        gdx = fmaf(Gc, (1.f - ly) * (x01 - x00) + ly * (x11 - x10), gdx);
+                        const float gmc = Gc * m;
+                        g00[c] = gmc * w00;
+                        g01[c] = gmc * w01;
+                        g10[c] = gmc * w10;
+                        g11[c] = gmc * w11;
+                    }
+                }
+                if (a.gx && cc + 32 <= nch) {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        if (i00) ptx::red_add_v4(a.gx + a00 + cc + 4 * q, g00[4 * q], g00[4 * q + 1], g00[4 * q + 2], g00[4 * q + 3]);
+                        if (i01) ptx::red_add_v4(a.gx + a01 + cc + 4 * q, g01[4 * q], g01[4 * q + 1], g01[4 * q + 2], g01[4 * q + 3]);
+                        if (i10) ptx::red_add_v4(a.gx + a10 + cc + 4 * q, g10[4 * q], g10[4 * q + 1], g10[4 * q + 2], g10[4 * q + 3]);
+                        if (i11) ptx::red_add_v4(a.gx + a11 + cc + 4 * q, g11[4 * q], g11[4 * q + 1], g11[4 * q + 2], g11[4 * q + 3]);
+                    }
+                } else if (a.gx) {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        if (cc + c >= nch) continue;
+                        if (i00) atomicAdd(a.gx + a00 + cc + c, g00[c]);
+                        if (i01) atomicAdd(a.gx + a01 + cc + c, g01[c]);
+                        if (i10) atomicAdd(a.gx + a10 + cc + c, g10[c]);
+                        if (i11) atomicAdd(a.gx + a11 + cc + c, g11[c]);
+                    }
+                }
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&acc_empty[abuf]));
+            if (any && nch > 0) {
+                const int pix = p - b * plane;
+                const size_t ob = ((size_t)b * 2 * s.G * s.K2 + (size_t)g * 2 * s.K2 + 2 * tap) * plane + pix;
+                if (a.goff) {
+                    atomicAdd(a.goff + ob, m * gdy);
+                    atomicAdd(a.goff + ob + plane, m * gdx);
+                }
+                if (a.gmask) atomicAdd(a.gmask + ((size_t)b * s.G * s.K2 + (size_t)g * s.K2 + tap) * plane + pix, gm);
+            }
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == MMA_WARP) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem_base, 512);
+    }
+}
+
+// Float32 sampling records [G*K2][Ppad] for the backward: fractions, mask and
+// the top-left neighbour (packed with +1 so that row/column -1 fits).
+__global__ void __launch_bounds__(256) dcn_records_f32_kernel(Shape s, const bf16* __restrict__ off,
+                                                              const bf16* __restrict__ mask, float4* __restrict__ rec,
+                                                              int ppad) {
+    const int p = blockIdx.x * blockDim.x + threadIdx.x;
+    const int gt = blockIdx.y;
+    if (p >= ppad) return;
+    float4 r = make_float4(0.f, 0.f, 0.f, __uint_as_float(0xFFFFFFFFu));
+    if (p < s.P) {
+        const int g = gt / s.K2, tap = gt - g * s.K2;
+        const TapSample t = tap_sample(s, off, mask, p, g, tap);
+        const bool any = inside(s, t.y0, t.x0) || inside(s, t.y0, t.x0 + 1) || inside(s, t.y0 + 1, t.x0) ||
+                         inside(s, t.y0 + 1, t.x0 + 1);
+        r = make_float4(t.ly, t.lx, t.m,
+                        __uint_as_float(any ? (((uint32_t)(t.y0 + 1) << 16) | (uint32_t)(t.x0 + 1)) : 0xFFFFFFFFu));
+    }
+    rec[(size_t)gt * ppad + p] = r;
+}
+
+// w [Cout, KC] -> wt [KC, Cout] (bf16), 32x32 tiles through shared memory.
+__global__ void __launch_bounds__(256) dcn_transpose_kernel(const bf16* __restrict__ w, bf16* __restrict__ wt,
+                                                            int Cout, int KC) {
+    __shared__ bf16 t[32][33];
+    const int k0 = blockIdx.x * 32, o0 = blockIdx.y * 32;
+    for (int i = threadIdx.y; i < 32; i += 8) {
+        const int o = o0 + i, k = k0 + threadIdx.x;
+        if (o < Cout && k < KC) t[i][threadIdx.x] = w[(size_t)o * KC + k];
+    }
+    __syncthreads();
+    for (int i = threadIdx.y; i < 32; i += 8) {
+        const int k = k0 + i, o = o0 + threadIdx.x;
+        if (o < Cout && k < KC) wt[(size_t)k * Cout + o] = t[threadIdx.x][i];
+    }
+}
+
+struct BdPlan {
+    bool ok;
+    int nblk, units_per_tile, m_tiles, ppad, ctas, stages, kchunks;
+    long long total_units;
+    uint32_t smem_bytes;
+    size_t rec_bytes, wt_off, ws_bytes;
+};
+
+BdPlan make_bd_plan(const Shape& s, int sms) {
+    BdPlan pl{};
+    if (s.Cin % 8 || s.Cg % 8 || s.Cout % 8 || s.H >= 65535 || s.W >= 65535) return pl;
+    pl.nblk = (s.Cg + NT - 1) / NT;
+    pl.units_per_tile = s.G * s.K2 * pl.nblk;
+    pl.m_tiles = (s.P + BM - 1) / BM;
+    pl.ppad = pl.m_tiles * BM;
+    pl.kchunks = (s.Cout + BK - 1) / BK;
+    pl.total_units = (long long)pl.m_tiles * pl.units_per_tile;
+    pl.ctas = (int)std::min<long long>(sms, pl.total_units);
+    const uint32_t budget = 227 * 1024;
+    int st = (int)((budget - 2048) / (A_BYTES + B_BYTES));
+    pl.stages = std::min(st, 4);
+    pl.smem_bytes = pl.stages * (A_BYTES + B_BYTES) + (2 * MAX_STAGES + 5) * 8 + 16 + 1024;
+    pl.rec_bytes = (size_t)s.G * s.K2 * pl.ppad * sizeof(float4);
+    pl.wt_off = (pl.rec_bytes + 255) & ~(size_t)255;
+    pl.ws_bytes = pl.wt_off + (size_t)s.KC * s.Cout * sizeof(bf16);
+    pl.ok = (long long)s.B * s.H * s.W * s.Cin < (1LL << 31);
+    return pl;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+bool encode_kmajor(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+    auto encode = encode_fn();
+    if (!encode) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)inner * 2};
+    cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool bwd_data_tc_supported(const Shape& s) { return make_bd_plan(s, num_sms()).ok; }
+
+size_t bwd_data_tc_workspace(const Shape& s) {
+    BdPlan pl = make_bd_plan(s, num_sms());
+    return pl.ok ? pl.ws_bytes : 0;
+}
+
+cudaError_t bwd_data_tc(const Shape& s, const void* x, const void* off, const void* mask, const void* w,
+                        const void* gy, float* gx, float* goff, float* gmask, void* ws, size_t ws_bytes,
+                        unsigned* status, cudaStream_t st, int* launches) {
+    BdPlan pl = make_bd_plan(s, num_sms());
+    if (!pl.ok || !ws || ws_bytes < pl.ws_bytes) return cudaErrorInvalidValue;
+    float4* rec = reinterpret_cast<float4*>(ws);
+    bf16* wt = reinterpret_cast<bf16*>(static_cast<uint8_t*>(ws) + pl.wt_off);
+    CUtensorMap map_dy, map_wt;
+    if (!encode_kmajor(&map_dy, gy, (uint64_t)s.Cout, (uint64_t)s.P, BM) ||
+        !encode_kmajor(&map_wt, wt, (uint64_t)s.Cout, (uint64_t)s.KC, NT))
+        return cudaErrorInvalidValue;
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        e = cudaFuncSetAttribute(dcn_bwd_data_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    int n = 0;
+    dim3 tg((s.KC + 31) / 32, (s.Cout + 31) / 32);
+    dcn_transpose_kernel<<<tg, dim3(32, 8), 0, st>>>((const bf16*)w, wt, s.Cout, s.KC);
+    ++n;
+    dim3 rg((pl.ppad + 255) / 256, s.G * s.K2);
+    dcn_records_f32_kernel<<<rg, 256, 0, st>>>(s, (const bf16*)off, (const bf16*)mask, rec, pl.ppad);
+    ++n;
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (gx) {
+        if ((e = cudaMemsetAsync(gx, 0, sizeof(float) * (size_t)s.B * s.H * s.W * s.Cin, st)) != cudaSuccess) return e;
+        ++n;
+    }
+    if (goff) {
+        if ((e = cudaMemsetAsync(goff, 0, sizeof(float) * (size_t)s.P * 2 * s.G * s.K2, st)) != cudaSuccess) return e;
+        ++n;
+    }
+    if (gmask) {
+        if ((e = cudaMemsetAsync(gmask, 0, sizeof(float) * (size_t)s.P * s.G * s.K2, st)) != cudaSuccess) return e;
+        ++n;
+    }
+    BdArgs a;
+    a.s = s;
+    a.x = (const bf16*)x;
+    a.rec = rec;
+    a.gx = gx;
+    a.goff = goff;
+    a.gmask = gmask;
+    a.status = status;
+    a.nblk = pl.nblk;
+    a.units_per_tile = pl.units_per_tile;
+    a.m_tiles = pl.m_tiles;
+    a.ppad = pl.ppad;
+    a.ctas = pl.ctas;
+    a.stages = pl.stages;
+    a.kchunks = pl.kchunks;
+    a.total_units = pl.total_units;
+    dcn_bwd_data_tc_kernel<<<pl.ctas, NUM_THREADS, pl.smem_bytes, st>>>(map_dy, map_wt, a);
+    ++n;
+    if (launches) *launches += n;
+    return cudaGetLastError();
+}
+
+}  // namespace dcn

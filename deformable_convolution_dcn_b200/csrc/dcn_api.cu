@@ -106,6 +106,16 @@ bool use_fwd_small(const dcn_params_t* p, const dcn::Shape& s) {
     return p->dtype == DCN_F32 && !(p->flags & DCN_FLAG_GENERIC) && dcn::fwd_f32_small_supported(s);
 }
 
+// The tensor-core weight gradient: bfloat16, channel counts multiples of 8, Cout <= 256.
+bool use_bwd_weight_tc(const dcn_params_t* p, const dcn::Shape& s) {
+    return p->dtype == DCN_BF16 && !(p->flags & DCN_FLAG_GENERIC) && dcn::bwd_weight_tc_supported(s);
+}
+
+// The tensor-core data-side backward: bfloat16, channel counts multiples of 8.
+bool use_bwd_data_tc(const dcn_params_t* p, const dcn::Shape& s) {
+    return p->dtype == DCN_BF16 && !(p->flags & DCN_FLAG_GENERIC) && dcn::bwd_data_tc_supported(s);
+}
+
 #define TRY(expr)                    \
     do {                             \
         int _rc = (expr);            \
@@ -134,6 +144,8 @@ size_t dcn_workspace_size(const dcn_params_t* params, int op) {
         return 0;
     }
     if (op == DCN_OP_FORWARD && use_fwd_tc(params, s)) return dcn::fwd_tc_workspace(s);
+    if (op == DCN_OP_BACKWARD_WEIGHT && use_bwd_weight_tc(params, s)) return dcn::bwd_weight_tc_workspace(s);
+    if (op == DCN_OP_BACKWARD_DATA && use_bwd_data_tc(params, s)) return dcn::bwd_data_tc_workspace(s);
     return 0;
 }
 
@@ -232,11 +244,24 @@ int dcn_backward_data(const dcn_params_t* params, const void* x, const void* off
     TRY(check_ptr(grad_offset, "grad_offset", 4, false));
     TRY(check_ptr(grad_mask, "grad_mask", 4, false));
     if (grad_mask && !mask) return fail(DCN_ERR_INVALID_ARG, "grad_mask requested but mask is NULL");
-    (void)workspace;
-    (void)workspace_bytes;
     if (!grad_x && !grad_offset && !grad_mask) return ok();
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e;
+    if (use_bwd_data_tc(params, s) && aligned16(x) && aligned16(weight) && aligned16(grad_y) && aligned16(grad_x)) {
+        const size_t need = dcn::bwd_data_tc_workspace(s);
+        if (!workspace || workspace_bytes < need)
+            return fail(DCN_ERR_WORKSPACE, "backward-data needs %zu bytes of workspace, got %zu", need,
+                        workspace ? workspace_bytes : (size_t)0);
+        unsigned* status = nullptr;
+        e = dcn::status_word_ptr(&status);
+        if (e != cudaSuccess) return cuda_fail(e, "status word");
+        int n = 0;
+        e = dcn::bwd_data_tc(s, x, offset, mask, weight, grad_y, grad_x, grad_offset, grad_mask, workspace,
+                             workspace_bytes, status, st, &n);
+        g_launches += n;
+        if (e != cudaSuccess) return cuda_fail(e, "tensor-core backward-data launch");
+        return ok();
+    }
     if (grad_x) {
         e = cudaMemsetAsync(grad_x, 0, sizeof(float) * (size_t)s.B * s.H * s.W * s.Cin, st);
         g_launches += 1;
@@ -277,15 +302,28 @@ int dcn_backward_weight(const dcn_params_t* params, const void* x, const void* o
     TRY(check_ptr(grad_y, "grad_y", es, true));
     TRY(check_ptr(grad_weight, "grad_weight", 4, true));
     TRY(check_ptr(grad_bias, "grad_bias", 4, false));
-    (void)workspace;
-    (void)workspace_bytes;
     cudaStream_t st = (cudaStream_t)stream;
-    cudaError_t e = cudaMemsetAsync(grad_weight, 0, sizeof(float) * (size_t)s.Cout * s.KC, st);
-    g_launches += 1;
-    if (e != cudaSuccess) return cuda_fail(e, "zeroing grad_weight");
-    e = dcn::generic_backward_weight(s, params->dtype, x, offset, mask, grad_y, grad_weight, st);
-    g_launches += 1;
-    if (e != cudaSuccess) return cuda_fail(e, "backward-weight launch");
+    cudaError_t e;
+    if (use_bwd_weight_tc(params, s) && aligned16(x) && aligned16(grad_y) && aligned16(grad_weight)) {
+        const size_t need = dcn::bwd_weight_tc_workspace(s);
+        if (!workspace || workspace_bytes < need)
+            return fail(DCN_ERR_WORKSPACE, "backward-weight needs %zu bytes of workspace, got %zu", need,
+                        workspace ? workspace_bytes : (size_t)0);
+        unsigned* status = nullptr;
+        e = dcn::status_word_ptr(&status);
+        if (e != cudaSuccess) return cuda_fail(e, "status word");
+        int n = 0;
+        e = dcn::bwd_weight_tc(s, x, offset, mask, grad_y, grad_weight, workspace, workspace_bytes, status, st, &n);
+        g_launches += n;
+        if (e != cudaSuccess) return cuda_fail(e, "tensor-core backward-weight launch");
+    } else {
+        e = cudaMemsetAsync(grad_weight, 0, sizeof(float) * (size_t)s.Cout * s.KC, st);
+        g_launches += 1;
+        if (e != cudaSuccess) return cuda_fail(e, "zeroing grad_weight");
+        e = dcn::generic_backward_weight(s, params->dtype, x, offset, mask, grad_y, grad_weight, st);
+        g_launches += 1;
+        if (e != cudaSuccess) return cuda_fail(e, "backward-weight launch");
+    }
     if (grad_bias) {
         e = cudaMemsetAsync(grad_bias, 0, sizeof(float) * (size_t)s.Cout, st);
         g_launches += 1;

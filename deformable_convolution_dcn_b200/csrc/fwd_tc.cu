@@ -717,18 +717,6 @@ struct Plan {
     size_t ws_partials, ws_counters_off, ws_bytes;
 };
 
-int num_sms() {
-    static int cached[64] = {0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (!cached[dev]) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-        cached[dev] = n;
-    }
-    return cached[dev];
-}
-
 Plan make_plan(const Shape& s, int sms) {
     Plan pl{};
     pl.ok = false;

@@ -34,7 +34,21 @@ bool fwd_f32_small_supported(const Shape& s);
 cudaError_t fwd_f32_small(const Shape& s, const void* x, const void* off, const void* mask, const void* w,
                           const void* bias, void* y, cudaStream_t st);
 
-// status.cu — the device status word that bounded waits report to.
+// bwd_weight_tc.cu — bfloat16 weight gradient on tcgen05 (workspace: sampling records).
+bool bwd_weight_tc_supported(const Shape& s);
+size_t bwd_weight_tc_workspace(const Shape& s);
+cudaError_t bwd_weight_tc(const Shape& s, const void* x, const void* off, const void* mask, const void* gy,
+                          float* gw, void* ws, size_t ws_bytes, unsigned* status, cudaStream_t st, int* launches);
+
+// bwd_data_tc.cu — bfloat16 grad_x / grad_offset / grad_mask on tcgen05 (workspace: records, w^T).
+bool bwd_data_tc_supported(const Shape& s);
+size_t bwd_data_tc_workspace(const Shape& s);
+cudaError_t bwd_data_tc(const Shape& s, const void* x, const void* off, const void* mask, const void* w,
+                        const void* gy, float* gx, float* goff, float* gmask, void* ws, size_t ws_bytes,
+                        unsigned* status, cudaStream_t st, int* launches);
+
+// status.cu — the device status word that bounded waits report to; SM count.
+int num_sms();
 cudaError_t status_word_ptr(unsigned int** ptr);
 cudaError_t read_and_clear_status(unsigned int* out);
 

@@ -27,4 +27,16 @@ cudaError_t read_and_clear_status(unsigned int* out) {
     return cudaMemcpyToSymbol(g_status_word, &zero, sizeof(unsigned int));
 }
 
+int num_sms() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cached[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
 }  // namespace dcn
