@@ -38,6 +38,7 @@ constexpr long long WAIT_LIMIT = 2000000000LL;
 constexpr int MAX_STAGES = 4;
 constexpr uint32_t A_BYTES = BM * BK * 2;   // 16 KB
 constexpr uint32_t B_BYTES = NT * BK * 2;   // 32 KB
+constexpr int TPITCH = 36;                  // floats per row of an epilogue warp's 32x32 transpose buffer
 
 struct BdArgs {
     Shape s;
@@ -181,9 +182,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------ epilogue --
+        // Thread = pixel row when reading TMEM; the 32x32 block of G is then
+        // staged in shared memory and re-read so that 8 lanes cover one pixel's
+        // 32 channels (4 each): neighbour loads are 64 contiguous bytes and the
+        // grad_x atomics 128 contiguous bytes per pixel and corner.
         const int quarter = warp & 3, half = warp >> 2;  // lane quarter of TMEM, channel half
         const int row = quarter * 32 + lane;
         const int plane = s.Ho * s.Wo;
+        float* tb = reinterpret_cast<float*>(smem + a.stages * stage_bytes + 1024) + warp * 32 * TPITCH;
+        const int pq = lane >> 3, cj = lane & 7;  // pixel within a group of 4, 4-channel slot
         int seg = 0;
         bool ok = true;
         for (long long u = ubeg; u < uend && ok; ++u, ++seg) {
@@ -197,94 +204,107 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const int mt = (int)(u / a.units_per_tile), r = (int)(u - (long long)mt * a.units_per_tile);
             const int gtap = r / a.nblk, cb = r - gtap * a.nblk;
             const int g = gtap / s.K2, tap = gtap - g * s.K2;
-            const int p = mt * BM + row;
-            const int c_lo = cb * NT + half * (NT / 2);               // channel within the group
+            const int c_lo = cb * NT + half * (NT / 2);  // channel within the group
             const int nch = max(0, min(NT / 2, s.Cg - c_lo));
             const uint32_t taddr = tmem_base + (uint32_t)(abuf * NT + half * (NT / 2)) + ((uint32_t)(quarter * 32) << 16);
-            // sample of (p, tap, g)
+            // this thread's own pixel: sample and address of its top-left neighbour
+            const int p = mt * BM + row;
             const float4 rc = (p < s.P) ? a.rec[(size_t)gtap * a.ppad + p] : make_float4(0.f, 0.f, 0.f, 0.f);
             const uint32_t yx = __float_as_uint(rc.w);
             const bool any = (p < s.P) && yx != 0xFFFFFFFFu;
             const int y0 = (int)(yx >> 16) - 1, x0 = (int)(yx & 0xFFFFu) - 1;
             const int b = p / plane;
-            const float ly = rc.x, lx = rc.y, m = rc.z;
-            const bool i00 = any && inside(s, y0, x0), i01 = any && inside(s, y0, x0 + 1);
-            const bool i10 = any && inside(s, y0 + 1, x0), i11 = any && inside(s, y0 + 1, x0 + 1);
-            const float w00 = (1.f - ly) * (1.f - lx), w01 = (1.f - ly) * lx, w10 = ly * (1.f - lx), w11 = ly * lx;
-            const size_t a00 = (((size_t)b * s.H + y0) * s.W + x0) * s.Cin + g * s.Cg + c_lo;
-            const size_t a01 = a00 + s.Cin, a10 = a00 + (size_t)s.W * s.Cin, a11 = a10 + s.Cin;
-            float gdy = 0.f, gdx = 0.f, gm = 0.f;
+            uint32_t flags = 0;
+            if (any) {
+                flags = (inside(s, y0, x0) ? 1u : 0u) | (inside(s, y0, x0 + 1) ? 2u : 0u) |
+                        (inside(s, y0 + 1, x0) ? 4u : 0u) | (inside(s, y0 + 1, x0 + 1) ? 8u : 0u);
+            }
+            const long long a00 =
+                any ? ((((long long)b * s.H + y0) * s.W + x0) * s.Cin + g * s.Cg + c_lo) : 0;
+            float part[8][3];  // per pixel group: m-less d/dy, d/dx and the mask gradient, over this lane's channels
+#pragma unroll
+            for (int q = 0; q < 8; ++q) part[q][0] = part[q][1] = part[q][2] = 0.f;
             for (int cc = 0; cc < NT / 2; cc += 32) {
                 float G[32];
                 ptx::tmem_ld32(taddr + cc, G);
-                if (!any || cc >= nch) continue;
-                // neighbours of 32 channels (zero outside the map), 4 x 64 bytes
-                uint4 v[4][4];
+                if (cc >= nch) continue;  // warp-uniform
+                __syncwarp();
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint4 z = make_uint4(0, 0, 0, 0);
-                    const bool cv = cc + 8 * q < nch;  // 8-channel vectors inside the group (Cin/G % 8 == 0)
-                    v[0][q] = (cv && i00) ? ptx::ldg_v4(a.x + a00 + cc + 8 * q) : z;
-                    v[1][q] = (cv && i01) ? ptx::ldg_v4(a.x + a01 + cc + 8 * q) : z;
-                    v[2][q] = (cv && i10) ? ptx::ldg_v4(a.x + a10 + cc + 8 * q) : z;
-                    v[3][q] = (cv && i11) ? ptx::ldg_v4(a.x + a11 + cc + 8 * q) : z;
-                }
-                float g00[32], g01[32], g10[32], g11[32];
+                for (int q = 0; q < 8; ++q)
+                    *reinterpret_cast<float4*>(tb + lane * TPITCH + 4 * q) = make_float4(G[4 * q], G[4 * q + 1], G[4 * q + 2], G[4 * q + 3]);
+                __syncwarp();
+                const bool cv = cc + 4 * cj < nch;  // this lane's 4 channels inside the group
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint32_t* p00 = reinterpret_cast<const uint32_t*>(&v[0][q]);
-                    const uint32_t* p01 = reinterpret_cast<const uint32_t*>(&v[1][q]);
-                    const uint32_t* p10 = reinterpret_cast<const uint32_t*>(&v[2][q]);
-                    const uint32_t* p11 = reinterpret_cast<const uint32_t*>(&v[3][q]);
+                for (int gp = 0; gp < 8; ++gp) {
+                    const int src = 4 * gp + pq;  // lane (pixel row) whose sample this lane works on
+                    const float ly = __shfl_sync(0xffffffffu, rc.x, src), lx = __shfl_sync(0xffffffffu, rc.y, src);
+                    const float m = __shfl_sync(0xffffffffu, rc.z, src);
+                    const uint32_t fl = __shfl_sync(0xffffffffu, flags, src);
+                    const long long base = __shfl_sync(0xffffffffu, a00, src);
+                    if (!fl || !cv) continue;
+                    const float4 Gv = *reinterpret_cast<const float4*>(tb + src * TPITCH + 4 * cj);
+                    const long long o00 = base + cc + 4 * cj;
+                    const long long o01 = o00 + s.Cin, o10 = o00 + (long long)s.W * s.Cin, o11 = o10 + s.Cin;
+                    const uint2 z = make_uint2(0, 0);
+                    const uint2 v00 = (fl & 1u) ? ptx::ldg_v2(a.x + o00) : z;
+                    const uint2 v01 = (fl & 2u) ? ptx::ldg_v2(a.x + o01) : z;
+                    const uint2 v10 = (fl & 4u) ? ptx::ldg_v2(a.x + o10) : z;
+                    const uint2 v11 = (fl & 8u) ? ptx::ldg_v2(a.x + o11) : z;
+                    const float w00 = (1.f - ly) * (1.f - lx), w01 = (1.f - ly) * lx, w10 = ly * (1.f - lx), w11 = ly * lx;
+                    const float Gc[4] = {Gv.x, Gv.y, Gv.z, Gv.w};
+                    float r00[4], r01[4], r10[4], r11[4];
 #pragma unroll
-                    for (int h = 0; h < 8; ++h) {
-                        const int c = 8 * q + h;
-                        const uint32_t w = h >> 1;
-                        const float x00 = (h & 1) ? bf_hi(p00[w]) : bf_lo(p00[w]);
-                        const float x01 = (h & 1) ? bf_hi(p01[w]) : bf_lo(p01[w]);
-                        const float x10 = (h & 1) ? bf_hi(p10[w]) : bf_lo(p10[w]);
-                        const float x11 = (h & 1) ? bf_hi(p11[w]) : bf_lo(p11[w]);
-                        const float Gc = (cc + c < nch) ? G[c] : 0.f;
-                        gm = fmaf(Gc, w00 * x00 + w01 * x01 + w10 * x10 + w11 * x11, gm);
-                        gdy = fmaf(Gc, (1.f - lx) * (x10 - x00) + lx * (x11 - x01), gdy);
-                        gdx = fmaf(Gc, (1.f - ly) * (x01 - x00) + ly * (x11 - x10), gdx);
-                        const float gmc = Gc * m;
-                        g00[c] = gmc * w00;
-                        g01[c] = gmc * w01;
-                        g10[c] = gmc * w10;
-                        g11[c] = gmc * w11;
+                    for (int h = 0; h < 4; ++h) {
+                        const uint32_t wsel = h >> 1;
+                        const uint32_t e00 = wsel ? v00.y : v00.x, e01 = wsel ? v01.y : v01.x;
+                        const uint32_t e10 = wsel ? v10.y : v10.x, e11 = wsel ? v11.y : v11.x;
+                        const float x00 = (h & 1) ? bf_hi(e00) : bf_lo(e00), x01 = (h & 1) ? bf_hi(e01) : bf_lo(e01);
+                        const float x10 = (h & 1) ? bf_hi(e10) : bf_lo(e10), x11 = (h & 1) ? bf_hi(e11) : bf_lo(e11);
+                        part[gp][2] = fmaf(Gc[h], w00 * x00 + w01 * x01 + w10 * x10 + w11 * x11, part[gp][2]);
+                        part[gp][0] = fmaf(Gc[h], (1.f - lx) * (x10 - x00) + lx * (x11 - x01), part[gp][0]);
+                        part[gp][1] = fmaf(Gc[h], (1.f - ly) * (x01 - x00) + ly * (x11 - x10), part[gp][1]);
+                        const float gmc = Gc[h] * m;
+                        r00[h] = gmc * w00;
+                        r01[h] = gmc * w01;
+                        r10[h] = gmc * w10;
+                        r11[h] = gmc * w11;
                     }
-                }
-                if (a.gx && cc + 32 <= nch) {
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        if (i00) ptx::red_add_v4(a.gx + a00 + cc + 4 * q, g00[4 * q], g00[4 * q + 1], g00[4 * q + 2], g00[4 * q + 3]);
-                        if (i01) ptx::red_add_v4(a.gx + a01 + cc + 4 * q, g01[4 * q], g01[4 * q + 1], g01[4 * q + 2], g01[4 * q + 3]);
-                        if (i10) ptx::red_add_v4(a.gx + a10 + cc + 4 * q, g10[4 * q], g10[4 * q + 1], g10[4 * q + 2], g10[4 * q + 3]);
-                        if (i11) ptx::red_add_v4(a.gx + a11 + cc + 4 * q, g11[4 * q], g11[4 * q + 1], g11[4 * q + 2], g11[4 * q + 3]);
-                    }
-                } else if (a.gx) {
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        if (cc + c >= nch) continue;
-                        if (i00) atomicAdd(a.gx + a00 + cc + c, g00[c]);
-                        if (i01) atomicAdd(a.gx + a01 + cc + c, g01[c]);
-                        if (i10) atomicAdd(a.gx + a10 + cc + c, g10[c]);
-                        if (i11) atomicAdd(a.gx + a11 + cc + c, g11[c]);
+                    if (a.gx) {
+                        if (fl & 1u) ptx::red_add_v4(a.gx + o00, r00[0], r00[1], r00[2], r00[3]);
+                        if (fl & 2u) ptx::red_add_v4(a.gx + o01, r01[0], r01[1], r01[2], r01[3]);
+                        if (fl & 4u) ptx::red_add_v4(a.gx + o10, r10[0], r10[1], r10[2], r10[3]);
+                        if (fl & 8u) ptx::red_add_v4(a.gx + o11, r11[0], r11[1], r11[2], r11[3]);
                     }
                 }
             }
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&acc_empty[abuf]));
-            if (any && nch > 0) {
-                const int pix = p - b * plane;
-                const size_t ob = ((size_t)b * 2 * s.G * s.K2 + (size_t)g * 2 * s.K2 + 2 * tap) * plane + pix;
-                if (a.goff) {
-                    atomicAdd(a.goff + ob, m * gdy);
-                    atomicAdd(a.goff + ob + plane, m * gdx);
+            // reduce each pixel's partial sums over its 8 lanes; lane cj == 0 adds them in
+#pragma unroll
+            for (int gp = 0; gp < 8; ++gp) {
+#pragma unroll
+                for (int k = 0; k < 3; ++k) {
+                    float v = part[gp][k];
+                    v += __shfl_xor_sync(0xffffffffu, v, 1);
+                    v += __shfl_xor_sync(0xffffffffu, v, 2);
+                    v += __shfl_xor_sync(0xffffffffu, v, 4);
+                    part[gp][k] = v;
                 }
-                if (a.gmask) atomicAdd(a.gmask + ((size_t)b * s.G * s.K2 + (size_t)g * s.K2 + tap) * plane + pix, gm);
+                const int src = 4 * gp + pq;
+                const float m = __shfl_sync(0xffffffffu, rc.z, src);
+                const uint32_t fl = __shfl_sync(0xffffffffu, flags, src);
+                const int pp = mt * BM + quarter * 32 + src;
+                if (cj == 0 && fl && nch > 0 && pp < s.P) {
+                    const int bb = pp / plane, pix = pp - bb * plane;
+                    const size_t ob = ((size_t)bb * 2 * s.G * s.K2 + (size_t)g * 2 * s.K2 + 2 * tap) * plane + pix;
+                    if (a.goff) {
+                        atomicAdd(a.goff + ob, m * part[gp][0]);
+                        atomicAdd(a.goff + ob + plane, m * part[gp][1]);
+                    }
+                    if (a.gmask)
+                        atomicAdd(a.gmask + ((size_t)bb * s.G * s.K2 + (size_t)g * s.K2 + tap) * plane + pix, part[gp][2]);
+                }
             }
         }
     }
@@ -352,9 +372,10 @@ BdPlan make_bd_plan(const Shape& s, int sms) {
     pl.total_units = (long long)pl.m_tiles * pl.units_per_tile;
     pl.ctas = (int)std::min<long long>(sms, pl.total_units);
     const uint32_t budget = 227 * 1024;
-    int st = (int)((budget - 2048) / (A_BYTES + B_BYTES));
-    pl.stages = std::min(st, 4);
-    pl.smem_bytes = pl.stages * (A_BYTES + B_BYTES) + (2 * MAX_STAGES + 5) * 8 + 16 + 1024;
+    const uint32_t tbytes = EPI_WARPS * 32 * TPITCH * 4;  // epilogue transpose buffers
+    int st = (int)((budget - 2048 - 1024 - tbytes) / (A_BYTES + B_BYTES));
+    pl.stages = std::min(st, 3);
+    pl.smem_bytes = pl.stages * (A_BYTES + B_BYTES) + 1024 + tbytes + 1024;
     pl.rec_bytes = (size_t)s.G * s.K2 * pl.ppad * sizeof(float4);
     pl.wt_off = (pl.rec_bytes + 255) & ~(size_t)255;
     pl.ws_bytes = pl.wt_off + (size_t)s.KC * s.Cout * sizeof(bf16);

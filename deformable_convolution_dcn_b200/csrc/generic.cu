@@ -265,15 +265,23 @@ __global__ void __launch_bounds__(256) generic_backward_weight_kernel(Shape s, c
     }
 }
 
-// grad_bias[o] = sum_p grad_y[p, o]; one thread per channel per pixel slice.
+// grad_bias[o] = sum_p grad_y[p, o]: one thread per channel and 64-pixel slice
+// (loads coalesced across the channels of a warp, eight in flight per thread),
+// one atomic per thread.
 template <typename T>
 __global__ void __launch_bounds__(256) bias_grad_kernel(Shape s, const T* __restrict__ gy, float* __restrict__ gb,
                                                         int pix_per_split) {
-    int o = blockIdx.x * blockDim.x + threadIdx.x;
+    const int o = blockIdx.x * blockDim.x + threadIdx.x;
     if (o >= s.Cout) return;
-    int pbeg = blockIdx.y * pix_per_split, pend = min(s.P, pbeg + pix_per_split);
+    const int pbeg = blockIdx.y * pix_per_split, pend = min(s.P, pbeg + pix_per_split);
     float acc = 0.f;
-    for (int p = pbeg; p < pend; ++p) acc += ldf(gy + (size_t)p * s.Cout + o);
+    for (int p = pbeg; p < pend; p += 8) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = (p + u < pend) ? ldf(gy + (size_t)(p + u) * s.Cout + o) : 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) acc += v[u];
+    }
     atomicAdd(gb + o, acc);
 }
 
@@ -339,12 +347,12 @@ cudaError_t generic_backward_weight(const Shape& s, int dtype, const void* x, co
 }
 
 cudaError_t bias_grad(const Shape& s, int dtype, const void* gy, float* gb, cudaStream_t st) {
-    int bsplit = (s.P + 1023) / 1024;
-    dim3 g2((s.Cout + 255) / 256, bsplit);
+    const int per = 64;
+    dim3 g2((s.Cout + 255) / 256, (s.P + per - 1) / per);
     if (dtype == 0)
-        bias_grad_kernel<float><<<g2, 256, 0, st>>>(s, (const float*)gy, gb, 1024);
+        bias_grad_kernel<float><<<g2, 256, 0, st>>>(s, (const float*)gy, gb, per);
     else
-        bias_grad_kernel<bf16><<<g2, 256, 0, st>>>(s, (const bf16*)gy, gb, 1024);
+        bias_grad_kernel<bf16><<<g2, 256, 0, st>>>(s, (const bf16*)gy, gb, per);
     return cudaGetLastError();
 }
 
