@@ -210,6 +210,19 @@ __device__ __forceinline__ void add_partial32(float (&v)[32], const float* src, 
     }
 }
 
+// As add_partial32, from a partial tile staged in shared memory.
+__device__ __forceinline__ void add_partial32_smem(float (&v)[32], const float* src, int cc) {
+    const float* b = src + (size_t)(cc >> 5) * 8 * BM * 4;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const float4 f = *reinterpret_cast<const float4*>(b + q * BM * 4);
+        v[4 * q] += f.x;
+        v[4 * q + 1] += f.y;
+        v[4 * q + 2] += f.z;
+        v[4 * q + 3] += f.w;
+    }
+}
+
 // y[row, n0 + cc .. n0 + cc + 31] = v + bias, as bf16 (columns < ncols).
 __device__ __forceinline__ void store_row32(bf16* yrow, int cc, int ncols, float (&v)[32], const bf16* bias, int n0) {
     if (bias) {
@@ -269,7 +282,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + a.bar_off);
     // barrier slots
     uint64_t* full_a = bars;
-    uint64_t* full_b = bars + MAX_STAGES;
+    uint64_t* tail_bar = bars + MAX_STAGES;  // bulk copy of other CTAs' partials for the last segment
     uint64_t* empty = bars + 2 * MAX_STAGES;
     uint64_t* acc_full = bars + 3 * MAX_STAGES;
     uint64_t* acc_empty = acc_full + 2;
@@ -282,8 +295,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < a.stages; ++i) {
-            ptx::mbar_init(ptx::smem_u32(&full_a[i]), NUM_PROD_WARPS / GROUPS);
-            ptx::mbar_init(ptx::smem_u32(&full_b[i]), 1);
+            // a stage is full when its producer group's warps and the weight TMA have both arrived
+            ptx::mbar_init(ptx::smem_u32(&full_a[i]), NUM_PROD_WARPS / GROUPS + 1);
             ptx::mbar_init(ptx::smem_u32(&empty[i]), 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -291,6 +304,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ptx::mbar_init(ptx::smem_u32(&acc_empty[i]), 4);
         }
         ptx::mbar_init(ptx::smem_u32(drain), 1);
+        ptx::mbar_init(ptx::smem_u32(tail_bar), 1);
         ptx::mbar_init(ptx::smem_u32(prod_bar), NUM_PROD_WARPS);
         ptx::mbar_init(ptx::smem_u32(epi_bar), 4);
         *s_abort = 0;
@@ -521,7 +535,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         break;
                     }
                     const int xk = ch.tap * s.Cin + ch.g * s.Cg + ch.q * BK;
-                    const uint32_t fb = ptx::smem_u32(&full_b[stage]);
+                    const uint32_t fb = ptx::smem_u32(&full_a[stage]);
                     ptx::mbar_arrive_expect_tx(fb, bytes);
                     for (int sub = 0; sub < a.nsub; ++sub)
                         ptx::tma_load_2d(ptx::smem_u32(sB + stage * a.b_stage_bytes + sub * a.box_rows * 128),
@@ -540,7 +554,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 volatile int dummy = 0;
                 for (int i = 0; i < a.stages; ++i)
                     if ((issued >> i) & 1u)
-                        ptx::mbar_wait(ptx::smem_u32(&full_b[i]), (issued_par >> i) & 1u, &dummy, nullptr,
+                        ptx::mbar_wait(ptx::smem_u32(&full_a[i]), (issued_par >> i) & 1u, &dummy, nullptr,
                                        WAIT_LIMIT);
             }
         }
@@ -568,8 +582,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 ptx::tc_fence_after();
                 const uint32_t d = tmem_base + (uint32_t)(abuf * a.acc_cols);
                 for (int k = k0; k < k1; ++k) {
-                    if (!ptx::mbar_wait(ptx::smem_u32(&full_a[stage]), phase, s_abort, a.status, WAIT_LIMIT) ||
-                        !ptx::mbar_wait(ptx::smem_u32(&full_b[stage]), phase, s_abort, a.status, WAIT_LIMIT)) {
+                    if (!ptx::mbar_wait(ptx::smem_u32(&full_a[stage]), phase, s_abort, a.status, WAIT_LIMIT)) {
                         ok = false;
                         break;
                     }
@@ -643,11 +656,43 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     break;
                 }
                 if (*s_last) {
+                    // The CTA's last segment: the pipeline buffers are idle, so when the other
+                    // contributors' partial tiles fit there they are bulk-copied in and read
+                    // from shared memory; otherwise they are read from global memory.
+                    const uint32_t tile_bytes = (uint32_t)BM * a.bn_total * 4;
+                    const bool last_seg = (long long)t * a.U + k1 == uend;
+                    const bool staged = last_seg && (uint32_t)(c_hi - c_lo) * tile_bytes <= a.b_off + a.stages * a.b_stage_bytes;
+                    if (staged) {
+                        if (threadIdx.x == 0) {
+                            ptx::fence_proxy_async_all();
+                            const uint32_t tb = ptx::smem_u32(tail_bar);
+                            ptx::mbar_arrive_expect_tx(tb, (uint32_t)(c_hi - c_lo) * tile_bytes);
+                            uint32_t dst = ptx::smem_u32(smem);
+                            for (int c = c_lo; c <= c_hi; ++c) {
+                                if (c == cta) continue;
+                                const uint8_t* src = reinterpret_cast<const uint8_t*>(partial_base(a, c, tu0, 0));
+                                for (uint32_t o = 0; o < tile_bytes; o += 16384u)
+                                    ptx::bulk_load(dst + o, src + o, min(16384u, tile_bytes - o), tb);
+                                dst += tile_bytes;
+                            }
+                        }
+                        if (!ptx::mbar_wait(ptx::smem_u32(tail_bar), 0, s_abort, a.status, WAIT_LIMIT)) {
+                            ok = false;
+                            break;
+                        }
+                    }
                     for (int cc = 0; cc < ncols; cc += 32) {
                         float v[32];
                         ptx::tmem_ld32(taddr + cc, v);
-                        for (int c = c_lo; c <= c_hi; ++c)
-                            if (c != cta) add_partial32(v, partial_base(a, c, tu0, row), cc);
+                        int slot = 0;
+                        for (int c = c_lo; c <= c_hi; ++c) {
+                            if (c == cta) continue;
+                            if (staged)
+                                add_partial32_smem(v, reinterpret_cast<const float*>(smem + (size_t)slot * tile_bytes) + row * 4, cc);
+                            else
+                                add_partial32(v, partial_base(a, c, tu0, row), cc);
+                            ++slot;
+                        }
                         if (p >= 0) store_row32(yrow, cc, ncols, v, a.bias, n0);
                     }
                     ptx::tc_fence_before();
