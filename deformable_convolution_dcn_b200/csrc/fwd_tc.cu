@@ -7,10 +7,10 @@
 // the y(p0) equations). Col is never written to HBM:
 //
 //   * producer warps (8) compute the sampling coordinates of a 128-pixel tile,
-//     load the four channel-contiguous NHWC neighbours of each sample as 16-byte
-//     vectors, blend them with the bilinear weights times the mask, and store
-//     the bf16 result straight into a shared-memory A tile laid out in the UMMA
-//     128-byte-swizzle K-major canonical form;
+//     load the four channel-contiguous NHWC neighbours of each sample as 32-byte
+//     vectors (16 channels per lane), blend them with the bilinear weights times
+//     the mask, and store the bf16 result straight into a shared-memory A tile
+//     laid out in the UMMA 128-byte-swizzle K-major canonical form;
 //   * one TMA warp stages the matching weight tile [N x 64] of W = [Cout, K*K*Cin];
 //   * one MMA warp issues tcgen05.mma (M=128, N<=256, K=16) into TMEM;
 //   * four epilogue warps read the accumulator back with tcgen05.ld, add the
@@ -40,21 +40,11 @@ constexpr int NUM_PROD_WARPS = 8;
 constexpr int TMA_WARP = 4, MMA_WARP = 5, PROD_WARP0 = 6;  // warps 0-3: epilogue
 constexpr int NUM_THREADS = (PROD_WARP0 + NUM_PROD_WARPS) * 32;
 constexpr int NUM_PROD_THREADS = NUM_PROD_WARPS * 32;
-#ifndef DCN_FWD_GROUPS
-#define DCN_FWD_GROUPS 2
-#endif
-#ifndef DCN_FWD_BLEND
-#define DCN_FWD_BLEND 1
-#endif
-constexpr int GROUPS = DCN_FWD_GROUPS;                    // producer groups taking alternate chunks
-constexpr int GROUP_THREADS = NUM_PROD_THREADS / GROUPS;
-constexpr int ROW_STEP = GROUP_THREADS / 8;                 // rows between a thread's rows
-constexpr int ROWS_PER_THREAD = BM / ROW_STEP;
-constexpr int INFO_BATCH = 5;
-#ifndef DCN_FWD_PREFETCH
-#define DCN_FWD_PREFETCH 1
-#endif
-constexpr bool PREFETCH = DCN_FWD_PREFETCH != 0;           // L1 prefetch of the next chunk's neighbours                               // sampling records per thread per pass
+constexpr int SLICE = 16;                                   // channels one lane gathers per sample (32 bytes)
+constexpr int LANES_PER_ROW = BK / SLICE;
+constexpr int ROW_STEP = NUM_PROD_THREADS / LANES_PER_ROW;  // rows between a thread's two rows
+static_assert(ROW_STEP % 8 == 0, "a thread's rows must share their swizzle phase");
+static_assert(2 * ROW_STEP == BM, "two rows per producer thread and chunk");
 constexpr long long WAIT_LIMIT = 2000000000LL;  // clock cycles (about a second)
 constexpr int MAX_STAGES = 8;
 #ifndef DCN_FWD_MAX_STAGES
@@ -74,91 +64,123 @@ struct FwdArgs {
     int n_tiles, tiles, U, nq, ctas;
     int sw, nf, wl;    // pixel order: vertical strips of width sw (nf full strips, last one wl wide)
     long long total_units;
+    int snap;          // a CTA never starts within the last snap-1 units of a tile (0: off)
     int bn_total;      // tile width in output channels (multiple of 16, <= 512)
     int nsub;          // accumulators per tile (1: N = bn_total; 2: 256 + rest)
     int box_rows;      // rows of one weight box
     int stages;
     int acc_cols;      // TMEM column stride between the two accumulator buffers (0: single buffer)
     int tmem_cols;
-    uint32_t b_off, info_off, base_off, row_off, bar_off, b_stage_bytes;
+    uint32_t b_off, info_off, row_off, bar_off, b_stage_bytes;
 };
 
+constexpr int MAX_CTAS = 256;  // entries of the per-CTA start table in shared memory
+
+// First unit of CTA c: an even split of the units, except that a start that
+// would fall within the last snap-1 units of a tile moves to the next tile's
+// first unit (the previous CTA takes those units), so that no CTA spends a
+// segment, and its epilogue, on a sliver of a tile. Every CTA tabulates these
+// starts once (starts[0..ctas], strictly increasing) and looks them up after.
 __device__ __forceinline__ long long unit_begin(int c, const FwdArgs& a) {
-    return a.total_units * c / a.ctas;
+    if (c >= a.ctas) return a.total_units;
+    long long u = a.total_units * c / a.ctas;
+    const long long k = u % a.U;
+    if (k != 0 && k > a.U - a.snap) u += a.U - k;
+    return u;
 }
-__device__ __forceinline__ int cta_of_unit(long long u, const FwdArgs& a) {
-    return (int)(((u + 1) * a.ctas + a.total_units - 1) / a.total_units) - 1;
+// The CTA whose range holds unit u: the last start at or before u.
+__device__ __forceinline__ int cta_of_unit(long long u, const long long* starts, int ctas) {
+    int lo = 0, hi = ctas - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (starts[mid] <= u) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+// The tiles a CTA's unit range touches (its segments), in unit order.
+struct SegList {
+    long long ubeg, uend;
+    int t0, ns, U;
+};
+struct Seg {
+    int t, k0, k1;  // tile, and its units [k0, k1) that this CTA owns
+};
+__device__ __forceinline__ SegList seg_list(long long ubeg, long long uend, int U) {
+    SegList L;
+    L.ubeg = ubeg;
+    L.uend = uend;
+    L.U = U;
+    if (uend <= ubeg) {
+        L.t0 = 0;
+        L.ns = 0;
+        return L;
+    }
+    L.t0 = (int)(ubeg / U);
+    L.ns = (int)((uend - 1) / U) - L.t0 + 1;
+    return L;
+}
+__device__ __forceinline__ Seg seg_at(const SegList& L, int i) {
+    Seg s;
+    s.t = L.t0 + i;
+    const long long tu = (long long)s.t * L.U;
+    s.k0 = (i == 0) ? (int)(L.ubeg - tu) : 0;
+    s.k1 = (i == L.ns - 1) ? (int)(L.uend - tu) : L.U;
+    return s;
 }
 
 // Per-(row, tap) sampling record kept in shared memory for the current group:
 // the four bilinear weights times the mask (zero for neighbours outside the
-// map), as bf16 for the mixed-precision blend, and the pixel index of the
-// top-left neighbour.
-struct __align__(8) TapW {
+// map) as bf16 pairs, the pixel index of the top-left neighbour, and a mask of
+// the neighbours to read (bit c for neighbour c = 2*dy + dx: inside the map
+// and of nonzero weight). Neighbours not read take their values from a zero
+// buffer instead.
+struct __align__(16) TapRec {
     uint32_t w01_00;  // lo: w00, hi: w01
     uint32_t w11_10;  // lo: w10, hi: w11
+    int base;         // (b*H + y0)*W + x0
+    uint32_t vmask;
 };
+
+// 32 zero bytes: the source of every neighbour that is not read.
+__device__ __align__(32) uint32_t g_zero_slice[8];
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&t);
 }
 
-// acc[0..7] += w * (8 bf16 of v), f32 accumulation of bf16 products.
-__device__ __forceinline__ void fma8(float (&acc)[8], const uint4& v, uint32_t wpair, bool hi_half) {
-    uint16_t w = hi_half ? (uint16_t)(wpair >> 16) : (uint16_t)(wpair & 0xFFFFu);
-    asm("{\n\t.reg .b16 a0, a1, a2, a3, a4, a5, a6, a7;\n\t"
-        "mov.b32 {a0, a1}, %8;\n\t"
-        "mov.b32 {a2, a3}, %9;\n\t"
-        "mov.b32 {a4, a5}, %10;\n\t"
-        "mov.b32 {a6, a7}, %11;\n\t"
-        "fma.rn.f32.bf16 %0, a0, %12, %0;\n\t"
-        "fma.rn.f32.bf16 %1, a1, %12, %1;\n\t"
-        "fma.rn.f32.bf16 %2, a2, %12, %2;\n\t"
-        "fma.rn.f32.bf16 %3, a3, %12, %3;\n\t"
-        "fma.rn.f32.bf16 %4, a4, %12, %4;\n\t"
-        "fma.rn.f32.bf16 %5, a5, %12, %5;\n\t"
-        "fma.rn.f32.bf16 %6, a6, %12, %6;\n\t"
-        "fma.rn.f32.bf16 %7, a7, %12, %7;\n\t}"
-        : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3]), "+f"(acc[4]), "+f"(acc[5]), "+f"(acc[6]),
-          "+f"(acc[7])
-        : "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "h"(w));
-}
-
-// Modulated bilinear blend of one row's four neighbour vectors (8 channels
-// each) into 8 bf16 values. DCN_FWD_BLEND == 1: packed bf16x2 FMAs (each
-// partial sum rounded to bf16); 0: bf16 products accumulated in f32.
-__device__ __forceinline__ uint4 blend4(const uint4 (&v)[4], const TapW& tw) {
-#if DCN_FWD_BLEND
-    const uint32_t w00 = __byte_perm(tw.w01_00, 0, 0x1010), w01 = __byte_perm(tw.w01_00, 0, 0x3232);
-    const uint32_t w10 = __byte_perm(tw.w11_10, 0, 0x1010), w11 = __byte_perm(tw.w11_10, 0, 0x3232);
-    const uint32_t* a0 = reinterpret_cast<const uint32_t*>(&v[0]);
-    const uint32_t* a1 = reinterpret_cast<const uint32_t*>(&v[1]);
-    const uint32_t* a2 = reinterpret_cast<const uint32_t*>(&v[2]);
-    const uint32_t* a3 = reinterpret_cast<const uint32_t*>(&v[3]);
-    uint32_t r[4];
+// Modulated bilinear blend of one sample's four neighbour slices (16 channels
+// each, as bf16 pairs) into 16 bf16 values: packed bf16x2 products and sums,
+// each partial result rounded to bf16.
+__device__ __forceinline__ void blend16(uint32_t (&r)[8], const uint32_t (&v)[4][8], uint32_t w01_00,
+                                        uint32_t w11_10) {
+    const uint32_t w00 = __byte_perm(w01_00, 0, 0x1010), w01 = __byte_perm(w01_00, 0, 0x3232);
+    const uint32_t w10 = __byte_perm(w11_10, 0, 0x1010), w11 = __byte_perm(w11_10, 0, 0x3232);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < 8; ++q) {
         asm("{\n\t"
             "mul.rn.bf16x2 %0, %1, %5;\n\t"
             "fma.rn.bf16x2 %0, %2, %6, %0;\n\t"
             "fma.rn.bf16x2 %0, %3, %7, %0;\n\t"
             "fma.rn.bf16x2 %0, %4, %8, %0;\n\t}"
             : "=&r"(r[q])
-            : "r"(a0[q]), "r"(a1[q]), "r"(a2[q]), "r"(a3[q]), "r"(w00), "r"(w01), "r"(w10), "r"(w11));
+            : "r"(v[0][q]), "r"(v[1][q]), "r"(v[2][q]), "r"(v[3][q]), "r"(w00), "r"(w01), "r"(w10), "r"(w11));
     }
-    return make_uint4(r[0], r[1], r[2], r[3]);
-#else
-    float acc[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-    fma8(acc, v[0], tw.w01_00, false);
-    fma8(acc, v[1], tw.w01_00, true);
-    fma8(acc, v[2], tw.w11_10, false);
-    fma8(acc, v[3], tw.w11_10, true);
-    return make_uint4(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]), pack_bf16(acc[4], acc[5]),
-                      pack_bf16(acc[6], acc[7]));
-#endif
+}
+
+// One neighbour's 16-channel slice. WIDE: a single 32-byte load from p;
+// otherwise two 16-byte loads, the upper half from p_hi.
+template <bool WIDE>
+__device__ __forceinline__ void load_slice(uint32_t (&v)[8], const uint8_t* p, const uint8_t* p_hi) {
+    if (WIDE) {
+        ptx::ldg_v8(v, p);
+    } else {
+        const uint4 lo = ptx::ldg_v4(p), hi = ptx::ldg_v4(p_hi);
+        v[0] = lo.x, v[1] = lo.y, v[2] = lo.z, v[3] = lo.w;
+        v[4] = hi.x, v[5] = hi.y, v[6] = hi.z, v[7] = hi.w;
+    }
 }
 
 // GEMM rows enumerate output pixels strip by strip: each image is cut into
@@ -187,59 +209,131 @@ __device__ __forceinline__ int strip_to_raster(int idx, const FwdArgs& a) {
 }
 
 // Partial tiles (float32) live in the workspace as [cta][slot][bn_total/32][8][BM][4]:
-// slot 0 holds a CTA's first segment, slot 1 its last; within a tile, the four
+// slot 0 holds a CTA's first segment in unit order, slot 1 its last; within a tile, the four
 // consecutive columns 4q..4q+3 of a 32-column block are stored for all 128
 // rows side by side, so each warp-wide 16-byte access covers 512 contiguous bytes.
-__device__ __forceinline__ const float* partial_base(const FwdArgs& a, int c, long long tu0, int row) {
-    const int slot = (unit_begin(c, a) >= tu0) ? 0 : 1;
+__device__ __forceinline__ const float* partial_base(const FwdArgs& a, const long long* starts, int c, long long tu0,
+                                                    int row) {
+    const int slot = (starts[c] >= tu0) ? 0 : 1;
     return a.partials + ((size_t)c * 2 + slot) * BM * a.bn_total + (size_t)row * 4;
 }
 
-// v[0..31] += partial columns cc..cc+31 of this row (src from partial_base).
-__device__ __forceinline__ void add_partial32(float (&v)[32], const float* src, int cc) {
+// r[0..31] (float bits) += partial columns cc..cc+31 of this row (src from partial_base).
+__device__ __forceinline__ void add_partial32(uint32_t (&r)[32], const float* src, int cc) {
     float4 f[8];
     const float* b = src + (size_t)(cc >> 5) * 8 * BM * 4;
 #pragma unroll
     for (int q = 0; q < 8; ++q) f[q] = ptx::ldcg_f4(b + q * BM * 4);
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-        v[4 * q] += f[q].x;
-        v[4 * q + 1] += f[q].y;
-        v[4 * q + 2] += f[q].z;
-        v[4 * q + 3] += f[q].w;
+        r[4 * q] = __float_as_uint(__uint_as_float(r[4 * q]) + f[q].x);
+        r[4 * q + 1] = __float_as_uint(__uint_as_float(r[4 * q + 1]) + f[q].y);
+        r[4 * q + 2] = __float_as_uint(__uint_as_float(r[4 * q + 2]) + f[q].z);
+        r[4 * q + 3] = __float_as_uint(__uint_as_float(r[4 * q + 3]) + f[q].w);
     }
 }
 
 // As add_partial32, from a partial tile staged in shared memory.
-__device__ __forceinline__ void add_partial32_smem(float (&v)[32], const float* src, int cc) {
+__device__ __forceinline__ void add_partial32_smem(uint32_t (&r)[32], const float* src, int cc) {
     const float* b = src + (size_t)(cc >> 5) * 8 * BM * 4;
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
         const float4 f = *reinterpret_cast<const float4*>(b + q * BM * 4);
-        v[4 * q] += f.x;
-        v[4 * q + 1] += f.y;
-        v[4 * q + 2] += f.z;
-        v[4 * q + 3] += f.w;
+        r[4 * q] = __float_as_uint(__uint_as_float(r[4 * q]) + f.x);
+        r[4 * q + 1] = __float_as_uint(__uint_as_float(r[4 * q + 1]) + f.y);
+        r[4 * q + 2] = __float_as_uint(__uint_as_float(r[4 * q + 2]) + f.z);
+        r[4 * q + 3] = __float_as_uint(__uint_as_float(r[4 * q + 3]) + f.w);
     }
 }
 
-// y[row, n0 + cc .. n0 + cc + 31] = v + bias, as bf16 (columns < ncols).
-__device__ __forceinline__ void store_row32(bf16* yrow, int cc, int ncols, float (&v)[32], const bf16* bias, int n0) {
-    if (bias) {
+// y[row, cc .. cc + 31] (columns < ncols of the tile) = r (float bits) + bias, as bf16;
+// sb: the tile's bias in shared memory, or null. Overwrites r.
+__device__ __forceinline__ void store_row32(bf16* yrow, int cc, int ncols, uint32_t (&r)[32], const float* sb) {
+    if (sb) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-            if (cc + e < ncols) v[e] += __bfloat162float(bias[n0 + cc + e]);
+        for (int q = 0; q < 8; ++q) {
+            const float4 b = *reinterpret_cast<const float4*>(sb + cc + 4 * q);
+            r[4 * q] = __float_as_uint(__uint_as_float(r[4 * q]) + b.x);
+            r[4 * q + 1] = __float_as_uint(__uint_as_float(r[4 * q + 1]) + b.y);
+            r[4 * q + 2] = __float_as_uint(__uint_as_float(r[4 * q + 2]) + b.z);
+            r[4 * q + 3] = __float_as_uint(__uint_as_float(r[4 * q + 3]) + b.w);
+        }
     }
     if (cc + 32 <= ncols) {
         uint4* dst = reinterpret_cast<uint4*>(yrow + cc);
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-            dst[q] = make_uint4(pack_bf16(v[8 * q], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
-                                pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7]));
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t* w = r + 8 * q;
+            dst[q] = make_uint4(pack_bf16(__uint_as_float(w[0]), __uint_as_float(w[1])),
+                                pack_bf16(__uint_as_float(w[2]), __uint_as_float(w[3])),
+                                pack_bf16(__uint_as_float(w[4]), __uint_as_float(w[5])),
+                                pack_bf16(__uint_as_float(w[6]), __uint_as_float(w[7])));
+        }
     } else {
 #pragma unroll
         for (int e = 0; e < 32; ++e)
-            if (cc + e < ncols) yrow[cc + e] = __float2bfloat16_rn(v[e]);
+            if (cc + e < ncols) yrow[cc + e] = __float2bfloat16_rn(__uint_as_float(r[e]));
+    }
+}
+
+// Walks this warp's 32 TMEM lanes over columns [0, ncols) in blocks of 32,
+// calling f(r, cc) on each block; PIPE: while the next block's load is in
+// flight (twice the registers). ncols is warp-uniform (the loads are
+// warp-collective).
+template <bool PIPE, typename F>
+__device__ __forceinline__ void tmem_rows(uint32_t taddr, int ncols, F&& f) {
+    if (!PIPE) {
+        for (int cc = 0; cc < ncols; cc += 32) {
+            uint32_t r[32];
+            ptx::tmem_ld32_issue(taddr + cc, r);
+            ptx::tmem_wait_ld(r);
+            f(r, cc);
+        }
+        return;
+    }
+    uint32_t ra[32], rb[32];
+    ptx::tmem_ld32_issue(taddr, ra);
+    ptx::tmem_wait_ld(ra);
+    for (int cc = 0; cc < ncols; cc += 64) {
+        const bool has_b = cc + 32 < ncols;
+        if (has_b) ptx::tmem_ld32_issue(taddr + cc + 32, rb);
+        f(ra, cc);
+        if (!has_b) break;
+        ptx::tmem_wait_ld(rb);
+        const bool has_a = cc + 64 < ncols;
+        if (has_a) ptx::tmem_ld32_issue(taddr + cc + 64, ra);
+        f(rb, cc + 32);
+        if (has_a) ptx::tmem_wait_ld(ra);
+    }
+}
+
+// y row = bias + the tile's partial sums in contributor order c_lo..c_hi, this
+// CTA's own taken from its TMEM accumulator and every other one from `part(c)`
+// (a row pointer in partial_base layout; in_smem: staged in shared memory).
+// The fixed order makes the result independent of which CTA finishes the tile.
+template <typename P>
+__device__ __forceinline__ void combine_rows(uint32_t taddr, int ncols, int c_lo, int c_hi, int cta, bool in_smem,
+                                             P&& part, bf16* yrow, bool store, const float* sb) {
+    for (int cc = 0; cc < ncols; cc += 32) {
+        uint32_t acc[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) acc[e] = 0u;
+        for (int c = c_lo; c < cta; ++c) {
+            if (in_smem) add_partial32_smem(acc, part(c), cc);
+            else add_partial32(acc, part(c), cc);
+        }
+        {
+            uint32_t r[32];
+            ptx::tmem_ld32_issue(taddr + cc, r);
+            ptx::tmem_wait_ld(r);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) acc[e] = __float_as_uint(__uint_as_float(acc[e]) + __uint_as_float(r[e]));
+        }
+        for (int c = cta + 1; c <= c_hi; ++c) {
+            if (in_smem) add_partial32_smem(acc, part(c), cc);
+            else add_partial32(acc, part(c), cc);
+        }
+        if (store) store_row32(yrow, cc, ncols, acc, sb);
     }
 }
 
@@ -266,6 +360,77 @@ __device__ __forceinline__ Chunk chunk_of(int u, const FwdArgs& a) {
     return c;
 }
 
+// Sampling records of tile row `row` for the taps of `part` (0..2: a third of
+// the taps each; -1: all), for group g of m-tile mt:
+// offsets and mask of the row's output pixel, split into integer corner and
+// fractional weights (the bilinear kernel of the DCNv2 sampling equation, a
+// neighbour outside the map contributing zero), written to recs[row*K2 + tap].
+// The loads of up to REC_BATCH taps are in flight together.
+constexpr int REC_BATCH = 9;
+__device__ __forceinline__ void build_records(const FwdArgs& a, int mt, int g, int row, int part, TapRec* recs,
+                                              const int2* s_tap) {
+    const Shape& s = a.s;
+    const int plane = s.Ho * s.Wo;
+    const int pr = strip_to_raster(mt * BM + row, a);
+    int pix = -1, bb = 0, oy = 0, ox = 0;
+    if (pr >= 0) {
+        bb = pr / plane;
+        pix = pr - bb * plane;
+        const int ho = pix / s.Wo, wo = pix - ho * s.Wo;
+        oy = ho * s.stride - s.pad;
+        ox = wo * s.stride - s.pad;
+    }
+    const bf16* offp = a.off + ((size_t)bb * 2 * s.G * s.K2 + (size_t)g * 2 * s.K2) * plane + (pix < 0 ? 0 : pix);
+    const bf16* mp = a.mask ? a.mask + ((size_t)bb * s.G * s.K2 + (size_t)g * s.K2) * plane + (pix < 0 ? 0 : pix) : nullptr;
+    const int tp_lo = part < 0 ? 0 : s.K2 * part / 3, tp_hi = part < 0 ? s.K2 : s.K2 * (part + 1) / 3;
+    for (int tp0 = tp_lo; tp0 < tp_hi; tp0 += REC_BATCH) {
+        float dy[REC_BATCH], dx[REC_BATCH], mk[REC_BATCH];
+#pragma unroll
+        for (int b = 0; b < REC_BATCH; ++b) {
+            const int tp = tp0 + b;
+            dy[b] = dx[b] = 0.f;
+            mk[b] = 1.f;
+            if (pix >= 0 && tp < tp_hi) {
+                dy[b] = __bfloat162float(offp[(size_t)(2 * tp) * plane]);
+                dx[b] = __bfloat162float(offp[(size_t)(2 * tp + 1) * plane]);
+                if (mp) mk[b] = __bfloat162float(mp[(size_t)tp * plane]);
+            }
+        }
+#pragma unroll
+        for (int b = 0; b < REC_BATCH; ++b) {
+            const int tp = tp0 + b;
+            if (tp >= tp_hi) break;
+            float w00 = 0.f, w01 = 0.f, w10 = 0.f, w11 = 0.f;
+            int base = 0;
+            if (pix >= 0) {
+                const int2 to = s_tap[tp];
+                int y0, x0;
+                float ly, lx;
+                split_coord(oy + to.x, dy[b], y0, ly);
+                split_coord(ox + to.y, dx[b], x0, lx);
+                const bool v00 = inside(s, y0, x0), v01 = inside(s, y0, x0 + 1);
+                const bool v10 = inside(s, y0 + 1, x0), v11 = inside(s, y0 + 1, x0 + 1);
+                w00 = v00 ? (1.f - ly) * (1.f - lx) * mk[b] : 0.f;
+                w01 = v01 ? (1.f - ly) * lx * mk[b] : 0.f;
+                w10 = v10 ? ly * (1.f - lx) * mk[b] : 0.f;
+                w11 = v11 ? ly * lx * mk[b] : 0.f;
+                if (v00 | v01 | v10 | v11) base = (bb * s.H + y0) * s.W + x0;
+            }
+            TapRec rc;
+            rc.w01_00 = pack_bf16(w00, w01);
+            rc.w11_10 = pack_bf16(w10, w11);
+            rc.base = base;
+            // read a neighbour only when it is inside the map and its bf16 weight is nonzero
+            rc.vmask = ((rc.w01_00 & 0x7FFFu) ? 1u : 0u) | ((rc.w01_00 & 0x7FFF0000u) ? 2u : 0u) |
+                       ((rc.w11_10 & 0x7FFFu) ? 4u : 0u) | ((rc.w11_10 & 0x7FFF0000u) ? 8u : 0u);
+            recs[row * s.K2 + tp] = rc;
+        }
+    }
+}
+
+// WIDE: x is 32-byte aligned and Cin, Cg are multiples of 16, so a lane's
+// 16-channel slice is one 32-byte load.
+template <bool WIDE>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     dcn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const FwdArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -275,10 +440,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     uint8_t* sA = smem;
     uint8_t* sB = smem + a.b_off;
-    TapW* s_w = reinterpret_cast<TapW*>(smem + a.info_off);
-    int* s_base = reinterpret_cast<int*>(smem + a.base_off);
-    int4* s_row = reinterpret_cast<int4*>(smem + a.row_off);   // per tile row: in-plane pixel, b, row/col origin
-    int2* s_tap = reinterpret_cast<int2*>(s_row + BM);          // per tap: (i*dil, j*dil)
+    TapRec* s_rec = reinterpret_cast<TapRec*>(smem + a.info_off);  // two buffers of BM * K2 records
+    int2* s_tap = reinterpret_cast<int2*>(smem + a.row_off);        // per tap: (i*dil, j*dil)
+    long long* s_starts = reinterpret_cast<long long*>(s_tap + 32);   // [ctas + 1] first unit of each CTA
+    float* s_bias = reinterpret_cast<float*>(s_starts + MAX_CTAS + 2);  // [2][512] bias of a tile's columns
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + a.bar_off);
     // barrier slots
     uint64_t* full_a = bars;
@@ -287,16 +452,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint64_t* acc_full = bars + 3 * MAX_STAGES;
     uint64_t* acc_empty = acc_full + 2;
     uint64_t* drain = acc_empty + 2;
-    uint64_t* prod_bar = drain + 1;
-    uint64_t* epi_bar = prod_bar + 1;
+    uint64_t* rec_full = drain + 1;    // [2] records of an epoch built
+    uint64_t* rec_empty = rec_full + 2;  // [2] every producer warp done with an epoch's records
+    uint64_t* rec0_bar = rec_empty + 2;  // the first epoch's records, built by all warps
+    uint64_t* epi_bar = rec0_bar + 1;
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(epi_bar + 1);
     volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
-    volatile int* s_last = s_abort + 1;
+    volatile int* s_last = s_abort + 1;  // [2], by segment parity
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < a.stages; ++i) {
-            // a stage is full when its producer group's warps and the weight TMA have both arrived
-            ptx::mbar_init(ptx::smem_u32(&full_a[i]), NUM_PROD_WARPS / GROUPS + 1);
+            // a stage is full when every producer warp and the weight TMA have arrived
+            ptx::mbar_init(ptx::smem_u32(&full_a[i]), NUM_PROD_WARPS + 1);
             ptx::mbar_init(ptx::smem_u32(&empty[i]), 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -305,16 +472,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         ptx::mbar_init(ptx::smem_u32(drain), 1);
         ptx::mbar_init(ptx::smem_u32(tail_bar), 1);
-        ptx::mbar_init(ptx::smem_u32(prod_bar), NUM_PROD_WARPS);
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(ptx::smem_u32(&rec_full[i]), 4);
+            ptx::mbar_init(ptx::smem_u32(&rec_empty[i]), NUM_PROD_WARPS);
+        }
+        ptx::mbar_init(ptx::smem_u32(rec0_bar), NUM_PROD_WARPS + 4);
         ptx::mbar_init(ptx::smem_u32(epi_bar), 4);
         *s_abort = 0;
-        *s_last = 0;
+        s_last[0] = s_last[1] = 0;
         ptx::fence_mbar_init();
     }
     if (threadIdx.x < s.K2) {
         const int i = threadIdx.x / s.K;
         s_tap[threadIdx.x] = make_int2(i * s.dil, (threadIdx.x - i * s.K) * s.dil);
     }
+    for (int c = threadIdx.x; c <= a.ctas; c += NUM_THREADS) s_starts[c] = unit_begin(c, a);
     if (warp == MMA_WARP) {
         ptx::tmem_alloc(ptx::smem_u32(s_tmem), (uint32_t)a.tmem_cols);
         ptx::tmem_relinquish();
@@ -326,194 +498,132 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t tmem_base = *s_tmem;
 
     const int cta = blockIdx.x;
-    const long long ubeg = unit_begin(cta, a), uend = unit_begin(cta + 1, a);
+    const long long ubeg = s_starts[cta], uend = s_starts[cta + 1];
+    const SegList L = seg_list(ubeg, uend, a.U);
     if (warp >= PROD_WARP0) {
         // ------------------------------------------------------ producers --
-        // Two groups of producer warps take alternate chunks, so that one group
-        // blends while the other's loads are in flight. Within a group, 8 lanes
-        // cover the 128-byte channel slice of one row (one 16-byte vector each).
+        // All producer warps work on every chunk: 4 lanes cover the 128-byte
+        // channel slice of one row (16 channels each), and a thread owns rows r0
+        // and r0 + ROW_STEP, which share one swizzle phase. The loads of the next
+        // chunk's row are issued right after this chunk's row is blended, so they
+        // are in flight while the other row is blended and stored.
         const int ptid = threadIdx.x - PROD_WARP0 * 32;
-        const int plane = s.Ho * s.Wo;
-        const int grp = ptid / GROUP_THREADS;
-        const int gtid = ptid - grp * GROUP_THREADS;
-        const int j = gtid & 7, r0 = gtid >> 3;
-        int stage = 0;
-        uint32_t phase = 0, pphase = 0;
-        int n = 0;  // chunk sequence number within this CTA
+        const int j4 = ptid % LANES_PER_ROW, r0 = ptid / LANES_PER_ROW;
+        const int r1 = r0 + ROW_STEP;
+        const uint32_t swz0 = (uint32_t)(((2 * j4) ^ (r0 & 7)) << 4);      // 16-byte chunk 2*j4 of the row
+        const uint32_t swz1 = (uint32_t)(((2 * j4 + 1) ^ (r0 & 7)) << 4);  // chunk 2*j4 + 1
+        const long long cin2 = (long long)s.Cin * 2, rp2 = (long long)s.W * cin2;
+        const uint8_t* zb = reinterpret_cast<const uint8_t*>(g_zero_slice);
         bool ok = true;
-        for (long long u = ubeg; u < uend && ok;) {
-            const int t = (int)(u / a.U);
-            const int k0 = (int)(u - (long long)t * a.U);
-            const int k1 = (int)min((long long)a.U, uend - (long long)t * a.U);
-            const int mt = t / a.n_tiles;
-            int cur_g = -1;
-            Chunk ch = chunk_of(k0, a);
-            for (int k = k0; k < k1 && ok; ++k) {
-                if (ch.g != cur_g) {
-                    // every producer is done with the previous records before they are overwritten
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(prod_bar));
-                    if (!ptx::mbar_wait(ptx::smem_u32(prod_bar), pphase, s_abort, a.status, WAIT_LIMIT)) {
-                        ok = false;
-                        break;
-                    }
-                    pphase ^= 1;
-                    if (cur_g < 0) {
-                        // new tile: pixel coordinates of its rows
-                        if (ptid < BM) {
-                            const int pr = strip_to_raster(mt * BM + ptid, a);
-                            int4 ri = make_int4(-1, 0, 0, 0);
-                            if (pr >= 0) {
-                                const int bb = pr / plane, pix = pr - bb * plane;
-                                const int ho = pix / s.Wo, wo = pix - ho * s.Wo;
-                                ri = make_int4(pix, bb, ho * s.stride - s.pad, wo * s.stride - s.pad);
-                            }
-                            s_row[ptid] = ri;
-                        }
-                        __syncwarp();
-                        if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(prod_bar));
-                        if (!ptx::mbar_wait(ptx::smem_u32(prod_bar), pphase, s_abort, a.status, WAIT_LIMIT)) {
-                            ok = false;
-                            break;
-                        }
-                        pphase ^= 1;
-                    }
-                    // sampling records of every (row, tap) of this tile for group ch.g; each
-                    // thread issues the loads of all its entries before using any of them
-                    for (int e0 = 0; e0 < BM * s.K2; e0 += INFO_BATCH * NUM_PROD_THREADS) {
-                        float dy[INFO_BATCH], dx[INFO_BATCH], mk[INFO_BATCH];
+        // the first epoch's records are built by all warps together
+        if (L.ns > 0) {
+            const Seg s0 = seg_at(L, 0);
+            build_records(a, s0.t / a.n_tiles, s0.k0 / (a.nq * s.K2), ptid & (BM - 1), 1 + (ptid >> 7), s_rec, s_tap);
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(rec0_bar));
+            ok = ptx::mbar_wait(ptx::smem_u32(rec0_bar), 0, s_abort, a.status, WAIT_LIMIT);
+        }
+        // issue cursor: the chunk whose loads are issued next
+        int isi = 0, ik = 0, ik1 = 0, icur_g = -1, iepoch = 0;
+        Chunk ich{0, 0, 0};
+        const TapRec* irecs = s_rec;
+        if (L.ns > 0) {
+            const Seg s0 = seg_at(L, 0);
+            ik = s0.k0;
+            ik1 = s0.k1;
+            ich = chunk_of(ik, a);
+            icur_g = ich.g;
+        }
+        // loads of row `row` of the cursor chunk into v, its weights into w
+        auto issue = [&](uint32_t(&v)[4][8], uint32_t(&w)[2], int row) {
+            const int cg = ich.q * BK + j4 * SLICE;  // first channel of this lane's slice, within the group
+            const uint32_t cmask = cg < s.Cg ? 0xFu : 0u;
+            const bool hi_ok = cg + 8 < s.Cg;      // upper 8 channels present (narrow loads only)
+            const uint8_t* xc = reinterpret_cast<const uint8_t*>(a.x + ich.g * s.Cg + cg);
+            const TapRec rc = irecs[row * s.K2 + ich.tap];
+            w[0] = rc.w01_00;
+            w[1] = rc.w11_10;
+            const uint32_t vm = rc.vmask & cmask;
+            const uint8_t* p = xc + (long long)rc.base * cin2;
+            const uint8_t* pc[4] = {p, p + cin2, p + rp2, p + rp2 + cin2};
 #pragma unroll
-                        for (int b = 0; b < INFO_BATCH; ++b) {
-                            const int e = e0 + b * NUM_PROD_THREADS + ptid;
-                            const int tp = e >> 7, row = e & (BM - 1);
-                            dy[b] = dx[b] = 0.f;
-                            mk[b] = 1.f;
-                            if (e < BM * s.K2) {
-                                const int4 ri = s_row[row];
-                                if (ri.x >= 0) {
-                                    const size_t ob =
-                                        ((size_t)ri.y * 2 * s.G * s.K2 + (size_t)ch.g * 2 * s.K2 + 2 * tp) * plane + ri.x;
-                                    dy[b] = __bfloat162float(a.off[ob]);
-                                    dx[b] = __bfloat162float(a.off[ob + plane]);
-                                    if (a.mask)
-                                        mk[b] = __bfloat162float(
-                                            a.mask[((size_t)ri.y * s.G * s.K2 + (size_t)ch.g * s.K2 + tp) * plane + ri.x]);
-                                }
-                            }
-                        }
-#pragma unroll
-                        for (int b = 0; b < INFO_BATCH; ++b) {
-                            const int e = e0 + b * NUM_PROD_THREADS + ptid;
-                            if (e >= BM * s.K2) continue;
-                            const int tp = e >> 7, row = e & (BM - 1);
-                            const int4 ri = s_row[row];
-                            float w00 = 0.f, w01 = 0.f, w10 = 0.f, w11 = 0.f;
-                            int base = 0;
-                            if (ri.x >= 0) {
-                                const int2 to = s_tap[tp];
-                                int y0, x0;
-                                float ly, lx;
-                                split_coord(ri.z + to.x, dy[b], y0, ly);
-                                split_coord(ri.w + to.y, dx[b], x0, lx);
-                                const bool v00 = inside(s, y0, x0), v01 = inside(s, y0, x0 + 1);
-                                const bool v10 = inside(s, y0 + 1, x0), v11 = inside(s, y0 + 1, x0 + 1);
-                                w00 = v00 ? (1.f - ly) * (1.f - lx) * mk[b] : 0.f;
-                                w01 = v01 ? (1.f - ly) * lx * mk[b] : 0.f;
-                                w10 = v10 ? ly * (1.f - lx) * mk[b] : 0.f;
-                                w11 = v11 ? ly * lx * mk[b] : 0.f;
-                                if (v00 | v01 | v10 | v11) base = (ri.y * s.H + y0) * s.W + x0;
-                            }
-                            TapW tw;
-                            tw.w01_00 = pack_bf16(w00, w01);
-                            tw.w11_10 = pack_bf16(w10, w11);
-                            s_w[row * s.K2 + tp] = tw;
-                            s_base[row * s.K2 + tp] = base;
-                        }
-                    }
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(prod_bar));
-                    if (!ptx::mbar_wait(ptx::smem_u32(prod_bar), pphase, s_abort, a.status, WAIT_LIMIT)) {
-                        ok = false;
-                        break;
-                    }
-                    pphase ^= 1;
-                    cur_g = ch.g;
-                }
-                if ((n % GROUPS) == grp) {
-                    if (!ptx::mbar_wait(ptx::smem_u32(&empty[stage]), phase ^ 1, s_abort, a.status, WAIT_LIMIT)) {
-                        ok = false;
-                        break;
-                    }
-                    const int cg = ch.q * BK + j * 8;  // channel within the group
-                    const bool cval = cg < s.Cg;
-                    const bf16* xc = a.x + ch.g * s.Cg + cg;
-                    const long long rowpitch = (long long)s.W * s.Cin;
-                    const uint32_t a_stage = ptx::smem_u32(sA + stage * A_STAGE_BYTES);
-#pragma unroll
-                    for (int bt = 0; bt < ROWS_PER_THREAD / 4; ++bt) {
-                        uint4 v[4][4];
-                        TapW tw[4];
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int row = r0 + ROW_STEP * (4 * bt + i);
-                            tw[i] = s_w[row * s.K2 + ch.tap];
-                            const int base = s_base[row * s.K2 + ch.tap];
-                            const bf16* pb = xc + (long long)base * s.Cin;
-                            uint32_t m = ((tw[i].w01_00 & 0xFFFFu) ? 1u : 0u) | ((tw[i].w01_00 >> 16) ? 2u : 0u) |
-                                         ((tw[i].w11_10 & 0xFFFFu) ? 4u : 0u) | ((tw[i].w11_10 >> 16) ? 8u : 0u);
-                            if (!cval) m = 0;
-                            ptx::ldg4_pred(v[i], pb, pb + s.Cin, pb + rowpitch, pb + rowpitch + s.Cin, m);
-                        }
-                        if (bt == 0 && PREFETCH) {
-                            // Pull the neighbours of this group's next chunk into L1 while this one
-                            // is blended: lane j takes row r0 + ROW_STEP*j, all four corners.
-                            Chunk nx = ch;
-                            int kn = k;
-                            for (int d = 0; d < GROUPS; ++d) {
-                                ++kn;
-                                if (++nx.tap == s.K2) {
-                                    nx.tap = 0;
-                                    if (++nx.q == a.nq) {
-                                        nx.q = 0;
-                                        ++nx.g;
-                                    }
-                                }
-                            }
-                            const int cgn = nx.q * BK;
-                            if (kn < k1 && nx.g == ch.g && cgn < s.Cg && j < ROWS_PER_THREAD) {
-                                const int row = r0 + ROW_STEP * j;
-                                const TapW tn = s_w[row * s.K2 + nx.tap];
-                                const bf16* pn = a.x + (long long)s_base[row * s.K2 + nx.tap] * s.Cin + ch.g * s.Cg + cgn;
-                                if (tn.w01_00 & 0xFFFFu) ptx::prefetch_l1(pn);
-                                if (tn.w01_00 >> 16) ptx::prefetch_l1(pn + s.Cin);
-                                if (tn.w11_10 & 0xFFFFu) ptx::prefetch_l1(pn + rowpitch);
-                                if (tn.w11_10 >> 16) ptx::prefetch_l1(pn + rowpitch + s.Cin);
-                            }
-                        }
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int row = r0 + ROW_STEP * (4 * bt + i);
-                            ptx::sts_v4(a_stage + row * 128 + ((j ^ (row & 7)) << 4), blend4(v[i], tw[i]));
-                        }
-                    }
-                    ptx::fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&full_a[stage]));
-                }
-                if (++stage == a.stages) {
-                    stage = 0;
-                    phase ^= 1;
-                }
-                ++n;
-                if (++ch.tap == s.K2) {
-                    ch.tap = 0;
-                    if (++ch.q == a.nq) {
-                        ch.q = 0;
-                        ++ch.g;
-                    }
+            for (int c = 0; c < 4; ++c) {
+                const bool rd = (vm >> c) & 1u;
+                load_slice<WIDE>(v[c], rd ? pc[c] : zb, (rd && hi_ok) ? pc[c] + 16 : zb);
+            }
+        };
+        // moves the cursor to the next chunk; at a new epoch (tile or group) releases the
+        // previous records and waits for the new ones
+        auto advance = [&]() -> bool {
+            ++ik;
+            if (++ich.tap == s.K2) {
+                ich.tap = 0;
+                if (++ich.q == a.nq) {
+                    ich.q = 0;
+                    ++ich.g;
                 }
             }
-            u = (long long)t * a.U + k1;
+            if (ik == ik1) {
+                const Seg sn = seg_at(L, ++isi);
+                ik = sn.k0;
+                ik1 = sn.k1;
+                ich = chunk_of(ik, a);
+                icur_g = -1;
+            }
+            if (ich.g != icur_g) {
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&rec_empty[iepoch & 1]));
+                ++iepoch;
+                const int b = iepoch & 1;
+                const uint32_t par = (uint32_t)(b ? (iepoch >> 1) : ((iepoch >> 1) - 1)) & 1u;
+                if (!ptx::mbar_wait(ptx::smem_u32(&rec_full[b]), par, s_abort, a.status, WAIT_LIMIT)) return false;
+                irecs = s_rec + b * BM * s.K2;
+                icur_g = ich.g;
+            }
+            return true;
+        };
+        const long long total = uend - ubeg;  // chunks of this CTA
+        uint32_t va[4][8], vb[4][8], wa[2], wb[2];
+        if (ok && total > 0) {
+            issue(va, wa, r0);
+            issue(vb, wb, r1);
+        }
+        int stage = 0;
+        uint32_t phase = 0;
+        for (long long n = 0; n < total && ok; ++n) {
+            if (!ptx::mbar_wait(ptx::smem_u32(&empty[stage]), phase ^ 1, s_abort, a.status, WAIT_LIMIT)) {
+                ok = false;
+                break;
+            }
+            const uint32_t a_stage = ptx::smem_u32(sA + stage * A_STAGE_BYTES);
+            const bool more = n + 1 < total;
+            {
+                uint32_t r[8];
+                blend16(r, va, wa[0], wa[1]);
+                ptx::sts_v4(a_stage + r0 * 128 + swz0, make_uint4(r[0], r[1], r[2], r[3]));
+                ptx::sts_v4(a_stage + r0 * 128 + swz1, make_uint4(r[4], r[5], r[6], r[7]));
+            }
+            if (more) {
+                if (!advance()) {
+                    ok = false;
+                    break;
+                }
+                issue(va, wa, r0);
+            }
+            {
+                uint32_t r[8];
+                blend16(r, vb, wb[0], wb[1]);
+                ptx::sts_v4(a_stage + r1 * 128 + swz0, make_uint4(r[0], r[1], r[2], r[3]));
+                ptx::sts_v4(a_stage + r1 * 128 + swz1, make_uint4(r[4], r[5], r[6], r[7]));
+            }
+            if (more) issue(vb, wb, r1);
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&full_a[stage]));
+            if (++stage == a.stages) {
+                stage = 0;
+                phase ^= 1;
+            }
         }
     } else if (warp == TMA_WARP) {
         // ------------------------------------------------------- weights --
@@ -523,12 +633,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t issued = 0, issued_par = 0;  // per stage: a load was issued / parity of the last one
             const uint32_t bytes = (uint32_t)(a.nsub * a.box_rows * BK * 2);
             bool ok = true;
-            for (long long u = ubeg; u < uend && ok;) {
-                const int t = (int)(u / a.U);
-                const int k0 = (int)(u - (long long)t * a.U);
-                const int k1 = (int)min((long long)a.U, uend - (long long)t * a.U);
-                const int n0 = (t % a.n_tiles) * a.bn_total;
-                for (int k = k0; k < k1; ++k) {
+            for (int si = 0; si < L.ns && ok; ++si) {
+                const Seg sg = seg_at(L, si);
+                const int n0 = (sg.t % a.n_tiles) * a.bn_total;
+                for (int k = sg.k0; k < sg.k1; ++k) {
                     const Chunk ch = chunk_of(k, a);
                     if (!ptx::mbar_wait(ptx::smem_u32(&empty[stage]), phase ^ 1, s_abort, a.status, WAIT_LIMIT)) {
                         ok = false;
@@ -547,7 +655,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         phase ^= 1;
                     }
                 }
-                u = (long long)t * a.U + k1;
             }
             if (*s_abort) {
                 // wait (bounded) for loads still in flight before shared memory is released
@@ -564,15 +671,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            int seg = 0;
             const uint32_t idesc0 = ptx::idesc_bf16_f32(BM, a.nsub == 1 ? a.bn_total : 256);
             const uint32_t idesc1 = ptx::idesc_bf16_f32(BM, a.nsub == 1 ? 16 : a.bn_total - 256);
             const uint32_t a0 = ptx::smem_u32(sA), b0 = ptx::smem_u32(sB);
             bool ok = true;
-            for (long long u = ubeg; u < uend && ok; ++seg) {
-                const int t = (int)(u / a.U);
-                const int k0 = (int)(u - (long long)t * a.U);
-                const int k1 = (int)min((long long)a.U, uend - (long long)t * a.U);
+            for (int seg = 0; seg < L.ns && ok; ++seg) {
+                const Seg sg = seg_at(L, seg);
                 const int abuf = a.acc_cols ? (seg & 1) : 0;
                 const uint32_t aphase = a.acc_cols ? ((seg >> 1) & 1) : (seg & 1);
                 if (!ptx::mbar_wait(ptx::smem_u32(&acc_empty[abuf]), aphase ^ 1, s_abort, a.status, WAIT_LIMIT)) {
@@ -581,7 +685,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 }
                 ptx::tc_fence_after();
                 const uint32_t d = tmem_base + (uint32_t)(abuf * a.acc_cols);
-                for (int k = k0; k < k1; ++k) {
+                for (int k = sg.k0; k < sg.k1; ++k) {
                     if (!ptx::mbar_wait(ptx::smem_u32(&full_a[stage]), phase, s_abort, a.status, WAIT_LIMIT)) {
                         ok = false;
                         break;
@@ -590,7 +694,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const uint32_t as = a0 + stage * A_STAGE_BYTES, bs = b0 + stage * a.b_stage_bytes;
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
-                        const uint32_t acc = (k > k0 || kk > 0) ? 1u : 0u;
+                        const uint32_t acc = (k > sg.k0 || kk > 0) ? 1u : 0u;
                         ptx::mma_bf16(d, ptx::sw128_desc(as + kk * 32), ptx::sw128_desc(bs + kk * 32), idesc0, acc);
                         if (a.nsub == 2)
                             ptx::mma_bf16(d + 256, ptx::sw128_desc(as + kk * 32),
@@ -604,7 +708,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 }
                 if (!ok) break;
                 ptx::mma_commit(ptx::smem_u32(&acc_full[abuf]));
-                u = (long long)t * a.U + k1;
             }
             // all MMAs issued by this thread complete before TMEM is released
             ptx::mma_commit(ptx::smem_u32(drain));
@@ -613,132 +716,151 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------ epilogue --
+        // ------------------------------------------- records and epilogue --
+        // These four warps also build the sampling records, one epoch (a run of
+        // the CTA's chunks with one tile and group) ahead of the producers, in
+        // two buffers. Before the epilogue of a segment they build every epoch
+        // of that segment and the first one of the next; building epoch e waits
+        // only for the producers to release epoch e - 2, which needs no
+        // epilogue of this segment, so the order cannot deadlock.
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
-        int seg = 0;
+        const int per_g = a.nq * s.K2;
         uint32_t ephase = 0;
+        int rec_epoch = 0;
+        int rseg = 0, rk = L.ns > 0 ? seg_at(L, 0).k0 : 0;  // next epoch to build: its segment and first unit
         bool ok = true;
-        for (long long u = ubeg; u < uend && ok; ++seg) {
-            const int t = (int)(u / a.U);
-            const int k0 = (int)(u - (long long)t * a.U);
-            const int k1 = (int)min((long long)a.U, uend - (long long)t * a.U);
+        for (int seg = 0; seg < L.ns && ok; ++seg) {
+            const Seg sg = seg_at(L, seg);
+            const int t = sg.t;
+            while (rseg < L.ns && (rseg <= seg || (rseg == seg + 1 && rk == seg_at(L, rseg).k0))) {
+                const Seg rs = seg_at(L, rseg);
+                const int b = rec_epoch & 1;
+                if (rec_epoch >= 2 && !ptx::mbar_wait(ptx::smem_u32(&rec_empty[b]), ((rec_epoch - 2) >> 1) & 1, s_abort,
+                                                      a.status, WAIT_LIMIT)) {
+                    ok = false;
+                    break;
+                }
+                const int rg = rk / per_g;
+                // the first epoch is shared with the producer warps
+                build_records(a, rs.t / a.n_tiles, rg, row, rec_epoch == 0 ? 0 : -1, s_rec + b * BM * s.K2, s_tap);
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(rec_epoch == 0 ? rec0_bar : &rec_full[b]));
+                rk = min((rg + 1) * per_g, rs.k1);
+                if (rk >= rs.k1 && ++rseg < L.ns) rk = seg_at(L, rseg).k0;
+                ++rec_epoch;
+            }
+            if (!ok) break;
+
             const int abuf = a.acc_cols ? (seg & 1) : 0;
             const uint32_t aphase = a.acc_cols ? ((seg >> 1) & 1) : (seg & 1);
+            const bool full = (sg.k0 == 0 && sg.k1 == a.U);
+            const bool last_proc = seg == L.ns - 1;  // the pipeline is idle after this segment's accumulator
+            const long long tu0 = (long long)t * a.U;
+            int c_lo = cta, c_hi = cta;
+            if (!full) {
+                c_lo = cta_of_unit(tu0, s_starts, a.ctas);
+                c_hi = cta_of_unit(tu0 + a.U - 1, s_starts, a.ctas);
+            }
+            // Thread 0 learns whether every other contributor of this tile has
+            // published its partial: one read before the accumulator is ready
+            // and, for the CTA's last segment, a fresh one after.
+            int cnt = -1;
+            if (!full && threadIdx.x == 0) cnt = ptx::ld_relaxed_gpu(a.counters + t);
             if (!ptx::mbar_wait(ptx::smem_u32(&acc_full[abuf]), aphase, s_abort, a.status, WAIT_LIMIT)) {
                 ok = false;
                 break;
             }
             ptx::tc_fence_after();
             const int mt = t / a.n_tiles, n0 = (t % a.n_tiles) * a.bn_total;
+            const int ncols = min(a.bn_total, s.Cout - n0);
+            if (threadIdx.x == 0) {
+                int last = full ? 1 : 0;
+                if (!full) {
+                    if (cnt != c_hi - c_lo && last_proc) cnt = ptx::ld_relaxed_gpu(a.counters + t);
+                    last = cnt == c_hi - c_lo;
+                    if (last) ptx::fence_acq_rel_gpu();  // the partials read below follow the counter
+                }
+                s_last[seg & 1] = last;
+            }
+            float* sbias = s_bias + (seg & 1) * 512;  // by segment parity, like s_last
+            if (a.bias)
+                for (int i = threadIdx.x; i < ncols; i += 4 * 32) sbias[i] = __bfloat162float(a.bias[n0 + i]);
+            if (!epi_sync(epi_bar, ephase, s_abort, a.status)) {
+                ok = false;
+                break;
+            }
+            const float* sb = a.bias ? sbias : nullptr;
             const int p = strip_to_raster(mt * BM + row, a);
             const uint32_t taddr = tmem_base + (uint32_t)(abuf * a.acc_cols) + ((uint32_t)(quarter * 32) << 16);
-            const bool full = (k0 == 0 && k1 == a.U);
-            const int ncols = min(a.bn_total, s.Cout - n0);
             bf16* yrow = a.y + (size_t)(p < 0 ? 0 : p) * s.Cout + n0;
-            if (full) {
-                for (int cc = 0; cc < a.bn_total; cc += 32) {
-                    float v[32];
-                    ptx::tmem_ld32(taddr + cc, v);
-                    if (p >= 0 && cc < ncols) store_row32(yrow, cc, ncols, v, a.bias, n0);
+            if (s_last[seg & 1]) {
+                // y = this CTA's accumulator + the other contributors' partials + bias. In
+                // the CTA's last segment the pipeline buffers are idle, so when the
+                // partials fit there they are bulk-copied in and read from shared memory.
+                const uint32_t tile_bytes = (uint32_t)BM * a.bn_total * 4;
+                const bool staged = !full && last_proc &&
+                                    (uint32_t)(c_hi - c_lo) * tile_bytes <= a.b_off + a.stages * a.b_stage_bytes;
+                if (staged) {
+                    if (threadIdx.x == 0) {
+                        ptx::fence_proxy_async_all();
+                        const uint32_t tb = ptx::smem_u32(tail_bar);
+                        ptx::mbar_arrive_expect_tx(tb, (uint32_t)(c_hi - c_lo) * tile_bytes);
+                        uint32_t dst = ptx::smem_u32(smem);
+                        for (int c = c_lo; c <= c_hi; ++c) {
+                            if (c == cta) continue;
+                            const uint8_t* src = reinterpret_cast<const uint8_t*>(partial_base(a, s_starts, c, tu0, 0));
+                            for (uint32_t o = 0; o < tile_bytes; o += 16384u)
+                                ptx::bulk_load(dst + o, src + o, min(16384u, tile_bytes - o), tb);
+                            dst += tile_bytes;
+                        }
+                    }
+                    if (!ptx::mbar_wait(ptx::smem_u32(tail_bar), 0, s_abort, a.status, WAIT_LIMIT)) {
+                        ok = false;
+                        break;
+                    }
                 }
+                combine_rows(taddr, ncols, c_lo, c_hi, cta, staged, [&](int c) -> const float* {
+                    // staged partials are packed in contributor order without this CTA's
+                    if (staged) return reinterpret_cast<const float*>(smem + (size_t)(c - c_lo - (c > cta)) * tile_bytes) + row * 4;
+                    return partial_base(a, s_starts, c, tu0, row);
+                }, yrow, p >= 0, sb);
                 ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&acc_empty[abuf]));
+                if (!full && threadIdx.x == 0) a.counters[t] = 0;
             } else {
-                const long long tu0 = (long long)t * a.U;
-                const int c_lo = cta_of_unit(tu0, a), c_hi = cta_of_unit(tu0 + a.U - 1, a);
-                // If every other contributor of this tile has already published its
-                // partial, add them to this CTA's accumulator straight from TMEM.
-                if (threadIdx.x == 0) *s_last = (ptx::ld_acquire_gpu(a.counters + t) == c_hi - c_lo) ? 1 : 0;
+                // publish this CTA's partial tile, then count it in; the accumulator
+                // stays in TMEM until it is known whether this CTA finishes the tile
+                float* dst = const_cast<float*>(partial_base(a, s_starts, cta, tu0, row));
+                tmem_rows<true>(taddr, a.bn_total, [&](uint32_t(&r)[32], int cc) {
+                    float* b = dst + (size_t)(cc >> 5) * 8 * BM * 4;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        *reinterpret_cast<uint4*>(b + q * BM * 4) = make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+                });
+                __threadfence();
                 if (!epi_sync(epi_bar, ephase, s_abort, a.status)) {
                     ok = false;
                     break;
                 }
-                if (*s_last) {
-                    // The CTA's last segment: the pipeline buffers are idle, so when the other
-                    // contributors' partial tiles fit there they are bulk-copied in and read
-                    // from shared memory; otherwise they are read from global memory.
-                    const uint32_t tile_bytes = (uint32_t)BM * a.bn_total * 4;
-                    const bool last_seg = (long long)t * a.U + k1 == uend;
-                    const bool staged = last_seg && (uint32_t)(c_hi - c_lo) * tile_bytes <= a.b_off + a.stages * a.b_stage_bytes;
-                    if (staged) {
-                        if (threadIdx.x == 0) {
-                            ptx::fence_proxy_async_all();
-                            const uint32_t tb = ptx::smem_u32(tail_bar);
-                            ptx::mbar_arrive_expect_tx(tb, (uint32_t)(c_hi - c_lo) * tile_bytes);
-                            uint32_t dst = ptx::smem_u32(smem);
-                            for (int c = c_lo; c <= c_hi; ++c) {
-                                if (c == cta) continue;
-                                const uint8_t* src = reinterpret_cast<const uint8_t*>(partial_base(a, c, tu0, 0));
-                                for (uint32_t o = 0; o < tile_bytes; o += 16384u)
-                                    ptx::bulk_load(dst + o, src + o, min(16384u, tile_bytes - o), tb);
-                                dst += tile_bytes;
-                            }
-                        }
-                        if (!ptx::mbar_wait(ptx::smem_u32(tail_bar), 0, s_abort, a.status, WAIT_LIMIT)) {
-                            ok = false;
-                            break;
-                        }
-                    }
-                    for (int cc = 0; cc < ncols; cc += 32) {
-                        float v[32];
-                        ptx::tmem_ld32(taddr + cc, v);
-                        int slot = 0;
-                        for (int c = c_lo; c <= c_hi; ++c) {
-                            if (c == cta) continue;
-                            if (staged)
-                                add_partial32_smem(v, reinterpret_cast<const float*>(smem + (size_t)slot * tile_bytes) + row * 4, cc);
-                            else
-                                add_partial32(v, partial_base(a, c, tu0, row), cc);
-                            ++slot;
-                        }
-                        if (p >= 0) store_row32(yrow, cc, ncols, v, a.bias, n0);
-                    }
-                    ptx::tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&acc_empty[abuf]));
-                    if (threadIdx.x == 0) a.counters[t] = 0;
-                } else {
-                    float* dst = const_cast<float*>(partial_base(a, cta, tu0, row));
-                    for (int cc = 0; cc < a.bn_total; cc += 32) {
-                        float v[32];
-                        ptx::tmem_ld32(taddr + cc, v);
-                        float* b = dst + (size_t)(cc >> 5) * 8 * BM * 4;
-#pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            *reinterpret_cast<float4*>(b + q * BM * 4) =
-                                make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-                    }
-                    ptx::tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&acc_empty[abuf]));
-                    __threadfence();
-                    if (!epi_sync(epi_bar, ephase, s_abort, a.status)) {
-                        ok = false;
-                        break;
-                    }
-                    if (threadIdx.x == 0) *s_last = (atomicAdd(a.counters + t, 1) == c_hi - c_lo) ? 1 : 0;
-                    if (!epi_sync(epi_bar, ephase, s_abort, a.status)) {
-                        ok = false;
-                        break;
-                    }
-                    if (*s_last) {
-                        __threadfence();
-                        if (p >= 0) {
-                            for (int cc = 0; cc < ncols; cc += 32) {
-                                float v[32];
-#pragma unroll
-                                for (int e = 0; e < 32; ++e) v[e] = 0.f;
-                                for (int c = c_lo; c <= c_hi; ++c) add_partial32(v, partial_base(a, c, tu0, row), cc);
-                                store_row32(yrow, cc, ncols, v, a.bias, n0);
-                            }
-                        }
-                        if (threadIdx.x == 0) a.counters[t] = 0;
-                    }
+                if (threadIdx.x == 0) s_last[seg & 1] = (atomicAdd(a.counters + t, 1) == c_hi - c_lo) ? 1 : 0;
+                if (!epi_sync(epi_bar, ephase, s_abort, a.status)) {
+                    ok = false;
+                    break;
                 }
+                if (s_last[seg & 1]) {
+                    // every other contributor's partial is in the workspace
+                    __threadfence();
+                    combine_rows(taddr, ncols, c_lo, c_hi, cta, false, [&](int c) -> const float* {
+                        return partial_base(a, s_starts, c, tu0, row);
+                    }, yrow, p >= 0, sb);
+                    if (threadIdx.x == 0) a.counters[t] = 0;
+                }
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&acc_empty[abuf]));
             }
-            u = (long long)t * a.U + k1;
         }
     }
 
@@ -756,9 +878,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 struct Plan {
     bool ok;
     int bn_total, n_tiles, m_tiles, tiles, nq, U, ctas, nsub, box_rows, stages, acc_cols, tmem_cols;
-    int sw, nf, wl;
+    int sw, nf, wl, snap;
     long long total_units;
-    uint32_t b_off, info_off, base_off, row_off, bar_off, b_stage_bytes, smem_bytes;
+    uint32_t b_off, info_off, row_off, bar_off, b_stage_bytes, smem_bytes;
     size_t ws_partials, ws_counters_off, ws_bytes;
 };
 
@@ -781,7 +903,20 @@ Plan make_plan(const Shape& s, int sms) {
     pl.wl = s.Wo - pl.nf * pl.sw;
     pl.U = s.G * pl.nq * s.K2;
     pl.total_units = (long long)pl.tiles * pl.U;
-    pl.ctas = (int)std::min<long long>(sms, pl.total_units);
+    pl.ctas = (int)std::min<long long>(std::min(sms, MAX_CTAS), pl.total_units);
+    // Snap starts away from a tile's last units when CTAs get at least 12 units
+    // each. A share of n units, U <= n < 2U, spans three tiles when fewer than
+    // n - U of them fall in its first tile, so snap at least that far; a CTA
+    // whose successor was snapped ends on a tile boundary and spans two tiles.
+    {
+        const long long per = (pl.total_units + pl.ctas - 1) / pl.ctas;
+        pl.snap = 0;
+        if (pl.U >= 4 && pl.total_units / pl.ctas >= 12) {
+            long long sn = 3;
+            if (per >= pl.U && per < 2 * pl.U) sn = std::max<long long>(sn, per - pl.U + 1);
+            pl.snap = (int)std::min<long long>(sn, pl.U / 2);
+        }
+    }
     pl.nsub = pl.bn_total > 256 ? 2 : 1;
     pl.box_rows = pl.nsub == 1 ? pl.bn_total : 256;
     pl.b_stage_bytes = (uint32_t)(pl.nsub * pl.box_rows * 128);
@@ -794,8 +929,8 @@ Plan make_plan(const Shape& s, int sms) {
         pl.tmem_cols = 512;
         pl.acc_cols = 0;
     }
-    const uint32_t info_bytes = (uint32_t)(BM * s.K2 * (sizeof(TapW) + sizeof(int)));
-    const uint32_t fixed = info_bytes + BM * 16 + 256 + 64 * 8 + 64 + 1024;  // info, barriers, flags, alignment slack
+    const uint32_t info_bytes = (uint32_t)(2 * BM * s.K2 * sizeof(TapRec));  // two record buffers
+    const uint32_t fixed = info_bytes + 256 + (MAX_CTAS + 2) * 8 + 4096 + (3 * MAX_STAGES + 14) * 8 + 16 + 1024;
     const uint32_t budget = 227 * 1024;
     const uint32_t stage_bytes = A_STAGE_BYTES + pl.b_stage_bytes;
     int st = (int)((budget - fixed) / stage_bytes);
@@ -804,10 +939,10 @@ Plan make_plan(const Shape& s, int sms) {
     pl.stages = st;
     pl.b_off = (uint32_t)(st * A_STAGE_BYTES);
     pl.info_off = pl.b_off + (uint32_t)st * pl.b_stage_bytes;
-    pl.base_off = pl.info_off + (uint32_t)(BM * s.K2 * sizeof(TapW));
-    pl.row_off = (pl.base_off + (uint32_t)(BM * s.K2 * sizeof(int)) + 15) & ~15u;
-    pl.bar_off = (pl.row_off + (uint32_t)(BM * sizeof(int4) + 32 * sizeof(int2)) + 7) & ~7u;
-    pl.smem_bytes = pl.bar_off + (3 * MAX_STAGES + 8) * 8 + 16 + 1024;
+    pl.row_off = pl.info_off + info_bytes;
+    // taps, CTA start table, bias of one tile
+    pl.bar_off = pl.row_off + (uint32_t)(32 * sizeof(int2) + (MAX_CTAS + 2) * sizeof(long long) + 2 * 512 * sizeof(float));
+    pl.smem_bytes = pl.bar_off + (3 * MAX_STAGES + 14) * 8 + 16 + 1024;
     if (pl.smem_bytes > budget) return pl;
     pl.ws_partials = (size_t)pl.ctas * 2 * BM * pl.bn_total * sizeof(float);
     pl.ws_counters_off = (pl.ws_partials + 255) & ~(size_t)255;
@@ -853,14 +988,17 @@ cudaError_t fwd_tc(const Shape& s, const void* x, const void* off, const void* m
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    static bool attr_set[64] = {false};
+    // one 32-byte load per neighbour slice when every slice start is 32-byte aligned
+    const bool wide = s.Cin % 16 == 0 && s.Cg % 16 == 0 && (reinterpret_cast<uintptr_t>(x) & 31) == 0;
+    auto kernel = wide ? dcn_fwd_tc_kernel<true> : dcn_fwd_tc_kernel<false>;
+    static bool attr_set[64][2] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        e = cudaFuncSetAttribute(dcn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    if (dev >= 0 && dev < 64 && !attr_set[dev][wide]) {
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
+        attr_set[dev][wide] = true;
     }
     int* counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + pl.ws_counters_off);
     e = cudaMemsetAsync(counters, 0, (size_t)pl.tiles * sizeof(int), st);
@@ -884,6 +1022,7 @@ cudaError_t fwd_tc(const Shape& s, const void* x, const void* off, const void* m
     a.wl = pl.wl;
     a.ctas = pl.ctas;
     a.total_units = pl.total_units;
+    a.snap = pl.snap;
     a.bn_total = pl.bn_total;
     a.nsub = pl.nsub;
     a.box_rows = pl.box_rows;
@@ -892,11 +1031,10 @@ cudaError_t fwd_tc(const Shape& s, const void* x, const void* off, const void* m
     a.tmem_cols = pl.tmem_cols;
     a.b_off = pl.b_off;
     a.info_off = pl.info_off;
-    a.base_off = pl.base_off;
     a.row_off = pl.row_off;
     a.bar_off = pl.bar_off;
     a.b_stage_bytes = pl.b_stage_bytes;
-    dcn_fwd_tc_kernel<<<pl.ctas, NUM_THREADS, pl.smem_bytes, st>>>(map, a);
+    kernel<<<pl.ctas, NUM_THREADS, pl.smem_bytes, st>>>(map, a);
     if (launches) *launches += 2;
     return cudaGetLastError();
 }
