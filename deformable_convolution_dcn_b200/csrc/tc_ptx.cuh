@@ -49,6 +49,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may stay suspended (issuing nothing) for up
+// to `hint_ns` nanoseconds while the phase is incomplete; it resumes as soon
+// as the phase completes.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Waits for the phase of `bar` with the given parity to complete. Gives up
 // after `limit` clock cycles, or early once another thread of the CTA has
 // raised *abort; on giving up it raises *abort, records kStatusTimeout in the
@@ -58,8 +73,10 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     if (mbar_try_wait(bar, parity)) return true;
     long long t0 = clock64();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 0) {
+        // suspended in hardware between checks rather than spinning, so that a
+        // waiting warp takes no issue slots from the warps doing the work
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        if ((it & 3u) == 0) {
             if (*abort) return false;
             if (clock64() - t0 > limit) {
                 *abort = 1;
