@@ -36,6 +36,7 @@ _lib = None
 
 DCN_F32, DCN_BF16 = 0, 1
 DCN_FLAG_GENERIC = 0x1
+DCN_FLAG_NO_TF32 = 0x2
 OP_FORWARD, OP_BACKWARD_DATA, OP_BACKWARD_WEIGHT = 0, 1, 2
 _DTYPES = {torch.float32: DCN_F32, torch.bfloat16: DCN_BF16}
 
@@ -107,7 +108,7 @@ def make_params(B, H, W, Cin, Cout, K, stride=1, pad=0, dil=1, G=1, dtype=DCN_F3
     return Params(B, H, W, Cin, Cout, K, stride, pad, dil, G, dtype, flags)
 
 
-def _params(x, weight, offset, stride, padding, dilation, generic):
+def _params(x, weight, offset, stride, padding, dilation, generic, flags=0):
     if x.dim() != 4 or weight.dim() != 4:
         raise ValueError("x must be [B, H, W, Cin] and weight [Cout, K, K, Cin]")
     B, H, W, Cin = x.shape
@@ -120,7 +121,7 @@ def _params(x, weight, offset, stride, padding, dilation, generic):
     if x.dtype not in _DTYPES:
         raise TypeError("x must be float32 or bfloat16, got %s" % x.dtype)
     return make_params(B, H, W, Cin, Cout, K, stride, padding, dilation, G, _DTYPES[x.dtype],
-                       DCN_FLAG_GENERIC if generic else 0)
+                       (DCN_FLAG_GENERIC if generic else 0) | flags)
 
 
 def _check_tensors(dtype, device, **ts):
@@ -167,10 +168,11 @@ def _workspace(p, op, device, workspace):
 
 
 def forward(x, offset, mask, weight, bias=None, stride=1, padding=0, dilation=1, *, out=None, workspace=None,
-            generic=False):
-    """y [B, Ho, Wo, Cout] = DCNv2(x, offset, mask, weight, bias) on x's device and current stream."""
+            generic=False, flags=0):
+    """y [B, Ho, Wo, Cout] = DCNv2(x, offset, mask, weight, bias) on x's device and current stream.
+    flags: extra DCN_FLAG_* bits (DCN_FLAG_NO_TF32 keeps float32 layers off the split-tf32 kernel)."""
     lib = _load()
-    p = _params(x, weight, offset, stride, padding, dilation, generic)
+    p = _params(x, weight, offset, stride, padding, dilation, generic, flags)
     _check_tensors(x.dtype, x.device, x=x, offset=offset, mask=mask, weight=weight, bias=bias, out=out)
     Ho, Wo = output_size(p)
     if out is None:

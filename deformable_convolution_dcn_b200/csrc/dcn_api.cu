@@ -101,6 +101,12 @@ bool use_fwd_tc(const dcn_params_t* p, const dcn::Shape& s) {
     return p->dtype == DCN_BF16 && !(p->flags & DCN_FLAG_GENERIC) && dcn::fwd_tc_supported(s);
 }
 
+// The float32 tensor-core forward for RGB-like layers: Cin <= 3, K*K <= 9,
+// Cout a multiple of 32. DCN_FLAG_NO_TF32 keeps such layers on CUDA cores.
+bool use_fwd_f32_tc(const dcn_params_t* p, const dcn::Shape& s) {
+    return p->dtype == DCN_F32 && !(p->flags & (DCN_FLAG_GENERIC | DCN_FLAG_NO_TF32)) && dcn::fwd_f32_tc_supported(s);
+}
+
 // The small-channel float32 forward: Cin <= 8, Cout a multiple of 32.
 bool use_fwd_small(const dcn_params_t* p, const dcn::Shape& s) {
     return p->dtype == DCN_F32 && !(p->flags & DCN_FLAG_GENERIC) && dcn::fwd_f32_small_supported(s);
@@ -157,6 +163,7 @@ const char* dcn_forward_path(const dcn_params_t* params) {
         return "invalid";
     }
     if (use_fwd_tc(params, s)) return "tcgen05_gather";
+    if (use_fwd_f32_tc(params, s)) return "tcgen05_tf32_split";
     if (use_fwd_small(params, s)) return "f32_small_channels";
     return "generic";
 }
@@ -185,6 +192,15 @@ int dcn_forward(const dcn_params_t* params, const void* x, const void* offset, c
         e = dcn::fwd_tc(s, x, offset, mask, weight, bias, y, workspace, workspace_bytes, status, st, &n);
         g_launches += n;
         if (e != cudaSuccess) return cuda_fail(e, "tensor-core forward launch");
+        return ok();
+    }
+    if (use_fwd_f32_tc(params, s) && aligned16(y)) {
+        unsigned* status = nullptr;
+        cudaError_t e = dcn::status_word_ptr(&status);
+        if (e != cudaSuccess) return cuda_fail(e, "status word");
+        e = dcn::fwd_f32_tc(s, x, offset, mask, weight, bias, y, status, st);
+        g_launches += 1;
+        if (e != cudaSuccess) return cuda_fail(e, "float32 tensor-core forward launch");
         return ok();
     }
     if (use_fwd_small(params, s) && aligned16(y)) {

@@ -29,6 +29,12 @@ size_t fwd_tc_static_scratch_bytes();
 cudaError_t fwd_tc_noalloc(const Shape& s, const void* x, const void* off, const void* mask, const void* w,
                            const void* bias, void* y, unsigned* status, cudaStream_t st, int* launches);
 
+// fwd_f32_tc.cu — float32 forward for layers with Cin <= 3, K*K <= 9 on tcgen05
+// (split tf32 operands, float32 accuracy); y 16-byte aligned.
+bool fwd_f32_tc_supported(const Shape& s);
+cudaError_t fwd_f32_tc(const Shape& s, const void* x, const void* off, const void* mask, const void* w,
+                       const void* bias, void* y, unsigned* status, cudaStream_t st);
+
 // fwd_f32_small.cu — float32 forward for layers with Cin <= 8 (CUDA cores, HBM-bound).
 bool fwd_f32_small_supported(const Shape& s);
 cudaError_t fwd_f32_small(const Shape& s, const void* x, const void* off, const void* mask, const void* w,

@@ -83,6 +83,7 @@ typedef enum {
 
 /* dcn_params_t.flags */
 #define DCN_FLAG_GENERIC 0x1u    /* use the generic CUDA-core kernels even where a specialised kernel exists */
+#define DCN_FLAG_NO_TF32 0x2u    /* float32 layers: keep the contraction on CUDA cores (no split-tf32 tensor-core kernel) */
 
 typedef struct dcn_params {
     int B, H, W;     /* batch, input height and width */

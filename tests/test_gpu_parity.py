@@ -210,19 +210,39 @@ def test_full_size_backward_sampled():
         assert abs(lhs - rhs) <= 2e-2 * abs(lhs), (gname, lhs, rhs)
 
 
-@pytest.mark.parametrize("shape", [
-    gen.LayerShape(B=1, Cin=3, H=23, W=19, Cout=64, K=3, stride=1, pad=1),
-    gen.LayerShape(B=2, Cin=1, H=9, W=12, Cout=32, K=5, stride=2, pad=2),
-    gen.LayerShape(B=1, Cin=8, H=10, W=7, Cout=128, K=3, stride=1, pad=2, dil=2, G=2),
-    gen.LayerShape(B=2, Cin=2, H=6, W=9, Cout=16, K=3, stride=1, pad=1, G=2),
-    gen.LayerShape(B=3, Cin=6, H=8, W=8, Cout=128, K=1, stride=1, pad=0, G=3),
-    gen.LayerShape(B=1, Cin=4, H=31, W=17, Cout=64, K=3, stride=2, pad=0),
-], ids=lambda s: "C%dx%dK%ds%dd%dG%d" % (s.Cin, s.Cout, s.K, s.stride, s.dil, s.G))
-def test_small_channel_f32_layers(shape):
-    """Float32 layers with few input channels (the stem-style kernel), compared in full."""
+def _tf32_split_applies(s):
+    """The float32 tensor-core kernel takes Cin <= 3, one group, K*K <= 9, Cout a multiple of 32 up to 256."""
+    return s.Cin <= 3 and s.G == 1 and s.K * s.K <= 9 and s.Cout % 32 == 0 and 32 <= s.Cout <= 256
+
+
+@pytest.mark.parametrize("kernel", ["default", "cuda_cores"])
+@pytest.mark.parametrize("shape,mask", [
+    (gen.LayerShape(B=1, Cin=3, H=23, W=19, Cout=64, K=3, stride=1, pad=1), True),
+    (gen.LayerShape(B=2, Cin=3, H=17, W=30, Cout=128, K=3, stride=2, pad=1), True),
+    (gen.LayerShape(B=1, Cin=2, H=13, W=11, Cout=32, K=3, stride=1, pad=2, dil=2), True),
+    (gen.LayerShape(B=1, Cin=1, H=20, W=21, Cout=256, K=3, stride=1, pad=0), True),
+    (gen.LayerShape(B=1, Cin=3, H=9, W=40, Cout=128, K=1, stride=1, pad=0), False),
+    (gen.LayerShape(B=2, Cin=1, H=9, W=12, Cout=32, K=5, stride=2, pad=2), True),
+    (gen.LayerShape(B=1, Cin=8, H=10, W=7, Cout=128, K=3, stride=1, pad=2, dil=2, G=2), True),
+    (gen.LayerShape(B=2, Cin=2, H=6, W=9, Cout=16, K=3, stride=1, pad=1, G=2), True),
+    (gen.LayerShape(B=3, Cin=6, H=8, W=8, Cout=128, K=1, stride=1, pad=0, G=3), True),
+    (gen.LayerShape(B=1, Cin=4, H=31, W=17, Cout=64, K=3, stride=2, pad=0), True),
+], ids=lambda v: v if isinstance(v, bool) else "C%dx%dK%ds%dd%dG%d" % (v.Cin, v.Cout, v.K, v.stride, v.dil, v.G))
+def test_small_channel_f32_layers(shape, mask, kernel):
+    """Float32 layers with few input channels, compared in full: the split-tf32
+    tensor-core kernel where it applies, and the CUDA-core kernel (forced with
+    DCN_FLAG_NO_TF32) on the same layers."""
     w = gen.Workload("smallc", shape, "f32", seed=9, offset_dist="normal1.5_edges", bias=True)
     d = gen.make_inputs(w)
-    p = dcn._params(d["x"], d["weight"], d["offset"], shape.stride, shape.pad, shape.dil, False)
-    assert dcn.forward_path(p) == "f32_small_channels"
-    y = run_forward(shape, to_dev(d))
+    if not mask:
+        d["mask"] = None
+    flags = dcn.DCN_FLAG_NO_TF32 if kernel == "cuda_cores" else 0
+    p = dcn._params(d["x"], d["weight"], d["offset"], shape.stride, shape.pad, shape.dil, False, flags)
+    expect = "tcgen05_tf32_split" if kernel == "default" and _tf32_split_applies(shape) else "f32_small_channels"
+    assert dcn.forward_path(p) == expect
+    dd = to_dev(d)
+    y = dcn.forward(dd["x"], dd["offset"], dd["mask"], dd["weight"], dd["bias"], shape.stride, shape.pad, shape.dil,
+                    flags=flags)
+    torch.cuda.synchronize()
+    dcn.check_status()
     assert_close(_cpu(y), _oracle_forward(shape, f64(d)), "f32", "y")
