@@ -307,13 +307,22 @@ __device__ __forceinline__ void tmem_rows(uint32_t taddr, int ncols, F&& f) {
     }
 }
 
-// y row = bias + the tile's partial sums in contributor order c_lo..c_hi, this
-// CTA's own taken from its TMEM accumulator and every other one from `part(c)`
-// (a row pointer in partial_base layout; in_smem: staged in shared memory).
-// The fixed order makes the result independent of which CTA finishes the tile.
+// y rows = bias + the tile's partial sums in contributor order c_lo..c_hi,
+// this CTA's own taken from its TMEM accumulator and every other one from
+// `part(c)` (a row pointer in partial_base layout; in_smem: staged in shared
+// memory). The fixed order makes the result independent of which CTA finishes
+// the tile. Called by all 32 lanes of an epilogue warp (TMEM loads are
+// warp-collective); lane l holds tile row warp*32 + l, whose output row is
+// pr (-1: past the end). With a staging buffer (ybuf != 0: 32 rows x 128 B,
+// 16-byte chunks swizzled by row) and a tile width that is a multiple of 64,
+// every 64 columns of the warp's 32 rows go through it and leave as full
+// 128-byte row segments, eight lanes per row; otherwise each lane stores its row.
 template <typename P>
 __device__ __forceinline__ void combine_rows(uint32_t taddr, int ncols, int c_lo, int c_hi, int cta, bool in_smem,
-                                             P&& part, bf16* yrow, bool store, const float* sb) {
+                                             P&& part, const float* sb, uint32_t ybuf, bf16* ycol0, int pr,
+                                             int ldy) {
+    const int lane = threadIdx.x & 31;
+    const bool coalesce = ybuf != 0 && (ncols & 63) == 0;
     for (int cc = 0; cc < ncols; cc += 32) {
         uint32_t acc[32];
 #pragma unroll
@@ -333,7 +342,41 @@ __device__ __forceinline__ void combine_rows(uint32_t taddr, int ncols, int c_lo
             if (in_smem) add_partial32_smem(acc, part(c), cc);
             else add_partial32(acc, part(c), cc);
         }
-        if (store) store_row32(yrow, cc, ncols, acc, sb);
+        if (!coalesce) {
+            if (pr >= 0) store_row32(ycol0 + (size_t)pr * ldy, cc, ncols, acc, sb);
+            continue;
+        }
+        if (sb) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float4 b = *reinterpret_cast<const float4*>(sb + cc + 4 * q);
+                acc[4 * q] = __float_as_uint(__uint_as_float(acc[4 * q]) + b.x);
+                acc[4 * q + 1] = __float_as_uint(__uint_as_float(acc[4 * q + 1]) + b.y);
+                acc[4 * q + 2] = __float_as_uint(__uint_as_float(acc[4 * q + 2]) + b.z);
+                acc[4 * q + 3] = __float_as_uint(__uint_as_float(acc[4 * q + 3]) + b.w);
+            }
+        }
+        const int h = (cc >> 5) & 1;  // which half of the 64-column group
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t* w = acc + 8 * j;
+            ptx::sts_v4(ybuf + lane * 128 + (((4 * h + j) ^ (lane & 7)) << 4),
+                        make_uint4(pack_bf16(__uint_as_float(w[0]), __uint_as_float(w[1])),
+                                   pack_bf16(__uint_as_float(w[2]), __uint_as_float(w[3])),
+                                   pack_bf16(__uint_as_float(w[4]), __uint_as_float(w[5])),
+                                   pack_bf16(__uint_as_float(w[6]), __uint_as_float(w[7]))));
+        }
+        if (h == 1) {
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int rr = 4 * i + (lane >> 3), ch = lane & 7;
+                const uint4 v = ptx::lds_v4(ybuf + rr * 128 + ((ch ^ (rr & 7)) << 4));
+                const int prr = __shfl_sync(0xffffffffu, pr, rr);
+                if (prr >= 0) *reinterpret_cast<uint4*>(ycol0 + (size_t)prr * ldy + (cc - 32) + ch * 8) = v;
+            }
+            __syncwarp();
+        }
     }
 }
 
@@ -793,7 +836,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const float* sb = a.bias ? sbias : nullptr;
             const int p = strip_to_raster(mt * BM + row, a);
             const uint32_t taddr = tmem_base + (uint32_t)(abuf * a.acc_cols) + ((uint32_t)(quarter * 32) << 16);
-            bf16* yrow = a.y + (size_t)(p < 0 ? 0 : p) * s.Cout + n0;
+            bf16* ycol0 = a.y + n0;  // y[pixel, n0 + col] = ycol0[pixel * Cout + col]
             if (s_last[seg & 1]) {
                 // y = this CTA's accumulator + the other contributors' partials + bias. In
                 // the CTA's last segment the pipeline buffers are idle, so when the
@@ -820,11 +863,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         break;
                     }
                 }
+                // In the CTA's last segment the output rows are staged for full-line stores
+                // in the idle pipeline buffers, after any staged partials (4 warps x 4 KB).
+                const uint32_t yoff = staged ? (uint32_t)(c_hi - c_lo) * tile_bytes : 0u;
+                const uint32_t ybuf = (last_proc && yoff + 4 * 4096 <= a.b_off + a.stages * a.b_stage_bytes)
+                                          ? ptx::smem_u32(smem + yoff) + quarter * 4096
+                                          : 0u;
                 combine_rows(taddr, ncols, c_lo, c_hi, cta, staged, [&](int c) -> const float* {
                     // staged partials are packed in contributor order without this CTA's
                     if (staged) return reinterpret_cast<const float*>(smem + (size_t)(c - c_lo - (c > cta)) * tile_bytes) + row * 4;
                     return partial_base(a, s_starts, c, tu0, row);
-                }, yrow, p >= 0, sb);
+                }, sb, ybuf, ycol0, p, s.Cout);
                 ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&acc_empty[abuf]));
@@ -854,7 +903,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     __threadfence();
                     combine_rows(taddr, ncols, c_lo, c_hi, cta, false, [&](int c) -> const float* {
                         return partial_base(a, s_starts, c, tu0, row);
-                    }, yrow, p >= 0, sb);
+                    }, sb, 0u, ycol0, p, s.Cout);
                     if (threadIdx.x == 0) a.counters[t] = 0;
                 }
                 ptx::tc_fence_before();
