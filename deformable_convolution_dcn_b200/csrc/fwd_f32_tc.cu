@@ -10,11 +10,12 @@
 // float32). The dropped term Col_lo * W_lo^T and the tf32 reading of the
 // residuals are each about 2^-21 of |Col||W|, far below the float32 tolerance.
 //
-// One CTA per 128 output pixels, 128 threads, several CTAs per SM:
-//   * every thread owns one tile row (pixel): it loads the row's offsets and
-//     mask, samples the K*K bilinear neighbours of its pixel (all Cin channels,
-//     each neighbour outside the map contributing zero), modulates them, and
-//     writes the 27 values, split, into two 128-byte-swizzled K-major A tiles;
+// One CTA per 128 output pixels, 384 threads, three CTAs per SM:
+//   * three threads share a tile row (pixel), each taking a third of the taps:
+//     it loads those taps' offsets and mask, samples the bilinear neighbours
+//     (all Cin channels, each neighbour outside the map contributing zero),
+//     modulates them, and writes its values, split, into two 128-byte-swizzled
+//     K-major A tiles;
 //   * the CTA splits the weights [Cout, K*K*Cin] the same way into two B tiles;
 //   * one thread issues the 12 tcgen05.mma (kind::tf32, M=128, N=Cout, K=8);
 //   * each warp reads its 32 TMEM lanes back, adds the bias, and writes the rows
@@ -32,7 +33,9 @@ namespace {
 
 constexpr int BM = 128;        // output pixels per CTA (UMMA M)
 constexpr int KP = 32;         // padded contraction depth: one 128-byte swizzle row of float32
-constexpr int THREADS = 128;   // one thread per tile row and TMEM lane
+constexpr int PARTS = 3;       // threads per tile row, each gathering a third of the taps
+constexpr int THREADS = PARTS * BM;
+constexpr int TAPS_PER_PART = 3;  // ceil(MAX_TAPS / PARTS)
 constexpr int MAX_TAPS = 9;
 constexpr uint32_t TILE_BYTES = BM * 128;  // one [128 x 32] float32 swizzled tile
 constexpr long long WAIT_LIMIT = 2000000000LL;
@@ -57,7 +60,7 @@ struct Args {
 __device__ __forceinline__ uint32_t sw_chunk(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
 
 template <int CIN>
-__global__ void __launch_bounds__(THREADS) stem_tc_kernel(const __grid_constant__ CUtensorMap tmap_y, const Args a) {
+__global__ void __launch_bounds__(THREADS, 3) stem_tc_kernel(const __grid_constant__ CUtensorMap tmap_y, const Args a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const Shape& s = a.s;
@@ -91,9 +94,11 @@ __global__ void __launch_bounds__(THREADS) stem_tc_kernel(const __grid_constant_
         ptx::tmem_relinquish();
     }
 
-    // ---- this thread's pixel, its offsets and mask (all loads issued first)
+    // ---- this thread's pixel and taps, their offsets and mask (all loads issued first)
+    const int row = tid % BM, part = tid / BM;
+    const int tp_lo = s.K2 * part / PARTS, tp_hi = s.K2 * (part + 1) / PARTS;
     const int plane = s.Ho * s.Wo;
-    const int p = blockIdx.x * BM + tid;
+    const int p = blockIdx.x * BM + row;
     const bool pv = p < s.P;
     int bb = 0, pix = 0, oy = 0, ox = 0;
     if (pv) {
@@ -105,15 +110,16 @@ __global__ void __launch_bounds__(THREADS) stem_tc_kernel(const __grid_constant_
     }
     const float* offp = a.off + (size_t)bb * 2 * s.K2 * plane + pix;
     const float* mp = a.mask ? a.mask + (size_t)bb * s.K2 * plane + pix : nullptr;
-    float dy[MAX_TAPS], dx[MAX_TAPS], mk[MAX_TAPS];
+    float dy[TAPS_PER_PART], dx[TAPS_PER_PART], mk[TAPS_PER_PART];
 #pragma unroll
-    for (int t = 0; t < MAX_TAPS; ++t) {
-        dy[t] = dx[t] = 0.f;
-        mk[t] = 1.f;
-        if (pv && t < s.K2) {
-            dy[t] = __ldg(offp + (size_t)(2 * t) * plane);
-            dx[t] = __ldg(offp + (size_t)(2 * t + 1) * plane);
-            if (mp) mk[t] = __ldg(mp + (size_t)t * plane);
+    for (int j = 0; j < TAPS_PER_PART; ++j) {
+        const int t = tp_lo + j;
+        dy[j] = dx[j] = 0.f;
+        mk[j] = 1.f;
+        if (pv && t < tp_hi) {
+            dy[j] = __ldg(offp + (size_t)(2 * t) * plane);
+            dx[j] = __ldg(offp + (size_t)(2 * t + 1) * plane);
+            if (mp) mk[j] = __ldg(mp + (size_t)t * plane);
         }
     }
 
@@ -142,49 +148,56 @@ __global__ void __launch_bounds__(THREADS) stem_tc_kernel(const __grid_constant_
                                         __float_as_uint(lo[3])));
     }
 
-    // ---- the row's modulated samples: col[tap*Cin + c]
-    float col[KP];
-#pragma unroll
-    for (int k = 0; k < KP; ++k) col[k] = 0.f;
+    // ---- this thread's modulated samples: k = tap*Cin + c for its taps
     const float* xb = a.x + (size_t)bb * s.H * s.W * CIN;
+    const uint32_t arow = ptx::smem_u32(sA) + (uint32_t)row * 128;
 #pragma unroll
-    for (int t = 0; t < MAX_TAPS; ++t) {
-        if (t >= s.K2 || !pv) continue;
-        const int ti = t / s.K, tj = t - ti * s.K;
-        int y0, x0;
-        float ly, lx;
-        split_coord(oy + ti * s.dil, dy[t], y0, ly);
-        split_coord(ox + tj * s.dil, dx[t], x0, lx);
-        float wt[4], v[4][CIN];
+    for (int j = 0; j < TAPS_PER_PART; ++j) {
+        const int t = tp_lo + j;
+        if (t >= tp_hi) break;
+        float col[CIN];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int r = y0 + (q >> 1), cc = x0 + (q & 1);
-            wt[q] = 0.f;
+        for (int c = 0; c < CIN; ++c) col[c] = 0.f;
+        if (pv) {
+            const int ti = t / s.K, tj = t - ti * s.K;
+            int y0, x0;
+            float ly, lx;
+            split_coord(oy + ti * s.dil, dy[j], y0, ly);
+            split_coord(ox + tj * s.dil, dx[j], x0, lx);
+            float wt[4], v[4][CIN];
 #pragma unroll
-            for (int c = 0; c < CIN; ++c) v[q][c] = 0.f;
-            if (!inside(s, r, cc)) continue;
-            wt[q] = ((q >> 1) ? ly : 1.f - ly) * ((q & 1) ? lx : 1.f - lx) * mk[t];
-            const float* pc = xb + ((size_t)r * s.W + cc) * CIN;
+            for (int q = 0; q < 4; ++q) {
+                const int r = y0 + (q >> 1), cc = x0 + (q & 1);
+                wt[q] = 0.f;
 #pragma unroll
-            for (int c = 0; c < CIN; ++c) v[q][c] = __ldg(pc + c);
+                for (int c = 0; c < CIN; ++c) v[q][c] = 0.f;
+                if (!inside(s, r, cc)) continue;
+                wt[q] = ((q >> 1) ? ly : 1.f - ly) * ((q & 1) ? lx : 1.f - lx) * mk[j];
+                const float* pc = xb + ((size_t)r * s.W + cc) * CIN;
+#pragma unroll
+                for (int c = 0; c < CIN; ++c) v[q][c] = __ldg(pc + c);
+            }
+#pragma unroll
+            for (int c = 0; c < CIN; ++c)
+                col[c] = wt[0] * v[0][c] + wt[1] * v[1][c] + wt[2] * v[2][c] + wt[3] * v[3][c];
         }
+        // element k of the row: 16-byte chunk k/4 (swizzled by row), word k%4
 #pragma unroll
-        for (int c = 0; c < CIN; ++c)
-            col[t * CIN + c] = wt[0] * v[0][c] + wt[1] * v[1][c] + wt[2] * v[2][c] + wt[3] * v[3][c];
+        for (int c = 0; c < CIN; ++c) {
+            const int k = t * CIN + c;
+            const float hi = ptx::to_tf32(col[c]);
+            const uint32_t o = arow + ((((k >> 2) ^ (row & 7)) << 4) | ((k & 3) << 2));
+            ptx::sts_f32(o, hi);
+            ptx::sts_f32(o + TILE_BYTES, col[c] - hi);
+        }
     }
-#pragma unroll
-    for (int c = 0; c < KP / 4; ++c) {
-        float hi[4], lo[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            hi[j] = ptx::to_tf32(col[4 * c + j]);
-            lo[j] = col[4 * c + j] - hi[j];
+    if (part == PARTS - 1) {
+        // zero padding of the contraction depth, in both A tiles
+        for (int k = KC; k < KP; ++k) {
+            const uint32_t o = arow + ((((k >> 2) ^ (row & 7)) << 4) | ((k & 3) << 2));
+            ptx::sts_f32(o, 0.f);
+            ptx::sts_f32(o + TILE_BYTES, 0.f);
         }
-        const uint32_t o = ptx::smem_u32(sA) + sw_chunk(tid, c);
-        ptx::sts_v4(o, make_uint4(__float_as_uint(hi[0]), __float_as_uint(hi[1]), __float_as_uint(hi[2]),
-                                  __float_as_uint(hi[3])));
-        ptx::sts_v4(o + TILE_BYTES, make_uint4(__float_as_uint(lo[0]), __float_as_uint(lo[1]),
-                                               __float_as_uint(lo[2]), __float_as_uint(lo[3])));
     }
 
     // ---- contraction on the tensor cores
@@ -213,7 +226,8 @@ __global__ void __launch_bounds__(THREADS) stem_tc_kernel(const __grid_constant_
     ptx::tc_fence_after();
 
     // ---- epilogue: TMEM -> registers (+ bias) -> swizzled staging -> TMA stores
-    if (ok) {
+    if (ok && warp < 4) {
+        // warps 0-3 reach TMEM lanes 0-127 (a warp reads the lane quarter of its index mod 4)
         const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
         for (int cb = 0; cb < s.Cout / 32; ++cb) {
             float v[32];
