@@ -93,3 +93,29 @@ def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(dcn, "_LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="not built"):
         dcn._load()
+
+
+F32, BF16 = 0, 1
+
+
+@pytest.mark.parametrize("kw,flags,expect", [
+    # float32 RGB-like layers: the split-tf32 tensor-core kernel
+    (dict(B=1, H=224, W=224, Cin=3, Cout=64, G=1, dtype=F32), 0, "tcgen05_tf32_split"),
+    (dict(B=1, H=224, W=224, Cin=3, Cout=64, G=1, dtype=F32), dcn.DCN_FLAG_NO_TF32, "f32_small_channels"),
+    (dict(B=1, H=224, W=224, Cin=3, Cout=64, G=1, dtype=F32), dcn.DCN_FLAG_GENERIC, "generic"),
+    (dict(B=1, H=20, W=21, Cin=1, Cout=256, G=1, dtype=F32), 0, "tcgen05_tf32_split"),
+    # outside the split-tf32 kernel's shapes: Cin > 3, K*K > 9, groups, Cout not a multiple of 32
+    (dict(B=1, H=31, W=17, Cin=4, Cout=64, G=1, dtype=F32), 0, "f32_small_channels"),
+    (dict(B=2, H=9, W=12, Cin=1, Cout=32, K=5, pad=2, G=1, dtype=F32), 0, "f32_small_channels"),
+    (dict(B=2, H=6, W=9, Cin=2, Cout=32, G=2, dtype=F32), 0, "f32_small_channels"),
+    (dict(B=1, H=16, W=16, Cin=3, Cout=48, G=1, dtype=F32), 0, "generic"),
+    (dict(B=1, H=16, W=16, Cin=16, Cout=64, G=1, dtype=F32), 0, "generic"),
+    # bfloat16: the tcgen05 gather kernel for channel counts in multiples of 8
+    (dict(B=8, H=50, W=50, Cin=256, Cout=256, G=1, dtype=BF16), 0, "tcgen05_gather"),
+    (dict(B=8, H=50, W=50, Cin=256, Cout=256, G=1, dtype=BF16), dcn.DCN_FLAG_GENERIC, "generic"),
+    (dict(B=8, H=25, W=25, Cin=512, Cout=512, G=4, pad=2, dil=2, dtype=BF16), 0, "tcgen05_gather"),
+    (dict(B=1, H=9, W=9, Cin=12, Cout=16, G=1, dtype=BF16), 0, "generic"),
+])
+def test_forward_dispatch(lib, kw, flags, expect):
+    """Which forward kernel a layer gets, decided on the host before any launch."""
+    assert dcn.forward_path(P(flags=flags, **kw)) == expect
