@@ -6,23 +6,27 @@
 // deformable convolution: the "Deformable ConvNets" notes, im2col appendix and
 // the y(p0) equations). Col is never written to HBM:
 //
-//   * producer warps (8) compute the sampling coordinates of a 128-pixel tile,
-//     load the four channel-contiguous NHWC neighbours of each sample as 32-byte
-//     vectors (16 channels per lane), blend them with the bilinear weights times
-//     the mask, and store the bf16 result straight into a shared-memory A tile
-//     laid out in the UMMA 128-byte-swizzle K-major canonical form;
+//   * producer warps (8) gather every chunk (one tap, 64 channels): each lane
+//     loads the four channel-contiguous NHWC neighbours of a sample as 32-byte
+//     vectors (16 channels), blends them with the bilinear weights times the
+//     mask, and stores the bf16 result straight into a shared-memory A tile laid
+//     out in the UMMA 128-byte-swizzle K-major canonical form; a thread owns two
+//     rows and issues the next chunk's loads for a row right after blending it;
 //   * one TMA warp stages the matching weight tile [N x 64] of W = [Cout, K*K*Cin];
 //   * one MMA warp issues tcgen05.mma (M=128, N<=256, K=16) into TMEM;
-//   * four epilogue warps read the accumulator back with tcgen05.ld, add the
+//   * four epilogue warps build the sampling records (bilinear weights times the
+//     mask, top-left neighbour, neighbours to read) one (tile, group) epoch ahead
+//     of the producers, and read the accumulator back with tcgen05.ld, add the
 //     bias and store bf16 NHWC rows.
 //
 // The K loop runs over (group, 64-channel chunk, tap), taps innermost, so that
 // consecutive chunks gather from the same 128-byte channel slice of nearby
 // pixels while it is in L1. Work is split stream-K style: the (tile, chunk)
-// units are divided evenly over one persistent CTA per SM; a tile that two or
-// more CTAs share is summed from float32 partial tiles in the workspace by the
-// CTA that finishes it last (counted with an atomic per tile; no CTA waits on
-// another). Every wait is bounded and reports a timeout through the status word.
+// units are divided evenly over one persistent CTA per SM (no CTA starting in
+// the last units of a tile); a tile that two or more CTAs share is summed from
+// float32 partial tiles in the workspace, in contributor order, by the CTA that
+// finishes it last (counted with an atomic per tile; no CTA waits on another).
+// Every wait is bounded and reports a timeout through the status word.
 #include <cudaTypedefs.h>
 
 #include <mutex>

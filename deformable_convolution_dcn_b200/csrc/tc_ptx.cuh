@@ -327,10 +327,6 @@ __device__ __forceinline__ void ldg4_pred(uint4 (&v)[4], const void* p0, const v
         : "r"(mask), "l"(p0), "l"(p1), "l"(p2), "l"(p3));
 }
 
-__device__ __forceinline__ void prefetch_l1(const void* p) {
-    asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
-}
-
 __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
     int v;
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
