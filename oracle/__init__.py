@@ -80,6 +80,7 @@ def _bind(lib):
     lib.dcn_oracle_grad_offset_mask_pixels.argtypes = [sp, dp, dp, dp, dp, dp, L, lp, dp, dp]
     lib.dcn_oracle_grad_weight_entries.argtypes = [sp, dp, dp, dp, dp, L, lp, dp]
     lib.dcn_oracle_grad_x_entries.argtypes = [sp, dp, dp, dp, dp, L, lp, dp]
+    lib.dcn_oracle_predict_offset_mask.argtypes = [sp, dp, dp, dp, dp, dp]
     return lib
 
 
@@ -241,3 +242,23 @@ def grad_x_at(x_shape, offset, mask, weight, grad_y, entries, stride=1, pad=0, d
     if rc != 0:
         raise ValueError("oracle rc=%d" % rc)
     return out
+
+
+def predict_offset_mask(x, w_pred, b_pred, K, stride=1, pad=0, dil=1, G=1, lib=None):
+    """(offset [B, 2GK^2, Ho, Wo], mask [B, GK^2, Ho, Wo]) of a DCNv2 layer from its
+    predictor convolution w_pred [3GK^2, K, K, Cin] (+ b_pred [3GK^2] or None)."""
+    lib = lib or load()
+    B, H, W, Cin = x.shape
+    assert tuple(w_pred.shape) == (3 * G * K * K, K, K, Cin), w_pred.shape
+    s = _shape(B, H, W, Cin, 3 * G * K * K, K, stride, pad, dil, G)
+    Ho, Wo = lib.dcn_oracle_out_h(ctypes.byref(s)), lib.dcn_oracle_out_w(ctypes.byref(s))
+    xs, xp = _d(x)
+    ws, wp = _d(w_pred)
+    bs, bp = _d(b_pred)
+    off = np.zeros((B, 2 * G * K * K, Ho, Wo))
+    mask = np.zeros((B, G * K * K, Ho, Wo))
+    rc = lib.dcn_oracle_predict_offset_mask(ctypes.byref(s), xp, wp, bp, off.ctypes.data_as(ctypes.POINTER(ctypes.c_double)),
+                                            mask.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
+    if rc != 0:
+        raise ValueError("oracle predictor rejected the shape (rc=%d)" % rc)
+    return off, mask

@@ -367,3 +367,43 @@ int dcn_oracle_grad_x_entries(const dcn_oracle_shape* s, const double* off, cons
     }
     return 0;
 }
+
+/* --------------------------------------------------- offset/mask predictor -- */
+
+/* The offsets and modulation scalars of a DCNv2 layer come from a separate
+ * plain convolution over the same input, at the layer's own spatial resolution
+ * (here: the layer's kernel size, stride, padding and dilation), with 3 output
+ * channels per tap and group: the first 2*G*K*K outputs are the offsets, the
+ * remaining G*K*K pass through a sigmoid and become the masks (notes, DCNv2
+ * section 3.2, the paragraph after the modulated y(p0) equation).
+ *   wp   [3*G*K*K, K, K, Cin]      bp [3*G*K*K] (NULL: no bias)
+ *   off  [B, 2*G*K*K, Ho, Wo]      mask [B, G*K*K, Ho, Wo]
+ * s->Cout is not used. */
+int dcn_oracle_predict_offset_mask(const dcn_oracle_shape* s, const double* x, const double* wp, const double* bp,
+                                   double* off, double* mask) {
+    if (s->G <= 0 || s->K <= 0) return -1;
+    const int Ho = dcn_oracle_out_h(s), Wo = dcn_oracle_out_w(s);
+    const int K2 = s->K * s->K, NO = 2 * s->G * K2, NM = s->G * K2;
+    long row;
+    const long rows = (long)s->B * Ho;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (row = 0; row < rows; ++row) {
+        const int b = (int)(row / Ho), ho = (int)(row % Ho);
+        for (int wo = 0; wo < Wo; ++wo) {
+            for (int ch = 0; ch < NO + NM; ++ch) {
+                double acc = bp ? bp[ch] : 0.0;
+                for (int i = 0; i < s->K; ++i)
+                    for (int j = 0; j < s->K; ++j)
+                        for (int c = 0; c < s->Cin; ++c)
+                            acc += wp[(((size_t)ch * s->K + i) * s->K + j) * s->Cin + c] *
+                                   pixel_or_zero(x, s, b, ho * s->stride - s->pad + i * s->dil,
+                                                 wo * s->stride - s->pad + j * s->dil, c);
+                if (ch < NO)
+                    off[(((size_t)b * NO + ch) * Ho + ho) * Wo + wo] = acc;
+                else
+                    mask[(((size_t)b * NM + (ch - NO)) * Ho + ho) * Wo + wo] = 1.0 / (1.0 + exp(-acc));
+            }
+        }
+    }
+    return 0;
+}

@@ -318,4 +318,40 @@ def pin_sampled_entries_match_full(lib):
                                                 *a, lib=lib), g["grad_x"].reshape(-1)[xe], atol=1e-12)
 
 
+# ------------------------------------------------ offset/mask predictor --
+
+def pin_predictor_is_conv2d_split_sigmoid(lib):
+    """The predictor is torch's own conv2d (float64) with the layer's geometry;
+    its first 2GK^2 output channels are the offsets and the rest, through
+    torch.sigmoid, the masks. Swept over K, stride, padding, dilation, groups."""
+    for n, (K, stride, pad, dil, G) in enumerate([(3, 1, 1, 1, 1), (3, 2, 1, 1, 2), (1, 1, 0, 1, 1),
+                                                   (3, 1, 2, 2, 1), (5, 1, 2, 1, 1)]):
+        r = _rng(200 + n)
+        B, H, W, Cin, NC = 2, 7, 9, 3, 3 * G * K * K
+        x = r.standard_normal((B, H, W, Cin))
+        w = r.standard_normal((NC, K, K, Cin)) * 0.3
+        b = r.standard_normal(NC)
+        off, mask = oracle.predict_offset_mask(x, w, b, K, stride, pad, dil, G, lib=lib)
+        ref = _conv2d_ref(x, w, b, stride, pad, dil).transpose(0, 3, 1, 2)  # [B, NC, Ho, Wo]
+        NO = 2 * G * K * K
+        assert off.shape == ref[:, :NO].shape and mask.shape == ref[:, NO:].shape
+        assert np.allclose(off, ref[:, :NO], rtol=1e-12, atol=1e-12)
+        assert np.allclose(mask, torch.sigmoid(torch.from_numpy(ref[:, NO:])).numpy(), rtol=1e-12, atol=1e-12)
+
+
+def pin_predictor_bias_only(lib):
+    """Zero weights: the offsets equal the bias everywhere; with no bias the
+    masks are exactly 1/2 (the logistic function at 0)."""
+    r = _rng(210)
+    K, G = 3, 2
+    NC = 3 * G * K * K
+    x = r.standard_normal((1, 6, 5, 4))
+    w = np.zeros((NC, K, K, 4))
+    b = r.standard_normal(NC)
+    off, mask = oracle.predict_offset_mask(x, w, b, K, 1, 1, 1, G, lib=lib)
+    assert np.array_equal(off, np.broadcast_to(b[:2 * G * K * K, None, None], off.shape[1:])[None].repeat(1, 0))
+    off0, mask0 = oracle.predict_offset_mask(x, w, None, K, 1, 1, 1, G, lib=lib)
+    assert np.all(off0 == 0.0) and np.all(mask0 == 0.5)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

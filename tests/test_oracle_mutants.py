@@ -45,6 +45,10 @@ MUTANTS = {
                             "*px = (double)(wo - s->pad + j * s->dil) + dx;"),
     "dilation_ignored": ("*py = (double)(ho * s->stride - s->pad + i * s->dil) + dy;",
                          "*py = (double)(ho * s->stride - s->pad + i) + dy;"),
+    "predictor_sigmoid_sign": ("= 1.0 / (1.0 + exp(-acc));", "= 1.0 / (1.0 + exp(acc));"),
+    "predictor_mask_not_squashed": ("= 1.0 / (1.0 + exp(-acc));", "= acc;"),
+    "predictor_dilation_ignored_in_x": ("wo * s->stride - s->pad + j * s->dil, c);",
+                                        "wo * s->stride - s->pad + j, c);"),
 }
 
 
