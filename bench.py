@@ -492,6 +492,96 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_predictor(args):
+    """Times the offset/mask predictor of the workload's layer (dcn_predict_offset_mask:
+    a plain convolution with 3*G*K*K outputs, offsets and sigmoid masks) on its own."""
+    import torch
+
+    import deformable_convolution_dcn_b200 as dcn
+    from deformable_convolution_dcn_b200 import inputs as gen
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist_init("nccl")
+    w = gen.WORKLOADS[args.workload]
+    s = w.shape
+    elem = 2 if w.dtype == "bf16" else 4
+    nc = 3 * s.G * s.K * s.K
+    work = {"flops": 2.0 * s.P * nc * s.K * s.K * s.Cin,
+            "bytes": elem * (s.B * s.H * s.W * s.Cin + nc * s.K * s.K * s.Cin + nc + s.P * nc)}
+    pk, pk_src = peaks()
+    host = gen.predictor_inputs(w.seed, s, w.dtype)
+    set_bytes = sum(t.numel() * t.element_size() for t in host.values() if t is not None) + elem * s.P * nc
+    n_sets = max(2, min(64, math.ceil(3 * L2_BYTES / set_bytes) + 1))
+    sets = [{k: (None if t is None else t.to(device)) for k, t in host.items()} for _ in range(n_sets)]
+    dt = host["x"].dtype
+    outs = [(torch.empty((s.B, 2 * s.G * s.K * s.K, s.Ho, s.Wo), dtype=dt, device=device),
+             torch.empty((s.B, s.G * s.K * s.K, s.Ho, s.Wo), dtype=dt, device=device)) for _ in range(n_sets)]
+    p = dcn.make_params(s.B, s.H, s.W, s.Cin, 1, s.K, s.stride, s.pad, s.dil, s.G, dcn._DTYPES[dt])
+    ws = torch.empty(dcn.predict_workspace_size(p), dtype=torch.uint8, device=device)
+
+    def run(k):
+        d = sets[k % n_sets]
+        dcn.predict_offset_mask(d["x"], d["w_pred"], d["b_pred"], s.K, s.stride, s.pad, s.dil, s.G,
+                                workspace=ws, out=outs[k % n_sets])
+
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        for k in range(max(args.warmup, n_sets)):
+            run(k)
+    torch.cuda.synchronize()
+    dcn.check_status()
+    graphs = []
+    with torch.cuda.stream(stream):
+        for k in range(n_sets):
+            l0 = dcn.launch_count()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                run(k)
+            launches_per_step = dcn.launch_count() - l0
+            graphs.append(g)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for k in range(args.warmup):
+            graphs[k % n_sets].replay()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(device)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(int(HOLD_CYCLES_PER_STEP * (args.steps + 4)))
+        t0.record(stream)
+        for k in range(args.steps):
+            graphs[(args.warmup + k) % n_sets].replay()
+        t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(device)
+    clk = clocks.stop()
+    dcn.check_status()
+    ms = max_over_ranks(t0.elapsed_time(t1), device) / args.steps
+    rl = roofline_entry(work, ms / 1e3, pk, sustained=False)
+    rl.update({"kernel": "predictor", "traffic": load_traffic(args.workload, "predictor"),
+               "peak_source": pk_src + " (burst bf16, HBM copy)"})
+    if rank == 0:
+        print(json.dumps({
+            "metric": "DCNv2 offset/mask predictor TFLOP/s", "value": round(world * work["flops"] / ms / 1e9, 2),
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": "offset/mask predictor of: " + w.description, "outputs": nc,
+                       "l2": "inputs and outputs rotate over %d independent sets" % n_sets,
+                       "forward_path_inner": dcn.forward_path(dcn.make_params(
+                           s.B, s.H, s.W, s.Cin, (nc + 31) // 32 * 32, s.K, s.stride, s.pad, s.dil, 1,
+                           dcn._DTYPES[dt]))},
+            "roofline": rl, "gpu_launches": launches_per_step * args.steps, "clocks": clk}), flush=True)
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -500,6 +590,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="conv4", help="conv4 | conv3_s2 | conv5_d2g4 | stem | tiny | conv4_bwd")
     ap.add_argument("--forward-only", action="store_true", help="time the forward alone (not the default step)")
+    ap.add_argument("--predictor", action="store_true",
+                    help="time the layer's offset/mask predictor instead of the default step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args(argv)
@@ -509,6 +601,8 @@ def main(argv=None):
         args.workload = "conv4"
     if args.impl == "reference":
         run_reference(args)
+    elif args.predictor:
+        run_predictor(args)
     else:
         run_ours(args)
 

@@ -77,6 +77,9 @@ def _load():
         lib.dcn_backward_input.argtypes = [P, vp, vp, vp, vp, vp, fp, vp, sz, vp]
         lib.dcn_backward_offset_mask.argtypes = [P, vp, vp, vp, vp, vp, fp, fp, vp, sz, vp]
         lib.dcn_backward_weight.argtypes = [P, vp, vp, vp, vp, fp, fp, vp, sz, vp]
+        lib.dcn_predict_workspace_size.argtypes = [P]
+        lib.dcn_predict_workspace_size.restype = sz
+        lib.dcn_predict_offset_mask.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
         lib.dcn_last_error_string.restype = ctypes.c_char_p
         lib.dcn_check_status.restype = ctypes.c_int
         lib.dcn_launch_count.restype = ctypes.c_ulonglong
@@ -194,6 +197,44 @@ def forward_noalloc(x, offset, mask, weight, bias=None, stride=1, padding=0, dil
     _check(lib.dcn_forward_noalloc(ctypes.byref(p), _ptr(x), _ptr(offset), _ptr(mask), _ptr(weight), _ptr(bias),
                                    _ptr(out), _stream(x.device)))
     return out
+
+
+def predict_workspace_size(p: Params) -> int:
+    return int(_load().dcn_predict_workspace_size(ctypes.byref(p)))
+
+
+def predict_offset_mask(x, w_pred, b_pred, K, stride=1, padding=0, dilation=1, G=1, *, workspace=None,
+                        generic=False, out=None):
+    """The offsets [B, 2GK^2, Ho, Wo] and masks [B, GK^2, Ho, Wo] of a DCNv2 layer with kernel size K, stride,
+    padding, dilation and G offset groups, from its predictor convolution w_pred [3GK^2, K, K, Cin]
+    (+ b_pred [3GK^2] or None) over x [B, H, W, Cin]. out: optional (offset, mask) to write."""
+    lib = _load()
+    if x.dim() != 4 or w_pred.dim() != 4:
+        raise ValueError("x must be [B, H, W, Cin] and w_pred [3*G*K*K, K, K, Cin]")
+    if x.dtype not in _DTYPES:
+        raise TypeError("x must be float32 or bfloat16, got %s" % x.dtype)
+    B, H, W, Cin = x.shape
+    if tuple(w_pred.shape) != (3 * G * K * K, K, K, Cin):
+        raise ValueError("w_pred must be %s, got %s" % ((3 * G * K * K, K, K, Cin), tuple(w_pred.shape)))
+    if b_pred is not None and tuple(b_pred.shape) != (3 * G * K * K,):
+        raise ValueError("b_pred must be [%d]" % (3 * G * K * K))
+    p = make_params(B, H, W, Cin, 1, K, stride, padding, dilation, G, _DTYPES[x.dtype],
+                    DCN_FLAG_GENERIC if generic else 0)
+    Ho, Wo = output_size(p)
+    if out is None:
+        out = (torch.empty((B, 2 * G * K * K, Ho, Wo), dtype=x.dtype, device=x.device),
+               torch.empty((B, G * K * K, Ho, Wo), dtype=x.dtype, device=x.device))
+    offset, mask = out
+    if tuple(offset.shape) != (B, 2 * G * K * K, Ho, Wo) or tuple(mask.shape) != (B, G * K * K, Ho, Wo):
+        raise ValueError("out must be (offset %s, mask %s)" % ((B, 2 * G * K * K, Ho, Wo), (B, G * K * K, Ho, Wo)))
+    _check_tensors(x.dtype, x.device, x=x, w_pred=w_pred, b_pred=b_pred, offset=offset, mask=mask)
+    n = predict_workspace_size(p)
+    if workspace is None:
+        workspace = torch.empty(n, dtype=torch.uint8, device=x.device)
+    _check(lib.dcn_predict_offset_mask(ctypes.byref(p), _ptr(x), _ptr(w_pred), _ptr(b_pred), _ptr(offset),
+                                       _ptr(mask), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                       _stream(x.device)))
+    return offset, mask
 
 
 def backward_data(x, offset, mask, weight, grad_y, stride=1, padding=0, dilation=1, *, need_input=True,

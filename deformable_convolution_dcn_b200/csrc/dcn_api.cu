@@ -351,6 +351,93 @@ int dcn_backward_weight(const dcn_params_t* params, const void* x, const void* o
     return ok();
 }
 
+// ------------------------------------------------- offset/mask predictor --
+
+// The predictor is the plain convolution with the layer's kernel size, stride,
+// padding and dilation and 3*G*K*K outputs (run as this library's layer with
+// zero offsets, no mask, one group and the outputs padded to a multiple of 32).
+// Workspace pieces, each 256-byte aligned: the zero offsets, the padded weights
+// and bias, the [P, NP] result, and the inner forward's own workspace.
+struct PredPlan {
+    dcn_params_t q;   // the inner plain convolution
+    int nc, np, no;   // 3GK^2 outputs, rounded up to 32, of which 2GK^2 offsets
+    size_t zoff, wpad, bpad, ypred, fws, fws_bytes, total;
+};
+
+static int pred_plan(const dcn_params_t* p, PredPlan& pl, dcn::Shape& s) {
+    if (!p) return fail(DCN_ERR_INVALID_ARG, "params is NULL");
+    dcn_params_t lay = *p;
+    lay.Cout = 1;  // the layer's Cout plays no part in the predictor
+    TRY(make_shape(&lay, s));
+    pl.nc = 3 * p->G * s.K2;
+    pl.no = 2 * p->G * s.K2;
+    pl.np = (pl.nc + 31) / 32 * 32;
+    pl.q = lay;
+    pl.q.Cout = pl.np;
+    pl.q.G = 1;
+    dcn::Shape sq;
+    TRY(make_shape(&pl.q, sq));
+    const size_t es = elem_size(p->dtype);
+    auto up = [](size_t v) { return (v + 255) & ~(size_t)255; };
+    size_t o = 0;
+    pl.zoff = o;
+    o = up(o + es * (size_t)s.P * 2 * s.K2);
+    pl.wpad = o;
+    o = up(o + es * (size_t)pl.np * s.KC);
+    pl.bpad = o;
+    o = up(o + es * (size_t)pl.np);
+    pl.ypred = o;
+    o = up(o + es * (size_t)s.P * pl.np);
+    pl.fws = o;
+    pl.fws_bytes = dcn_workspace_size(&pl.q, DCN_OP_FORWARD);
+    pl.total = up(o + pl.fws_bytes);
+    return DCN_OK;
+}
+
+size_t dcn_predict_workspace_size(const dcn_params_t* params) {
+    PredPlan pl;
+    dcn::Shape s;
+    std::string keep = g_err;
+    if (pred_plan(params, pl, s) != DCN_OK) {
+        g_err = keep;
+        return 0;
+    }
+    return pl.total;
+}
+
+int dcn_predict_offset_mask(const dcn_params_t* params, const void* x, const void* w_pred, const void* b_pred,
+                            void* offset, void* mask, void* workspace, size_t workspace_bytes, void* stream) {
+    PredPlan pl;
+    dcn::Shape s;
+    TRY(pred_plan(params, pl, s));
+    const size_t es = elem_size(params->dtype);
+    TRY(check_ptr(x, "x", es, true));
+    TRY(check_ptr(w_pred, "w_pred", es, true));
+    TRY(check_ptr(b_pred, "b_pred", es, false));
+    TRY(check_ptr(offset, "offset", es, true));
+    TRY(check_ptr(mask, "mask", es, true));
+    if (!workspace || workspace_bytes < pl.total)
+        return fail(DCN_ERR_WORKSPACE, "the predictor needs %zu bytes of workspace, got %zu", pl.total,
+                    workspace ? workspace_bytes : (size_t)0);
+    TRY(check_ptr(workspace, "workspace", 256, true));
+    cudaStream_t st = (cudaStream_t)stream;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const int bf = params->dtype == DCN_BF16;
+    cudaError_t e = cudaMemsetAsync(ws + pl.zoff, 0, es * (size_t)s.P * 2 * s.K2, st);
+    g_launches += 1;
+    if (e != cudaSuccess) return cuda_fail(e, "zeroing the predictor's offsets");
+    e = dcn::predict_pad(bf, w_pred, b_pred, ws + pl.wpad, ws + pl.bpad, pl.nc, pl.np, s.KC, st);
+    g_launches += 1;
+    if (e != cudaSuccess) return cuda_fail(e, "padding the predictor weights");
+    const int rc = dcn_forward(&pl.q, x, ws + pl.zoff, nullptr, ws + pl.wpad, ws + pl.bpad, ws + pl.ypred,
+                               ws + pl.fws, pl.fws_bytes, stream);
+    if (rc != DCN_OK) return rc;
+    e = dcn::predict_split(bf, ws + pl.ypred, offset, mask, s.P, s.Ho * s.Wo, pl.np, pl.no, pl.nc, st);
+    g_launches += 1;
+    if (e != cudaSuccess) return cuda_fail(e, "splitting the predictor output");
+    return ok();
+}
+
 const char* dcn_last_error_string(void) { return g_err.c_str(); }
 
 int dcn_check_status(void) {

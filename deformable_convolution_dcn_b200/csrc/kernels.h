@@ -29,6 +29,12 @@ size_t fwd_tc_static_scratch_bytes();
 cudaError_t fwd_tc_noalloc(const Shape& s, const void* x, const void* off, const void* mask, const void* w,
                            const void* bias, void* y, unsigned* status, cudaStream_t st, int* launches);
 
+// predict.cu — the offset/mask predictor's weight padding and output split.
+cudaError_t predict_pad(int dtype_bf16, const void* w, const void* b, void* wpad, void* bpad, int nc, int np, int kc,
+                        cudaStream_t st);
+cudaError_t predict_split(int dtype_bf16, const void* y, void* off, void* mask, int P, int plane, int np, int no,
+                          int nc, cudaStream_t st);
+
 // fwd_f32_tc.cu — float32 forward for layers with Cin <= 3, K*K <= 9 on tcgen05
 // (split tf32 operands, float32 accuracy); y 16-byte aligned.
 bool fwd_f32_tc_supported(const Shape& s);

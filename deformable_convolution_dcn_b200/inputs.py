@@ -208,6 +208,25 @@ def random_case(seed: int, dtype: str = "f32", B=None, Cin=None, H=None, W=None,
     return s, {k: (None if v is None else v.to(dt).to(device)) for k, v in out.items()}
 
 
+def predictor_inputs(seed: int, s: LayerShape, dtype: str = "f32", bias: bool = True, device="cpu"):
+    """Inputs of a layer's offset/mask predictor: x [B, H, W, Cin], w_pred
+    [3*G*K*K, K, K, Cin] and b_pred [3*G*K*K] (None without bias).
+
+    DCNv2 starts the predictor at zero weights (DCNv2 section 3.2); a trained
+    one does not stay there, so the weights here are normal with std
+    1/sqrt(Cin*K*K) (outputs of unit scale: offsets of about one pixel, masks
+    spread over (0, 1)) and the bias is normal with std 0.5. s.Cout is unused.
+    """
+    g = torch.Generator().manual_seed(seed)
+    nc = 3 * s.G * s.K * s.K
+    x = torch.randn((s.B, s.Cin, s.H, s.W), generator=g).permute(0, 2, 3, 1).contiguous()
+    w = torch.randn((nc, s.Cin, s.K, s.K), generator=g) / math.sqrt(s.Cin * s.K * s.K)
+    b = torch.randn((nc,), generator=g) * 0.5 if bias else None
+    out = {"x": x, "w_pred": w.permute(0, 2, 3, 1).contiguous(), "b_pred": b}
+    dt = torch_dtype(dtype)
+    return {k: (None if v is None else v.to(dt).to(device)) for k, v in out.items()}
+
+
 def as_f64(t):
     """numpy float64 copy of a tensor's stored values (None passes through)."""
     if t is None:

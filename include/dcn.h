@@ -167,6 +167,31 @@ DCN_API int dcn_backward_weight(const dcn_params_t* params, const void* x, const
 DCN_API int dcn_forward_noalloc(const dcn_params_t* params, const void* x, const void* offset, const void* mask,
                                 const void* weight, const void* bias, void* y, void* stream);
 
+/* Offset/mask predictor of a DCNv2 layer (notes, DCNv2 section 3.2, the
+ * paragraph after the modulated y(p0) equation): a plain convolution over the
+ * layer's input x with the layer's kernel size, stride, padding and dilation
+ * and 3*G*K*K output channels. The first 2*G*K*K outputs are the offsets, the
+ * remaining G*K*K pass through a sigmoid, 1 / (1 + exp(-v)), computed in
+ * float32, and are the masks. params describes the DCN layer the outputs feed:
+ * B, H, W, Cin, K, stride, pad, dil, G, dtype and flags are used, Cout is not.
+ *   x       [B, H, W, Cin]                (as for dcn_forward)
+ *   w_pred  [3*G*K*K, K, K, Cin]          (output channel, tap row, tap column, input channel)
+ *   b_pred  [3*G*K*K], may be NULL (no bias)
+ *   offset  [B, 2*G*K*K, Ho, Wo]          written; the layout dcn_forward reads
+ *   mask    [B, G*K*K, Ho, Wo]            written
+ * All in params->dtype, device memory owned by the caller, element-aligned.
+ * workspace: device memory of at least dcn_predict_workspace_size(params)
+ * bytes, 256-byte aligned, used as scratch for the duration of the stream
+ * work. The convolution runs on this library's forward kernels with zero
+ * offsets and no mask, one group and the outputs padded to a multiple of 32,
+ * so its precision is the forward's for that layer shape.
+ * Errors as for dcn_forward: argument problems return before anything is
+ * enqueued; DCN_ERR_WORKSPACE when workspace is NULL or too small. */
+DCN_API size_t dcn_predict_workspace_size(const dcn_params_t* params);
+DCN_API int dcn_predict_offset_mask(const dcn_params_t* params, const void* x, const void* w_pred,
+                                    const void* b_pred, void* offset, void* mask, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
 /* The calling thread's last error message ("" after success). */
 DCN_API const char* dcn_last_error_string(void);
 

@@ -87,6 +87,29 @@ def test_misaligned_pointers(lib):
     assert lib.dcn_backward_weight(ctypes.byref(p16), f, f, None, f, odd, None, None, 0, None) == EUNSUP
 
 
+def test_predictor_arguments(lib):
+    f = ctypes.c_void_p(1 << 20)
+    p = P()
+    n = lib.dcn_predict_workspace_size(ctypes.byref(p))
+    # at least the zero offsets, the padded weights and the [P, 32] result
+    P_ = 2 * 9 * 8
+    assert n >= 4 * (P_ * 18 + 32 * 9 * 8 + P_ * 32)
+    assert n % 256 == 0
+    # Cout plays no part
+    assert lib.dcn_predict_workspace_size(ctypes.byref(P(Cout=77))) == n
+    assert lib.dcn_predict_workspace_size(ctypes.byref(P(B=0))) == 0
+    assert lib.dcn_predict_offset_mask(ctypes.byref(P(B=0)), f, f, None, f, f, f, n, None) == EINVAL
+    assert lib.dcn_predict_offset_mask(ctypes.byref(p), None, f, None, f, f, f, n, None) == EINVAL
+    assert lib.dcn_predict_offset_mask(ctypes.byref(p), f, f, None, f, None, f, n, None) == EINVAL
+    assert lib.dcn_predict_offset_mask(ctypes.byref(p), f, f, None, f, f, None, n, None) == EWS
+    assert lib.dcn_predict_offset_mask(ctypes.byref(p), f, f, None, f, f, f, n - 1, None) == EWS
+    assert str(n) in lib.dcn_last_error_string().decode()
+    odd = ctypes.c_void_p((1 << 20) + 2)
+    assert lib.dcn_predict_offset_mask(ctypes.byref(p), f, odd, None, f, f, f, n, None) == EUNSUP
+    assert lib.dcn_predict_offset_mask(ctypes.byref(p), f, f, None, f, f, ctypes.c_void_p((1 << 20) + 128), n,
+                                       None) == EUNSUP
+
+
 def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     import importlib
     monkeypatch.setattr(dcn, "_lib", None)
