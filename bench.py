@@ -519,7 +519,8 @@ def run_predictor(args):
     outs = [(torch.empty((s.B, 2 * s.G * s.K * s.K, s.Ho, s.Wo), dtype=dt, device=device),
              torch.empty((s.B, s.G * s.K * s.K, s.Ho, s.Wo), dtype=dt, device=device)) for _ in range(n_sets)]
     p = dcn.make_params(s.B, s.H, s.W, s.Cin, 1, s.K, s.stride, s.pad, s.dil, s.G, dcn._DTYPES[dt])
-    ws = torch.empty(dcn.predict_workspace_size(p), dtype=torch.uint8, device=device)
+    nws = dcn.predict_workspace_size(p)
+    ws = torch.empty(nws, dtype=torch.uint8, device=device) if nws > 0 else None
 
     def run(k):
         d = sets[k % n_sets]
@@ -573,9 +574,10 @@ def run_predictor(args):
             "dtype": w.dtype, "data": "synthetic",
             "config": {"workload": "offset/mask predictor of: " + w.description, "outputs": nc,
                        "l2": "inputs and outputs rotate over %d independent sets" % n_sets,
-                       "forward_path_inner": dcn.forward_path(dcn.make_params(
-                           s.B, s.H, s.W, s.Cin, (nc + 31) // 32 * 32, s.K, s.stride, s.pad, s.dil, 1,
-                           dcn._DTYPES[dt]))},
+                       "path": "tcgen05 implicit GEMM, sigmoid and split fused" if nws == 0 else
+                               "forward kernels with zero offsets (%s), then split" % dcn.forward_path(dcn.make_params(
+                                   s.B, s.H, s.W, s.Cin, (nc + 31) // 32 * 32, s.K, s.stride, s.pad, s.dil, 1,
+                                   dcn._DTYPES[dt]))},
             "roofline": rl, "gpu_launches": launches_per_step * args.steps, "clocks": clk}), flush=True)
     import torch.distributed as dist
     if dist.is_initialized():

@@ -229,11 +229,11 @@ def predict_offset_mask(x, w_pred, b_pred, K, stride=1, padding=0, dilation=1, G
         raise ValueError("out must be (offset %s, mask %s)" % ((B, 2 * G * K * K, Ho, Wo), (B, G * K * K, Ho, Wo)))
     _check_tensors(x.dtype, x.device, x=x, w_pred=w_pred, b_pred=b_pred, offset=offset, mask=mask)
     n = predict_workspace_size(p)
-    if workspace is None:
+    if workspace is None and n > 0:
         workspace = torch.empty(n, dtype=torch.uint8, device=x.device)
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.dcn_predict_offset_mask(ctypes.byref(p), _ptr(x), _ptr(w_pred), _ptr(b_pred), _ptr(offset),
-                                       _ptr(mask), _ptr(workspace), workspace.numel() * workspace.element_size(),
-                                       _stream(x.device)))
+                                       _ptr(mask), _ptr(workspace), nbytes, _stream(x.device)))
     return offset, mask
 
 

@@ -354,10 +354,12 @@ int dcn_backward_weight(const dcn_params_t* params, const void* x, const void* o
 // ------------------------------------------------- offset/mask predictor --
 
 // The predictor is the plain convolution with the layer's kernel size, stride,
-// padding and dilation and 3*G*K*K outputs (run as this library's layer with
-// zero offsets, no mask, one group and the outputs padded to a multiple of 32).
-// Workspace pieces, each 256-byte aligned: the zero offsets, the padded weights
-// and bias, the [P, NP] result, and the inner forward's own workspace.
+// padding and dilation and 3*G*K*K outputs. bfloat16 layers of stride 1 run it
+// as one tensor-core kernel (no workspace); the others run it as this library's
+// layer with zero offsets, no mask, one group and the outputs padded to a
+// multiple of 32, then split the result. Workspace pieces of that path, each
+// 256-byte aligned: the zero offsets, the padded weights and bias, the [P, NP]
+// result, and the inner forward's own workspace.
 struct PredPlan {
     dcn_params_t q;   // the inner plain convolution
     int nc, np, no;   // 3GK^2 outputs, rounded up to 32, of which 2GK^2 offsets
@@ -394,6 +396,10 @@ static int pred_plan(const dcn_params_t* p, PredPlan& pl, dcn::Shape& s) {
     return DCN_OK;
 }
 
+static bool use_pred_tc(const dcn_params_t* p, const dcn::Shape& s) {
+    return p->dtype == DCN_BF16 && !(p->flags & DCN_FLAG_GENERIC) && dcn::pred_tc_supported(s);
+}
+
 size_t dcn_predict_workspace_size(const dcn_params_t* params) {
     PredPlan pl;
     dcn::Shape s;
@@ -402,7 +408,7 @@ size_t dcn_predict_workspace_size(const dcn_params_t* params) {
         g_err = keep;
         return 0;
     }
-    return pl.total;
+    return use_pred_tc(params, s) ? 0 : pl.total;
 }
 
 int dcn_predict_offset_mask(const dcn_params_t* params, const void* x, const void* w_pred, const void* b_pred,
@@ -416,11 +422,23 @@ int dcn_predict_offset_mask(const dcn_params_t* params, const void* x, const voi
     TRY(check_ptr(b_pred, "b_pred", es, false));
     TRY(check_ptr(offset, "offset", es, true));
     TRY(check_ptr(mask, "mask", es, true));
+    cudaStream_t st = (cudaStream_t)stream;
+    if (use_pred_tc(params, s)) {
+        // the tensor maps of x and w_pred need 16-byte aligned bases
+        if (!aligned16(x) || !aligned16(w_pred))
+            return fail(DCN_ERR_UNSUPPORTED, "x and w_pred must be 16-byte aligned for this layer");
+        unsigned* status = nullptr;
+        cudaError_t e = dcn::status_word_ptr(&status);
+        if (e != cudaSuccess) return cuda_fail(e, "status word");
+        e = dcn::pred_tc(s, x, w_pred, b_pred, offset, mask, status, st);
+        g_launches += 1;
+        if (e != cudaSuccess) return cuda_fail(e, "tensor-core predictor launch");
+        return ok();
+    }
     if (!workspace || workspace_bytes < pl.total)
         return fail(DCN_ERR_WORKSPACE, "the predictor needs %zu bytes of workspace, got %zu", pl.total,
                     workspace ? workspace_bytes : (size_t)0);
     TRY(check_ptr(workspace, "workspace", 256, true));
-    cudaStream_t st = (cudaStream_t)stream;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     const int bf = params->dtype == DCN_BF16;
     cudaError_t e = cudaMemsetAsync(ws + pl.zoff, 0, es * (size_t)s.P * 2 * s.K2, st);

@@ -29,6 +29,11 @@ size_t fwd_tc_static_scratch_bytes();
 cudaError_t fwd_tc_noalloc(const Shape& s, const void* x, const void* off, const void* mask, const void* w,
                            const void* bias, void* y, unsigned* status, cudaStream_t st, int* launches);
 
+// pred_tc.cu — the bfloat16 stride-1 offset/mask predictor on tcgen05, sigmoid and split fused (no workspace).
+bool pred_tc_supported(const Shape& s);
+cudaError_t pred_tc(const Shape& s, const void* x, const void* w, const void* bias, void* off, void* mask,
+                    unsigned* status, cudaStream_t st);
+
 // predict.cu — the offset/mask predictor's weight padding and output split.
 cudaError_t predict_pad(int dtype_bf16, const void* w, const void* b, void* wpad, void* bpad, int nc, int np, int kc,
                         cudaStream_t st);

@@ -110,6 +110,20 @@ def test_predictor_arguments(lib):
                                        None) == EUNSUP
 
 
+def test_predictor_tensor_core_path_needs_no_workspace(lib):
+    f = ctypes.c_void_p(1 << 20)
+    p16 = P(dtype=1, Cin=64, G=1)
+    assert lib.dcn_predict_workspace_size(ctypes.byref(p16)) == 0
+    # stride 2 and float32 layers take the forward-kernel path, which does
+    assert lib.dcn_predict_workspace_size(ctypes.byref(P(dtype=1, Cin=64, G=1, stride=2))) > 0
+    assert lib.dcn_predict_workspace_size(ctypes.byref(P(dtype=0, Cin=64, G=1))) > 0
+    # its tensor maps need 16-byte aligned x and w_pred
+    odd = ctypes.c_void_p((1 << 20) + 2)
+    assert lib.dcn_predict_offset_mask(ctypes.byref(p16), odd, f, None, f, f, None, 0, None) == EUNSUP
+    assert "16-byte" in lib.dcn_last_error_string().decode()
+    assert lib.dcn_predict_offset_mask(ctypes.byref(p16), f, odd, None, f, f, None, 0, None) == EUNSUP
+
+
 def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     import importlib
     monkeypatch.setattr(dcn, "_lib", None)

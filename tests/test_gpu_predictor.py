@@ -28,6 +28,12 @@ SHAPES = [
     (S(B=1, Cin=48, H=9, W=21, Cout=1, K=5, pad=2, G=2), "bf16"),
     (S(B=2, Cin=16, H=8, W=8, Cout=1, K=1, pad=0), "bf16"),
     (S(B=1, Cin=128, H=17, W=9, Cout=1, stride=2), "bf16"),
+    # bfloat16 stride 1: the implicit-GEMM kernel (ragged slabs and tiles, no padding, dilation, wide rows)
+    (S(B=3, Cin=136, H=20, W=30, Cout=1), "bf16"),
+    (S(B=1, Cin=8, H=40, W=100, Cout=1), "bf16"),
+    (S(B=2, Cin=64, H=9, W=9, Cout=1, pad=0), "bf16"),
+    (S(B=1, Cin=32, H=11, W=13, Cout=1, pad=1, dil=2), "bf16"),
+    (S(B=2, Cin=24, H=6, W=7, Cout=1, K=1, pad=0, G=2), "bf16"),
 ]
 
 
