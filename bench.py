@@ -144,11 +144,11 @@ def barrier(device=None):
 
 # -------------------------------------------------------------- work model --
 
-def work_model(s, elem=2):
-    """Algorithmic FLOPs and minimal HBM bytes per launch of each pass."""
+def work_model(s, elem=2, mask=True):
+    """Algorithmic FLOPs and minimal HBM bytes per launch of each pass (mask=False: DCNv1, no mask tensor)."""
     nx = s.B * s.H * s.W * s.Cin
     noff = s.P * 2 * s.G * s.K * s.K
-    nm = s.P * s.G * s.K * s.K
+    nm = s.P * s.G * s.K * s.K if mask else 0
     nw = s.Cout * s.K * s.K * s.Cin
     ny = s.P * s.Cout
     f = s.flops()
@@ -193,7 +193,7 @@ def run_ours(args):
     s = w.shape
     do_bwd = not args.forward_only
     elem = 2 if w.dtype == "bf16" else 4
-    wm = work_model(s, elem)
+    wm = work_model(s, elem, mask=w.mask_dist != "none")
     pk, pk_src = peaks()
 
     # rotating input sets so that every step reads its inputs from HBM
@@ -590,7 +590,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="conv4", help="conv4 | conv3_s2 | conv5_d2g4 | stem | tiny | conv4_bwd")
+    ap.add_argument("--workload", default="conv4",
+                    help="conv4 | conv3_s2 | conv5_d2g4 | conv4_v1 | conv4_k5 | stem | tiny | conv4_bwd")
     ap.add_argument("--forward-only", action="store_true", help="time the forward alone (not the default step)")
     ap.add_argument("--predictor", action="store_true",
                     help="time the layer's offset/mask predictor instead of the default step")

@@ -89,6 +89,12 @@ WORKLOADS = {
     "conv5_d2g4": Workload(
         "conv5_d2g4", LayerShape(B=8, Cin=512, H=25, W=25, Cout=512, pad=2, dil=2, G=4), "bf16", seed=4,
         description="ResNet-50 conv5 DCNv2 forward bf16, B8 Cin=Cout=512 25x25 s1 p2 d2 G4"),
+    "conv4_v1": Workload(
+        "conv4_v1", LayerShape(B=8, Cin=256, H=50, W=50, Cout=256), "bf16", seed=6, mask_dist="none",
+        description="ResNet-50 conv4 3x3 DCNv1 forward bf16 (no modulation mask), B8 Cin=Cout=256 50x50 K3 s1 p1 G1"),
+    "conv4_k5": Workload(
+        "conv4_k5", LayerShape(B=8, Cin=256, H=50, W=50, Cout=256, K=5, pad=2), "bf16", seed=7,
+        description="conv4-sized 5x5 DCNv2 forward bf16 (50 offset channels), B8 Cin=Cout=256 50x50 K5 s1 p2 G1"),
     "conv4_bwd": Workload(
         "conv4_bwd", LayerShape(B=8, Cin=256, H=50, W=50, Cout=256), "bf16", seed=5,
         offset_dist="normal1.5_edges", backward=True,

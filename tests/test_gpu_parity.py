@@ -153,7 +153,7 @@ def test_repeated_calls_identical():
 
 # ---------------------------------------------------------- full-size shapes --
 
-@pytest.mark.parametrize("name", ["stem", "conv4", "conv3_s2", "conv5_d2g4"])
+@pytest.mark.parametrize("name", ["stem", "conv4", "conv3_s2", "conv5_d2g4", "conv4_v1", "conv4_k5"])
 def test_full_size_forward_sampled(name):
     w = gen.WORKLOADS[name]
     s = w.shape
@@ -208,6 +208,55 @@ def test_full_size_backward_sampled():
     for gname, prim in (("grad_x", "x"), ("grad_weight", "weight"), ("grad_mask", "mask")):
         rhs = float((g[gname].double() * dd[prim].double()).sum())
         assert abs(lhs - rhs) <= 2e-2 * abs(lhs), (gname, lhs, rhs)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("shape,mask", [
+    (gen.LayerShape(B=1, Cin=16, H=11, W=9, Cout=24, K=7, pad=3), True),
+    (gen.LayerShape(B=2, Cin=32, H=9, W=14, Cout=16, K=7, pad=3, dil=1, G=2), False),
+    (gen.LayerShape(B=1, Cin=8, H=16, W=10, Cout=8, K=7, stride=2, pad=6, dil=2), True),
+], ids=["k7", "k7_g2_v1", "k7_s2_d2"])
+def test_seven_by_seven_layers(shape, mask, dtype):
+    """K = 7 (49 taps, 98 offset channels per group), DCNv2 and DCNv1, forward and backward in full."""
+    w = gen.Workload("k7", shape, dtype, seed=17, offset_dist="uniform2.5",
+                     mask_dist="uniform" if mask else "none", bias=True, backward=True)
+    d = gen.make_inputs(w)
+    a = f64(d)
+    dd = to_dev(d)
+    assert_close(_cpu(run_forward(shape, dd)), _oracle_forward(shape, a), dtype, "y")
+    g = run_backward(shape, dd)
+    ref = _oracle_backward(shape, a)
+    for k in ("grad_x", "grad_offset", "grad_mask", "grad_weight", "grad_bias"):
+        if ref[k] is None:
+            assert g[k] is None
+            continue
+        assert_close(_cpu(g[k]), ref[k], dtype, k)
+
+
+def test_full_size_v1_backward_sampled():
+    """DCNv1 (no mask) backward on the conv4 layer at sampled entries."""
+    w = gen.WORKLOADS["conv4_v1"]
+    s = w.shape
+    d = gen.make_inputs(w)
+    g0 = torch.Generator().manual_seed(21)
+    d["grad_y"] = torch.randn((s.B, s.Ho, s.Wo, s.Cout), generator=g0).to(torch.bfloat16)
+    a = f64(d)
+    g = run_backward(s, to_dev(d))
+    assert g["grad_mask"] is None
+    pix = sample_pixels(s, 32, seed=22)
+    goff, _ = oracle.grad_offset_mask_at(a["x"], a["offset"], None, a["weight"], a["grad_y"], pix, s.stride, s.pad,
+                                         s.dil, s.G)
+    got_off = _cpu(g["grad_offset"]).transpose(0, 2, 3, 1).reshape(s.P, -1)[pix]
+    assert_close(got_off, goff, "bf16", "grad_offset")
+    r = np.random.default_rng(23)
+    went = r.choice(s.Cout * s.K * s.K * s.Cin, 48, replace=False)
+    gw_ref = oracle.grad_weight_at(a["x"], a["offset"], None, a["grad_y"], a["weight"].shape, went, s.stride, s.pad,
+                                   s.dil, s.G)
+    assert_close(_cpu(g["grad_weight"]).reshape(-1)[went], gw_ref, "bf16", "grad_weight")
+    xent = r.choice(s.B * s.H * s.W * s.Cin, 48, replace=False)
+    gx_ref = oracle.grad_x_at(a["x"].shape, a["offset"], None, a["weight"], a["grad_y"], xent, s.stride, s.pad,
+                              s.dil, s.G)
+    assert_close(_cpu(g["grad_x"]).reshape(-1)[xent], gx_ref, "bf16", "grad_x")
 
 
 def _tf32_split_applies(s):
