@@ -221,8 +221,12 @@ def run_ours(args):
             o["grad_x"] = torch.empty((s.B, s.H, s.W, s.Cin), **f32)
             o["grad_offset"] = torch.empty(tuple(host["offset"].shape), **f32)
             o["grad_mask"] = torch.empty(tuple(host["mask"].shape), **f32) if host["mask"] is not None else None
-            o["grad_weight"] = torch.empty(tuple(host["weight"].shape), **f32)
-            o["grad_bias"] = torch.empty((s.Cout,), **f32)
+            # grad_weight and grad_bias are views of one buffer: the data-parallel step sums it over ranks
+            # with a single all-reduce
+            nw = host["weight"].numel()
+            o["grad_wb"] = torch.empty((nw + s.Cout,), **f32)
+            o["grad_weight"] = o["grad_wb"][:nw].view(tuple(host["weight"].shape))
+            o["grad_bias"] = o["grad_wb"][nw:]
         outs.append(o)
     p = dcn._params(sets[0]["x"], sets[0]["weight"], sets[0]["offset"], s.stride, s.pad, s.dil, False)
     ws = {op: (torch.empty(max(1, dcn.workspace_size(p, op)), dtype=torch.uint8, device=device))
@@ -267,12 +271,20 @@ def run_ours(args):
     torch.cuda.synchronize()
     npass = len(graphs[0])
 
+    dp = args.dp and do_bwd and world > 1
+    import torch.distributed as dist
+
     def step(k, ev=None):
         row = graphs[k % n_sets]
         for i, g in enumerate(row):
             g.replay()
             if ev is not None:
                 ev[i + 1].record(stream)
+        if dp:
+            # data parallel: the weight gradients summed over ranks (NCCL, ordered on this stream)
+            dist.all_reduce(outs[k % n_sets]["grad_wb"], op=dist.ReduceOp.SUM)
+            if ev is not None:
+                ev[npass + 1].record(stream)
 
     with torch.cuda.stream(stream):
         for k in range(args.warmup):
@@ -280,7 +292,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     dcn.check_status()
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(npass + 1)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(npass + 2)] for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
     clocks.start()
@@ -305,6 +317,7 @@ def run_ours(args):
     fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
     bd_ms = [e[1].elapsed_time(e[2]) for e in evs] if do_bwd else []
     bw_ms = [e[2].elapsed_time(e[3]) for e in evs] if do_bwd else []
+    ar_ms = [e[npass].elapsed_time(e[npass + 1]) for e in evs] if dp else []
 
     total_ms_max = max_over_ranks(total_ms, device)
     fwd_sum_max = max_over_ranks(sum(fwd_ms), device)
@@ -336,7 +349,10 @@ def run_ours(args):
                        "step": "forward + backward_data + backward_weight" if do_bwd else "forward",
                        "l2": "inputs and outputs rotate over %d independent sets (%.0f MB each) so each step "
                              "reads from HBM" % (n_sets, (set_bytes + out_bytes) / 1e6),
-                       "parallelism": "1 GPU" if world == 1 else "%d independent replicas" % world,
+                       "parallelism": "1 GPU" if world == 1 else (
+                           "data parallel over %d ranks: a batch of %d per rank, grad_weight and grad_bias summed "
+                           "by one NCCL all-reduce per step" % (world, s.B) if dp else
+                           "%d independent replicas" % world),
                        "timing": "each pass of each input set captured once in a CUDA graph and replayed; CUDA "
                                  "events on the replay stream, which a device-side sleep holds while the host "
                                  "enqueues the timed steps",
@@ -348,6 +364,9 @@ def run_ours(args):
                         "roofline_frac": rl["forward"]["roofline_frac"]},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
         }
+        if dp:
+            line["allreduce"] = {"us": round(statistics.mean(ar_ms) * 1e3, 2),
+                                 "bytes": int(outs[0]["grad_wb"].numel() * 4)}
         print(json.dumps(line), flush=True)
     import torch.distributed as dist
     if dist.is_initialized():
@@ -595,6 +614,9 @@ def main(argv=None):
     ap.add_argument("--forward-only", action="store_true", help="time the forward alone (not the default step)")
     ap.add_argument("--predictor", action="store_true",
                     help="time the layer's offset/mask predictor instead of the default step")
+    ap.add_argument("--dp", action="store_true",
+                    help="with several GPUs: data-parallel step (grad_weight and grad_bias all-reduced every step) "
+                         "instead of independent replicas")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args(argv)
