@@ -180,13 +180,18 @@ DCN_API int dcn_forward_noalloc(const dcn_params_t* params, const void* x, const
  *   offset  [B, 2*G*K*K, Ho, Wo]          written; the layout dcn_forward reads
  *   mask    [B, G*K*K, Ho, Wo]            written
  * All in params->dtype, device memory owned by the caller, element-aligned.
- * workspace: device memory of at least dcn_predict_workspace_size(params)
- * bytes, 256-byte aligned, used as scratch for the duration of the stream
- * work. The convolution runs on this library's forward kernels with zero
- * offsets and no mask, one group and the outputs padded to a multiple of 32,
- * so its precision is the forward's for that layer shape.
+ * bfloat16 layers of stride 1 with Cin a multiple of 8, 3*G*K*K <= 256 and
+ * W + 2*pad <= 256 run one tensor-core kernel (float32 accumulation, the
+ * sigmoid in float32, outputs rounded to bfloat16 once): it needs no workspace
+ * (dcn_predict_workspace_size returns 0) and 16-byte aligned x and w_pred
+ * (DCN_ERR_UNSUPPORTED otherwise). Other layers run the convolution on this
+ * library's forward kernels with zero offsets and no mask, one group and the
+ * outputs padded to a multiple of 32, then split it; their precision is the
+ * forward's for that shape, and they need workspace: device memory of at
+ * least dcn_predict_workspace_size(params) bytes, 256-byte aligned, used as
+ * scratch for the duration of the stream work.
  * Errors as for dcn_forward: argument problems return before anything is
- * enqueued; DCN_ERR_WORKSPACE when workspace is NULL or too small. */
+ * enqueued; DCN_ERR_WORKSPACE when a needed workspace is NULL or too small. */
 DCN_API size_t dcn_predict_workspace_size(const dcn_params_t* params);
 DCN_API int dcn_predict_offset_mask(const dcn_params_t* params, const void* x, const void* w_pred,
                                     const void* b_pred, void* offset, void* mask, void* workspace,
