@@ -181,10 +181,12 @@ DCN_API int dcn_forward_noalloc(const dcn_params_t* params, const void* x, const
  *   mask    [B, G*K*K, Ho, Wo]            written
  * All in params->dtype, device memory owned by the caller, element-aligned.
  * bfloat16 layers of stride 1 with Cin a multiple of 8, 3*G*K*K <= 256 and
- * W + 2*pad <= 256 run one tensor-core kernel (float32 accumulation, the
- * sigmoid in float32, outputs rounded to bfloat16 once): it needs no workspace
- * (dcn_predict_workspace_size returns 0) and 16-byte aligned x and w_pred
- * (DCN_ERR_UNSUPPORTED otherwise). Other layers run the convolution on this
+ * padded rows (W + 2*pad) short enough for the kernel's shared memory (up to
+ * 212 pixels at K = 3) run one tensor-core kernel (float32
+ * accumulation, the sigmoid in float32, outputs rounded to bfloat16 once): it
+ * needs no workspace (dcn_predict_workspace_size returns 0 exactly when this
+ * kernel applies) and 16-byte aligned x and w_pred (DCN_ERR_UNSUPPORTED
+ * otherwise). Other layers run the convolution on this
  * library's forward kernels with zero offsets and no mask, one group and the
  * outputs padded to a multiple of 32, then split it; their precision is the
  * forward's for that shape, and they need workspace: device memory of at
