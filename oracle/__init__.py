@@ -81,6 +81,9 @@ def _bind(lib):
     lib.dcn_oracle_grad_weight_entries.argtypes = [sp, dp, dp, dp, dp, L, lp, dp]
     lib.dcn_oracle_grad_x_entries.argtypes = [sp, dp, dp, dp, dp, L, lp, dp]
     lib.dcn_oracle_predict_offset_mask.argtypes = [sp, dp, dp, dp, dp, dp]
+    I, D = ctypes.c_int, ctypes.c_double
+    lib.dcn_oracle_droi_pool_forward.argtypes = [sp, I, I, D, dp, dp, dp, dp, dp]
+    lib.dcn_oracle_droi_pool_backward.argtypes = [sp, I, I, D, dp, dp, dp, dp, dp, dp, dp, dp]
     return lib
 
 
@@ -262,3 +265,46 @@ def predict_offset_mask(x, w_pred, b_pred, K, stride=1, pad=0, dil=1, G=1, lib=N
     if rc != 0:
         raise ValueError("oracle predictor rejected the shape (rc=%d)" % rc)
     return off, mask
+
+
+def droi_pool_forward(x, rois, offset, mask, k, gamma=1.0, lib=None):
+    """(Modulated) deformable RoI pooling: y [R, k, k, C] from x [B, H, W, C],
+    rois [R, 5] = (b, x1, y1, x2, y2), offset [R, 2k^2] (normalised, or None)
+    and mask [R, k^2] (or None)."""
+    lib = lib or load()
+    B, H, W, C = x.shape
+    R = int(np.asarray(rois).shape[0])
+    s = _shape(B, H, W, C, 1, 1)
+    xs, xp = _d(x)
+    rs, rp = _d(rois)
+    os_, op = _d(offset)
+    ms, mp = _d(mask)
+    y = np.zeros((R, k, k, C))
+    rc = lib.dcn_oracle_droi_pool_forward(ctypes.byref(s), R, int(k), float(gamma), xp, rp, op, mp,
+                                          y.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
+    if rc != 0:
+        raise ValueError("oracle RoI pooling: a batch index is out of range")
+    return y
+
+
+def droi_pool_backward(x, rois, offset, mask, grad_y, k, gamma=1.0, lib=None):
+    """(grad_x [B, H, W, C], grad_offset [R, 2k^2] or None, grad_mask [R, k^2] or None)."""
+    lib = lib or load()
+    B, H, W, C = x.shape
+    R = int(np.asarray(rois).shape[0])
+    s = _shape(B, H, W, C, 1, 1)
+    xs, xp = _d(x)
+    rs, rp = _d(rois)
+    os_, op = _d(offset)
+    ms, mp = _d(mask)
+    gs, gp = _d(grad_y)
+    gx = np.zeros((B, H, W, C))
+    goff = np.zeros((R, 2 * k * k)) if offset is not None else None
+    gm = np.zeros((R, k * k)) if mask is not None else None
+    P = ctypes.POINTER(ctypes.c_double)
+    rc = lib.dcn_oracle_droi_pool_backward(ctypes.byref(s), R, int(k), float(gamma), xp, rp, op, mp, gp,
+                                           gx.ctypes.data_as(P), None if goff is None else goff.ctypes.data_as(P),
+                                           None if gm is None else gm.ctypes.data_as(P))
+    if rc != 0:
+        raise ValueError("oracle RoI pooling: a batch index is out of range")
+    return gx, goff, gm

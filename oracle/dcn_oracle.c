@@ -407,3 +407,126 @@ int dcn_oracle_predict_offset_mask(const dcn_oracle_shape* s, const double* x, c
     }
     return 0;
 }
+
+/* --------------------------------------------------- deformable RoI pooling -- */
+
+/* Deformable RoI pooling (notes, "可变形ROI pooling": RoI pooling cuts a RoI of
+ * w x h into k x k bins and averages the pixels of each bin; the deformable form
+ * first moves every bin as a whole by an offset given as a fraction of the RoI's
+ * width and height, the moved positions being read by bilinear interpolation;
+ * the explainer's "可变形RoI池化" paragraph: the offsets are normalised to the
+ * RoI size; DCNv2 section 3.2: a modulation scalar per bin). The pages print no
+ * formula for it; this follows the plainest reading of that text:
+ *
+ *   roi r = (b, x1, y1, x2, y2) in feature-map pixel coordinates,
+ *   h = y2 - y1, w = x2 - x1 (a negative size counts as 0);
+ *   bin (i, j), t = i*k + j, holds the integer offsets (u, v) with
+ *     floor(i*h/k) <= u < ceil((i+1)*h/k),   floor(j*w/k) <= v < ceil((j+1)*w/k),
+ *   n of them;
+ *   its shift is (dy, dx) = gamma * (off[r][2t] * h, off[r][2t+1] * w);
+ *   y[r][i][j][c] = m / n * sum over (u, v) of x_b(y1 + u + dy, x1 + v + dx, c),
+ *   with m = mask[r][t] (1 without a mask), bilinear sampling whose neighbours
+ *   outside the map contribute zero (as in the layer), and 0 for an empty bin.
+ *
+ * Layouts: x [B, H, W, C] (s->Cin = C; s->Cout, K, stride, pad, dil, G unused),
+ * rois [R, 5], off [R, 2*k*k] or NULL (plain RoI pooling), mask [R, k*k] or
+ * NULL, y and grad_y [R, k, k, C]. Returns -1 for a batch index out of range. */
+static void roi_bin(const double* roi, int k, int i, int j, int* u0, int* u1, int* v0, int* v1, double* h,
+                    double* w) {
+    double hh = roi[4] - roi[2], ww = roi[3] - roi[1];
+    if (hh < 0.0) hh = 0.0;
+    if (ww < 0.0) ww = 0.0;
+    *h = hh;
+    *w = ww;
+    *u0 = (int)floor(i * hh / k);
+    *u1 = (int)ceil((i + 1) * hh / k);
+    *v0 = (int)floor(j * ww / k);
+    *v1 = (int)ceil((j + 1) * ww / k);
+}
+
+int dcn_oracle_droi_pool_forward(const dcn_oracle_shape* s, int R, int k, double gamma, const double* x,
+                                 const double* rois, const double* off, const double* mask, double* y) {
+    const int C = s->Cin, kk = k * k;
+    for (int r = 0; r < R; ++r) {
+        const double* roi = rois + (size_t)r * 5;
+        const int b = (int)roi[0];
+        if (b < 0 || b >= s->B) return -1;
+        for (int i = 0; i < k; ++i)
+            for (int j = 0; j < k; ++j) {
+                int u0, u1, v0, v1;
+                double h, w;
+                roi_bin(roi, k, i, j, &u0, &u1, &v0, &v1, &h, &w);
+                const int t = i * k + j;
+                const double dy = off ? gamma * off[(size_t)r * 2 * kk + 2 * t] * h : 0.0;
+                const double dx = off ? gamma * off[(size_t)r * 2 * kk + 2 * t + 1] * w : 0.0;
+                const double m = mask ? mask[(size_t)r * kk + t] : 1.0;
+                const int n = (u1 - u0) * (v1 - v0);
+                double* yb = y + (((size_t)r * k + i) * k + j) * C;
+                for (int c = 0; c < C; ++c) {
+                    double acc = 0.0;
+                    for (int u = u0; u < u1; ++u)
+                        for (int v = v0; v < v1; ++v) acc += bilinear(x, s, b, c, roi[2] + u + dy, roi[1] + v + dx);
+                    yb[c] = n > 0 ? m * acc / n : 0.0;
+                }
+            }
+    }
+    return 0;
+}
+
+/* Backward of the above: grad_x [B, H, W, C] (overwritten), grad_off [R, 2*k*k]
+ * (the derivative with respect to the normalised offsets: gamma*h and gamma*w
+ * times d/dy and d/dx of the bilinear samples, through floor() as in the layer),
+ * grad_mask [R, k*k]; either of the last two may be NULL. */
+int dcn_oracle_droi_pool_backward(const dcn_oracle_shape* s, int R, int k, double gamma, const double* x,
+                                  const double* rois, const double* off, const double* mask, const double* gy,
+                                  double* gx, double* goff, double* gmask) {
+    const int C = s->Cin, kk = k * k;
+    memset(gx, 0, sizeof(double) * (size_t)s->B * s->H * s->W * C);
+    if (goff) memset(goff, 0, sizeof(double) * (size_t)R * 2 * kk);
+    if (gmask) memset(gmask, 0, sizeof(double) * (size_t)R * kk);
+    for (int r = 0; r < R; ++r) {
+        const double* roi = rois + (size_t)r * 5;
+        const int b = (int)roi[0];
+        if (b < 0 || b >= s->B) return -1;
+        for (int i = 0; i < k; ++i)
+            for (int j = 0; j < k; ++j) {
+                int u0, u1, v0, v1;
+                double h, w;
+                roi_bin(roi, k, i, j, &u0, &u1, &v0, &v1, &h, &w);
+                const int t = i * k + j;
+                const int n = (u1 - u0) * (v1 - v0);
+                if (n == 0) continue;
+                const double dy = off ? gamma * off[(size_t)r * 2 * kk + 2 * t] * h : 0.0;
+                const double dx = off ? gamma * off[(size_t)r * 2 * kk + 2 * t + 1] * w : 0.0;
+                const double m = mask ? mask[(size_t)r * kk + t] : 1.0;
+                const double* gyb = gy + (((size_t)r * k + i) * k + j) * C;
+                double g_dy = 0.0, g_dx = 0.0, g_m = 0.0;
+                for (int c = 0; c < C; ++c) {
+                    const double g = gyb[c] / n;
+                    for (int u = u0; u < u1; ++u)
+                        for (int v = v0; v < v1; ++v) {
+                            const double py = roi[2] + u + dy, px = roi[1] + v + dx;
+                            const double y0 = floor(py), x0 = floor(px);
+                            for (int a = 0; a < 2; ++a)
+                                for (int e = 0; e < 2; ++e) {
+                                    const int rr = (int)y0 + a, qq = (int)x0 + e;
+                                    if (rr < 0 || rr >= s->H || qq < 0 || qq >= s->W) continue;
+                                    const double wt = (1.0 - fabs(py - rr)) * (1.0 - fabs(px - qq));
+                                    gx[(((size_t)b * s->H + rr) * s->W + qq) * C + c] += g * m * wt;
+                                }
+                            double dpy, dpx;
+                            bilinear_grad(x, s, b, c, py, px, &dpy, &dpx);
+                            g_dy += g * m * dpy;
+                            g_dx += g * m * dpx;
+                            g_m += g * bilinear(x, s, b, c, py, px);
+                        }
+                }
+                if (goff && off) {
+                    goff[(size_t)r * 2 * kk + 2 * t] = g_dy * gamma * h;
+                    goff[(size_t)r * 2 * kk + 2 * t + 1] = g_dx * gamma * w;
+                }
+                if (gmask && mask) gmask[(size_t)r * kk + t] = g_m;
+            }
+    }
+    return 0;
+}

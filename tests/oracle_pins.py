@@ -22,7 +22,11 @@ AssertionError when the oracle disagrees with the fact it checks:
 * the backward is the adjoint of the forward (the forward is linear in x, in
   the weight, in the mask and in the bias), and the offset gradient matches
   finite differences of the forward (notes "计算梯度"), one-sided at exact
-  integer coordinates.
+  integer coordinates;
+* deformable RoI pooling: without offsets it is avg_pool2d of the RoI's k x k
+  blocks, whole-pixel shifts move the blocks, half-pixel corners average four
+  neighbours, the mask scales each bin, and its backward is the adjoint in x
+  and the mask and matches finite differences in the offsets.
 """
 from __future__ import annotations
 
@@ -352,6 +356,115 @@ def pin_predictor_bias_only(lib):
     assert np.array_equal(off, np.broadcast_to(b[:2 * G * K * K, None, None], off.shape[1:])[None].repeat(1, 0))
     off0, mask0 = oracle.predict_offset_mask(x, w, None, K, 1, 1, 1, G, lib=lib)
     assert np.all(off0 == 0.0) and np.all(mask0 == 0.5)
+
+
+# --------------------------------------------------- deformable RoI pooling --
+
+def _avg_pool_blocks(x, b, y1, x1, h, w, k, pad=0):
+    """torch avg_pool2d (float64) of the h x w block at (y1, x1) of image b, cut
+    into k x k equal blocks; the image is zero-padded by `pad` first, so blocks
+    reaching outside the map average zeros there. Returns [k, k, C]."""
+    img = torch.from_numpy(x[b]).permute(2, 0, 1)[None]  # [1, C, H, W]
+    img = torch.nn.functional.pad(img, (pad, pad, pad, pad))
+    crop = img[:, :, y1 + pad:y1 + pad + h, x1 + pad:x1 + pad + w]
+    out = torch.nn.functional.avg_pool2d(crop, kernel_size=(h // k, w // k))
+    return out[0].permute(1, 2, 0).numpy()
+
+
+def pin_droi_plain_is_avg_pool(lib):
+    """Without offsets, a RoI with integer corners whose sides are multiples of k
+    pools to torch's avg_pool2d of its k x k blocks, zeros outside the map
+    (notes, "可变形ROI pooling": each output averages its bin's pixels)."""
+    r = _rng(300)
+    x = r.standard_normal((2, 9, 11, 3))
+    k = 3
+    rois = np.array([[0, 2, 0, 8, 9], [1, 0, 3, 9, 9], [1, -2, -1, 7, 5], [0, 6, 4, 12, 10]], dtype=float)
+    y = oracle.droi_pool_forward(x, rois, None, None, k, lib=lib)
+    for n, (b, x1, y1, x2, y2) in enumerate(rois.astype(int)):
+        ref = _avg_pool_blocks(x, b, y1, x1, y2 - y1, x2 - x1, k, pad=4)
+        assert np.allclose(y[n], ref, rtol=1e-12, atol=1e-12), n
+
+
+def pin_droi_integer_shifts_move_blocks(lib):
+    """Offsets whose shift gamma*off*h (and *w) is a whole number of pixels move
+    each bin's block by that many pixels: the mean of the moved block, zeros
+    outside the map; normalised offsets scale with the RoI's size and gamma."""
+    r = _rng(301)
+    x = r.standard_normal((1, 10, 12, 2))
+    k, gamma = 2, 0.5
+    rois = np.array([[0, 2, 1, 10, 9]], dtype=float)  # w = 8, h = 8: blocks of 4 x 4
+    h = w = 8
+    sh = r.integers(-3, 4, size=(k * k, 2))
+    off = np.zeros((1, 2 * k * k))
+    off[0, 0::2] = sh[:, 0] / (gamma * h)
+    off[0, 1::2] = sh[:, 1] / (gamma * w)
+    y = oracle.droi_pool_forward(x, rois, off, None, k, gamma, lib=lib)
+    xp = np.pad(x[0], ((6, 6), (6, 6), (0, 0)))
+    for i in range(k):
+        for j in range(k):
+            t = i * k + j
+            r0, c0 = 1 + i * 4 + sh[t, 0] + 6, 2 + j * 4 + sh[t, 1] + 6
+            ref = xp[r0:r0 + 4, c0:c0 + 4].mean(axis=(0, 1))
+            assert np.allclose(y[0, i, j], ref, rtol=1e-12, atol=1e-12), (i, j)
+
+
+def pin_droi_half_pixel_corners_average_neighbours(lib):
+    """A RoI whose corners sit on half-integers samples midway between four
+    pixels: the pooled values equal avg_pool2d of the 2 x 2 box-filtered map."""
+    r = _rng(302)
+    x = r.standard_normal((1, 8, 8, 2))
+    k = 2
+    rois = np.array([[0, 1.5, 0.5, 5.5, 6.5]], dtype=float)  # w = 4, h = 6
+    y = oracle.droi_pool_forward(x, rois, None, None, k, lib=lib)
+    img = torch.from_numpy(x[0]).permute(2, 0, 1)[:, None]  # [C, 1, H, W]
+    box = torch.nn.functional.conv2d(img, torch.full((1, 1, 2, 2), 0.25, dtype=torch.float64))  # [C,1,H-1,W-1]
+    # sample (0.5 + u, 1.5 + v) is the box filter at (u, v + 1)
+    crop = box[:, :, 0:6, 1:5]
+    ref = torch.nn.functional.avg_pool2d(crop, kernel_size=(3, 2))[:, 0].permute(1, 2, 0).numpy()
+    assert np.allclose(y[0], ref, rtol=1e-12, atol=1e-12)
+
+
+def pin_droi_mask_scales_and_gamma_zero_is_plain(lib):
+    """The per-bin mask multiplies the bin's output (DCNv2 section 3.2); gamma = 0
+    removes every offset."""
+    r = _rng(303)
+    x = r.standard_normal((2, 7, 9, 3))
+    k = 3
+    rois = np.array([[0, 0.3, 1.2, 7.9, 6.1], [1, 2, 2, 5, 5]], dtype=float)
+    off = r.uniform(-0.4, 0.4, (2, 2 * k * k))
+    mask = r.uniform(0, 1, (2, k * k))
+    y1 = oracle.droi_pool_forward(x, rois, off, None, k, 0.3, lib=lib)
+    ym = oracle.droi_pool_forward(x, rois, off, mask, k, 0.3, lib=lib)
+    assert np.allclose(ym, y1 * mask.reshape(2, k, k, 1), rtol=1e-12, atol=1e-12)
+    assert np.array_equal(oracle.droi_pool_forward(x, rois, off, None, k, 0.0, lib=lib),
+                          oracle.droi_pool_forward(x, rois, None, None, k, lib=lib))
+
+
+def pin_droi_backward_adjoint_and_finite_differences(lib):
+    """The backward is the adjoint of the forward in x and in the mask (the
+    forward is linear in both), and its offset gradient matches central finite
+    differences of the forward."""
+    r = _rng(304)
+    x = r.standard_normal((2, 8, 9, 3))
+    k, gamma = 3, 0.2
+    rois = np.array([[0, 0.7, 1.3, 7.6, 6.9], [1, 1.2, 0.4, 8.8, 7.7], [1, 3.1, 2.2, 5.3, 4.9]], dtype=float)
+    off = r.uniform(-0.5, 0.5, (3, 2 * k * k))
+    mask = r.uniform(0, 1, (3, k * k))
+    gy = r.standard_normal((3, k, k, 3))
+    y = oracle.droi_pool_forward(x, rois, off, mask, k, gamma, lib=lib)
+    gx, goff, gm = oracle.droi_pool_backward(x, rois, off, mask, gy, k, gamma, lib=lib)
+    lhs = float((gy * y).sum())
+    assert abs(lhs - float((gx * x).sum())) <= 1e-10 * (1 + abs(lhs))
+    assert abs(lhs - float((gm * mask).sum())) <= 1e-10 * (1 + abs(lhs))
+    eps = 1e-6
+    for n in range(3):
+        for q in r.choice(2 * k * k, 6, replace=False):
+            op, om = off.copy(), off.copy()
+            op[n, q] += eps
+            om[n, q] -= eps
+            fd = ((gy * oracle.droi_pool_forward(x, rois, op, mask, k, gamma, lib=lib)).sum() -
+                  (gy * oracle.droi_pool_forward(x, rois, om, mask, k, gamma, lib=lib)).sum()) / (2 * eps)
+            assert abs(fd - goff[n, q]) <= 1e-6 * (1 + abs(fd)), (n, q, fd, goff[n, q])
 
 
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -49,6 +49,17 @@ MUTANTS = {
     "predictor_mask_not_squashed": ("= 1.0 / (1.0 + exp(-acc));", "= acc;"),
     "predictor_dilation_ignored_in_x": ("wo * s->stride - s->pad + j * s->dil, c);",
                                         "wo * s->stride - s->pad + j, c);"),
+    "droi_offset_not_scaled_by_roi": ("gamma * off[(size_t)r * 2 * kk + 2 * t] * h : 0.0;",
+                                      "gamma * off[(size_t)r * 2 * kk + 2 * t] : 0.0;"),
+    "droi_swap_dy_dx": ("const double dy = off ? gamma * off[(size_t)r * 2 * kk + 2 * t] * h : 0.0;",
+                        "const double dy = off ? gamma * off[(size_t)r * 2 * kk + 2 * t + 1] * h : 0.0;"),
+    "droi_mean_over_rows_only": ("yb[c] = n > 0 ? m * acc / n : 0.0;", "yb[c] = n > 0 ? m * acc / (u1 - u0) : 0.0;"),
+    "droi_corner_x_for_y": ("acc += bilinear(x, s, b, c, roi[2] + u + dy, roi[1] + v + dx);",
+                            "acc += bilinear(x, s, b, c, roi[1] + u + dy, roi[1] + v + dx);"),
+    "droi_grad_x_missing_mask": ("gx[(((size_t)b * s->H + rr) * s->W + qq) * C + c] += g * m * wt;",
+                                 "gx[(((size_t)b * s->H + rr) * s->W + qq) * C + c] += g * wt;"),
+    "droi_grad_offset_missing_width": ("goff[(size_t)r * 2 * kk + 2 * t + 1] = g_dx * gamma * w;",
+                                       "goff[(size_t)r * 2 * kk + 2 * t + 1] = g_dx * gamma;"),
 }
 
 
