@@ -603,6 +603,106 @@ def run_predictor(args):
         dist.destroy_process_group()
 
 
+ROI_WORKLOAD = dict(B=2, H=38, W=50, C=256, R=600, k=7, gamma=0.1, max_side=32.0)
+
+
+def run_roi_pool(args):
+    """Times (modulated) deformable RoI pooling, forward and backward, on a
+    detector head: two 38x50x256 stride-16 maps, 300 RoIs per image, k = 7, bf16."""
+    import torch
+
+    import deformable_convolution_dcn_b200 as dcn
+    from deformable_convolution_dcn_b200 import inputs as gen
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist_init("nccl")
+    w = ROI_WORKLOAD
+    B, H, W, C, R, k, gamma = w["B"], w["H"], w["W"], w["C"], w["R"], w["k"], w["gamma"]
+    host = gen.roi_inputs(41, B, H, W, C, R, k, "bf16", max_side=w["max_side"])
+    fwd_bytes = 2 * (B * H * W * C + R * 3 * k * k + R * k * k * C) + 4 * R * 5
+    bwd_bytes = fwd_bytes + 4 * (B * H * W * C + R * 3 * k * k)
+    set_bytes = fwd_bytes + 4 * B * H * W * C
+    n_sets = max(2, min(64, math.ceil(3 * L2_BYTES / set_bytes) + 1))
+    sets = [{n: (None if t is None else t.to(device)) for n, t in host.items()} for _ in range(n_sets)]
+    f32 = dict(dtype=torch.float32, device=device)
+    outs = [dict(y=torch.empty((R, k, k, C), dtype=torch.bfloat16, device=device), gx=torch.empty((B, H, W, C), **f32),
+                 goff=torch.empty((R, 2 * k * k), **f32), gm=torch.empty((R, k * k), **f32)) for _ in range(n_sets)]
+    lib = dcn._load()
+    p = dcn.RoiParams(B, H, W, C, R, k, gamma, dcn.DCN_BF16, 0)
+    import ctypes
+    P = dcn._ptr
+
+    def passes(i):
+        d, o = sets[i % n_sets], outs[i % n_sets]
+        st = dcn._stream(device)
+        fw = lambda: dcn._check(lib.dcn_droi_pool_forward(ctypes.byref(p), P(d["x"]), P(d["rois"]), P(d["offset"]),
+                                                          P(d["mask"]), P(o["y"]), st))
+        bw = lambda: dcn._check(lib.dcn_droi_pool_backward(ctypes.byref(p), P(d["x"]), P(d["rois"]), P(d["offset"]),
+                                                           P(d["mask"]), P(d["grad_y"]), P(o["gx"]), P(o["goff"]),
+                                                           P(o["gm"]), st))
+        return [fw, bw]
+
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, n_sets)):
+            for f in passes(i):
+                f()
+    torch.cuda.synchronize()
+    dcn.check_status()
+    graphs = []
+    with torch.cuda.stream(stream):
+        for i in range(n_sets):
+            row = []
+            l0 = dcn.launch_count()
+            for f in passes(i):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    f()
+                row.append(g)
+            launches_per_step = dcn.launch_count() - l0
+            graphs.append(row)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(device)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(int(HOLD_CYCLES_PER_STEP * (2 * args.steps + 4)))
+        for i in range(args.steps):
+            evs[i][0].record(stream)
+            for j, g in enumerate(graphs[(args.warmup + i) % n_sets]):
+                g.replay()
+                evs[i][j + 1].record(stream)
+    torch.cuda.synchronize()
+    barrier(device)
+    clk = clocks.stop()
+    dcn.check_status()
+    fwd_us = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in evs) * 1e3, device)
+    bwd_us = max_over_ranks(statistics.mean(e[1].elapsed_time(e[2]) for e in evs) * 1e3, device)
+    pk, pk_src = peaks()
+    ach = fwd_bytes / (fwd_us * 1e-6) / 1e9
+    if rank == 0:
+        print(json.dumps({
+            "metric": "deformable RoI pooling forward GB/s (algorithmic bytes)", "value": round(world * ach, 1),
+            "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round((fwd_us + bwd_us) / 1e3, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "modulated deformable RoI pooling, two 38x50x256 maps (600x800 image at stride "
+                                   "16), 300 RoIs per image with sides up to 32 feature pixels, k=7, gamma=0.1",
+                       "l2": "inputs and outputs rotate over %d independent sets" % n_sets},
+            "forward": {"us": round(fwd_us, 2), "bytes": fwd_bytes},
+            "backward": {"us": round(bwd_us, 2), "bytes": bwd_bytes},
+            "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(ach / pk["hbm_gbs"], 4), "traffic": None, "peak_source": pk_src},
+            "gpu_launches": launches_per_step * args.steps, "clocks": clk}), flush=True)
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -614,6 +714,8 @@ def main(argv=None):
     ap.add_argument("--forward-only", action="store_true", help="time the forward alone (not the default step)")
     ap.add_argument("--predictor", action="store_true",
                     help="time the layer's offset/mask predictor instead of the default step")
+    ap.add_argument("--roi-pool", action="store_true",
+                    help="time deformable RoI pooling (forward and backward) on a detector-head workload")
     ap.add_argument("--dp", action="store_true",
                     help="with several GPUs: data-parallel step (grad_weight and grad_bias all-reduced every step) "
                          "instead of independent replicas")
@@ -628,6 +730,8 @@ def main(argv=None):
         run_reference(args)
     elif args.predictor:
         run_predictor(args)
+    elif args.roi_pool:
+        run_roi_pool(args)
     else:
         run_ours(args)
 

@@ -52,6 +52,11 @@ class Params(ctypes.Structure):
                                             "dtype")] + [("flags", ctypes.c_uint)]
 
 
+class RoiParams(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("B", "H", "W", "C", "R", "k")] + [
+        ("gamma", ctypes.c_float), ("dtype", ctypes.c_int), ("flags", ctypes.c_uint)]
+
+
 def library_path() -> str:
     return _LIB_PATH
 
@@ -80,6 +85,9 @@ def _load():
         lib.dcn_predict_workspace_size.argtypes = [P]
         lib.dcn_predict_workspace_size.restype = sz
         lib.dcn_predict_offset_mask.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
+        RP = ctypes.POINTER(RoiParams)
+        lib.dcn_droi_pool_forward.argtypes = [RP, vp, vp, vp, vp, vp, vp]
+        lib.dcn_droi_pool_backward.argtypes = [RP, vp, vp, vp, vp, vp, fp, fp, fp, vp]
         lib.dcn_last_error_string.restype = ctypes.c_char_p
         lib.dcn_check_status.restype = ctypes.c_int
         lib.dcn_launch_count.restype = ctypes.c_ulonglong
@@ -235,6 +243,58 @@ def predict_offset_mask(x, w_pred, b_pred, K, stride=1, padding=0, dilation=1, G
     _check(lib.dcn_predict_offset_mask(ctypes.byref(p), _ptr(x), _ptr(w_pred), _ptr(b_pred), _ptr(offset),
                                        _ptr(mask), _ptr(workspace), nbytes, _stream(x.device)))
     return offset, mask
+
+
+def _roi_params(x, rois, k, gamma):
+    if x.dim() != 4:
+        raise ValueError("x must be [B, H, W, C]")
+    if x.dtype not in _DTYPES:
+        raise TypeError("x must be float32 or bfloat16, got %s" % x.dtype)
+    if rois.dim() != 2 or rois.shape[1] != 5 or rois.dtype != torch.float32:
+        raise ValueError("rois must be a float32 [R, 5] tensor of (b, x1, y1, x2, y2)")
+    B, H, W, C = x.shape
+    return RoiParams(B, H, W, C, rois.shape[0], int(k), float(gamma), _DTYPES[x.dtype], 0)
+
+
+def _check_roi_inputs(p, x, rois, offset, mask):
+    kk = p.k * p.k
+    if offset is not None and tuple(offset.shape) != (p.R, 2 * kk):
+        raise ValueError("offset must be [R, 2*k*k] = %s" % ((p.R, 2 * kk),))
+    if mask is not None and tuple(mask.shape) != (p.R, kk):
+        raise ValueError("mask must be [R, k*k] = %s" % ((p.R, kk),))
+    _check_tensors(x.dtype, x.device, x=x, offset=offset, mask=mask)
+    _check_tensors(torch.float32, x.device, rois=rois)
+
+
+def droi_pool_forward(x, rois, offset, mask, k, gamma=1.0, *, out=None):
+    """(Modulated) deformable RoI pooling: y [R, k, k, C] from x [B, H, W, C], rois float32 [R, 5]
+    = (b, x1, y1, x2, y2), offset [R, 2k^2] (normalised, or None) and mask [R, k^2] (or None)."""
+    lib = _load()
+    p = _roi_params(x, rois, k, gamma)
+    _check_roi_inputs(p, x, rois, offset, mask)
+    if out is None:
+        out = torch.empty((p.R, p.k, p.k, p.C), dtype=x.dtype, device=x.device)
+    if tuple(out.shape) != (p.R, p.k, p.k, p.C):
+        raise ValueError("out must be [R, k, k, C]")
+    _check_tensors(x.dtype, x.device, out=out)
+    _check(lib.dcn_droi_pool_forward(ctypes.byref(p), _ptr(x), _ptr(rois), _ptr(offset), _ptr(mask), _ptr(out),
+                                     _stream(x.device)))
+    return out
+
+
+def droi_pool_backward(x, rois, offset, mask, grad_y, k, gamma=1.0, *, need_offset=True, need_mask=True):
+    """(grad_x [B, H, W, C], grad_offset [R, 2k^2] or None, grad_mask [R, k^2] or None), float32."""
+    lib = _load()
+    p = _roi_params(x, rois, k, gamma)
+    _check_roi_inputs(p, x, rois, offset, mask)
+    _check_tensors(x.dtype, x.device, grad_y=grad_y)
+    f32 = dict(dtype=torch.float32, device=x.device)
+    gx = torch.empty(tuple(x.shape), **f32)
+    goff = torch.empty((p.R, 2 * p.k * p.k), **f32) if (need_offset and offset is not None) else None
+    gm = torch.empty((p.R, p.k * p.k), **f32) if (need_mask and mask is not None) else None
+    _check(lib.dcn_droi_pool_backward(ctypes.byref(p), _ptr(x), _ptr(rois), _ptr(offset), _ptr(mask), _ptr(grad_y),
+                                      _ptr(gx), _ptr(goff), _ptr(gm), _stream(x.device)))
+    return gx, goff, gm
 
 
 def backward_data(x, offset, mask, weight, grad_y, stride=1, padding=0, dilation=1, *, need_input=True,

@@ -456,6 +456,75 @@ int dcn_predict_offset_mask(const dcn_params_t* params, const void* x, const voi
     return ok();
 }
 
+// ------------------------------------------------ deformable RoI pooling --
+
+static int roi_args(const dcn_roi_params_t* p, dcn::RoiArgs& a, const float* rois) {
+    if (!p) return fail(DCN_ERR_INVALID_ARG, "params is NULL");
+    if (p->B < 1 || p->H < 1 || p->W < 1 || p->C < 1 || p->R < 0 || p->k < 1 || p->k > 64)
+        return fail(DCN_ERR_INVALID_ARG,
+                    "need B, H, W, C >= 1, R >= 0 and 1 <= k <= 64 (B=%d H=%d W=%d C=%d R=%d k=%d)", p->B, p->H, p->W,
+                    p->C, p->R, p->k);
+    if (p->dtype != DCN_F32 && p->dtype != DCN_BF16) return fail(DCN_ERR_UNSUPPORTED, "unknown dtype %d", p->dtype);
+    if (!(p->gamma > -3.0e38f && p->gamma < 3.0e38f)) return fail(DCN_ERR_INVALID_ARG, "gamma must be finite");
+    if ((long long)p->B * p->H * p->W * p->C > kMaxElems || (long long)p->R * p->k * p->k * p->C > kMaxElems)
+        return fail(DCN_ERR_UNSUPPORTED, "a tensor exceeds 2^31-1 elements");
+    a.rois = rois;
+    a.B = p->B;
+    a.H = p->H;
+    a.W = p->W;
+    a.C = p->C;
+    a.R = p->R;
+    a.k = p->k;
+    a.gamma = p->gamma;
+    return DCN_OK;
+}
+
+int dcn_droi_pool_forward(const dcn_roi_params_t* params, const void* x, const float* rois, const void* offset,
+                          const void* mask, void* y, void* stream) {
+    dcn::RoiArgs a;
+    TRY(roi_args(params, a, rois));
+    const size_t es = elem_size(params->dtype);
+    const bool any = params->R > 0;
+    TRY(check_ptr(x, "x", es, true));
+    TRY(check_ptr(rois, "rois", 4, any));
+    TRY(check_ptr(offset, "offset", es, false));
+    TRY(check_ptr(mask, "mask", es, false));
+    TRY(check_ptr(y, "y", es, any));
+    if (!any) return ok();
+    cudaError_t e = dcn::droi_forward(a, params->dtype == DCN_BF16, x, offset, mask, y, (cudaStream_t)stream);
+    g_launches += 1;
+    if (e != cudaSuccess) return cuda_fail(e, "RoI pooling forward launch");
+    return ok();
+}
+
+int dcn_droi_pool_backward(const dcn_roi_params_t* params, const void* x, const float* rois, const void* offset,
+                           const void* mask, const void* grad_y, float* grad_x, float* grad_offset, float* grad_mask,
+                           void* stream) {
+    dcn::RoiArgs a;
+    TRY(roi_args(params, a, rois));
+    const size_t es = elem_size(params->dtype);
+    const bool any = params->R > 0;
+    TRY(check_ptr(x, "x", es, true));
+    TRY(check_ptr(rois, "rois", 4, any));
+    TRY(check_ptr(offset, "offset", es, false));
+    TRY(check_ptr(mask, "mask", es, false));
+    TRY(check_ptr(grad_y, "grad_y", es, any));
+    TRY(check_ptr(grad_x, "grad_x", 4, true));
+    TRY(check_ptr(grad_offset, "grad_offset", 4, false));
+    TRY(check_ptr(grad_mask, "grad_mask", 4, false));
+    if (grad_offset && !offset) return fail(DCN_ERR_INVALID_ARG, "grad_offset needs offset");
+    if (grad_mask && !mask) return fail(DCN_ERR_INVALID_ARG, "grad_mask needs mask");
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cudaMemsetAsync(grad_x, 0, sizeof(float) * (size_t)a.B * a.H * a.W * a.C, st);
+    g_launches += 1;
+    if (e != cudaSuccess) return cuda_fail(e, "zeroing grad_x");
+    if (!any) return ok();
+    e = dcn::droi_backward(a, params->dtype == DCN_BF16, x, offset, mask, grad_y, grad_x, grad_offset, grad_mask, st);
+    g_launches += 1;
+    if (e != cudaSuccess) return cuda_fail(e, "RoI pooling backward launch");
+    return ok();
+}
+
 const char* dcn_last_error_string(void) { return g_err.c_str(); }
 
 int dcn_check_status(void) {

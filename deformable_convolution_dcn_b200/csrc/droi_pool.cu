@@ -1,0 +1,210 @@
+// (Modulated) deformable RoI pooling, forward and backward (notes, "可变形ROI
+// pooling": a RoI of w x h is cut into k x k bins, each output averages the
+// pixels of its bin; the deformable form moves every bin by an offset given as
+// a fraction of the RoI's width and height, read by bilinear interpolation;
+// DCNv2 section 3.2: a modulation scalar per bin).
+//
+//   roi r = (b, x1, y1, x2, y2), h = max(y2 - y1, 0), w = max(x2 - x1, 0);
+//   bin t = i*k + j holds the integer offsets (u, v), floor(i*h/k) <= u <
+//   ceil((i+1)*h/k) and likewise v with w, n of them;
+//   y[r][i][j][c] = m / n * sum over (u, v) of x_b(y1 + u + dy, x1 + v + dx, c),
+//   (dy, dx) = gamma * (off[r][2t] * h, off[r][2t+1] * w), m = mask[r][t] or 1,
+//   bilinear with neighbours outside the map contributing zero; 0 for an empty
+//   bin or a batch index outside [0, B).
+//
+// One block per (RoI, bin), threads over channels (NHWC: a warp reads 32
+// consecutive channels of one neighbour). Samples whose bilinear footprint
+// misses the map contribute exactly zero, so the sample loops run only over the
+// rows and columns that can touch it, which also bounds them for any RoI size;
+// n still counts the whole bin. The backward scatters grad_x with float atomics
+// and reduces the bin's offset and mask gradients over its channels in a fixed
+// order in shared memory (no atomics).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dcn {
+namespace {
+
+struct BinGeom {
+    int b;             // batch index, -1 when outside [0, B)
+    float y1, x1, h, w;
+    float dy, dx, m;
+    float n;           // samples in the bin (the divisor)
+    int u_lo, u_hi, v_lo, v_hi;  // sample rows / columns that can touch the map
+};
+
+template <typename T>
+__device__ __forceinline__ BinGeom bin_geom(const RoiArgs& a, const T* off, const T* mask, int r, int t) {
+    BinGeom g;
+    const float* roi = a.rois + (size_t)r * 5;
+    // the batch index is the RoI's first value truncated toward zero; outside [0, B) the RoI pools to zeros
+    g.b = (roi[0] > -1.f && roi[0] < (float)a.B) ? (int)roi[0] : -1;
+    g.x1 = roi[1];
+    g.y1 = roi[2];
+    g.h = fmaxf(roi[4] - roi[2], 0.f);
+    g.w = fmaxf(roi[3] - roi[1], 0.f);
+    const int i = t / a.k, j = t - i * a.k;
+    const float fu0 = floorf(i * g.h / a.k), fu1 = ceilf((i + 1) * g.h / a.k);
+    const float fv0 = floorf(j * g.w / a.k), fv1 = ceilf((j + 1) * g.w / a.k);
+    g.n = (fu1 - fu0) * (fv1 - fv0);
+    const int kk = a.k * a.k;
+    g.dy = off ? a.gamma * ldf(off + (size_t)r * 2 * kk + 2 * t) * g.h : 0.f;
+    g.dx = off ? a.gamma * ldf(off + (size_t)r * 2 * kk + 2 * t + 1) * g.w : 0.f;
+    g.m = mask ? ldf(mask + (size_t)r * kk + t) : 1.f;
+    // rows u with y1 + u + dy in (-1, H) (a sample at -1 or H exactly adds zero), clamped before conversion
+    const float lim = 1073741824.f;
+    const float ulo = fmaxf(fu0, floorf(-1.f - g.y1 - g.dy)), uhi = fminf(fu1, ceilf((float)a.H - g.y1 - g.dy) + 1.f);
+    const float vlo = fmaxf(fv0, floorf(-1.f - g.x1 - g.dx)), vhi = fminf(fv1, ceilf((float)a.W - g.x1 - g.dx) + 1.f);
+    g.u_lo = (int)fminf(fmaxf(ulo, -lim), lim);
+    g.u_hi = (int)fminf(fmaxf(uhi, -lim), lim);
+    g.v_lo = (int)fminf(fmaxf(vlo, -lim), lim);
+    g.v_hi = (int)fminf(fmaxf(vhi, -lim), lim);
+    if (!(g.n > 0.f)) g.b = -1;
+    return g;
+}
+
+struct Corner {
+    int y0, x0;
+    float ly, lx;
+};
+
+__device__ __forceinline__ Corner corner(float py, float px) {
+    Corner c;
+    const float fy = floorf(py), fx = floorf(px);
+    c.y0 = (int)fy;
+    c.x0 = (int)fx;
+    c.ly = py - fy;
+    c.lx = px - fx;
+    return c;
+}
+
+template <typename T>
+__device__ __forceinline__ float px_or_zero(const T* xb, const RoiArgs& a, int r, int q, int c) {
+    if (r < 0 || r >= a.H || q < 0 || q >= a.W) return 0.f;
+    return ldf(xb + ((size_t)r * a.W + q) * a.C + c);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) droi_fwd_kernel(RoiArgs a, const T* __restrict__ x, const T* __restrict__ off,
+                                                       const T* __restrict__ mask, T* __restrict__ y) {
+    const int bin = blockIdx.x, kk = a.k * a.k;
+    const int r = bin / kk, t = bin - r * kk;
+    const BinGeom g = bin_geom(a, off, mask, r, t);
+    T* yb = y + (size_t)bin * a.C;
+    if (g.b < 0) {
+        for (int c = threadIdx.x; c < a.C; c += blockDim.x) yb[c] = from_float<T>(0.f);
+        return;
+    }
+    const T* xb = x + (size_t)g.b * a.H * a.W * a.C;
+    for (int c = threadIdx.x; c < a.C; c += blockDim.x) {
+        float acc = 0.f;
+        for (int u = g.u_lo; u < g.u_hi; ++u)
+            for (int v = g.v_lo; v < g.v_hi; ++v) {
+                const Corner q = corner(g.y1 + u + g.dy, g.x1 + v + g.dx);
+                acc += (1.f - q.ly) * ((1.f - q.lx) * px_or_zero(xb, a, q.y0, q.x0, c) +
+                                       q.lx * px_or_zero(xb, a, q.y0, q.x0 + 1, c)) +
+                       q.ly * ((1.f - q.lx) * px_or_zero(xb, a, q.y0 + 1, q.x0, c) +
+                               q.lx * px_or_zero(xb, a, q.y0 + 1, q.x0 + 1, c));
+            }
+        yb[c] = from_float<T>(g.m * acc / g.n);
+    }
+}
+
+__device__ __forceinline__ void add_if_inside(float* gxb, const RoiArgs& a, int r, int q, int c, float v) {
+    if (r < 0 || r >= a.H || q < 0 || q >= a.W) return;
+    atomicAdd(gxb + ((size_t)r * a.W + q) * a.C + c, v);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) droi_bwd_kernel(RoiArgs a, const T* __restrict__ x, const T* __restrict__ off,
+                                                       const T* __restrict__ mask, const T* __restrict__ gy,
+                                                       float* __restrict__ gx, float* __restrict__ goff,
+                                                       float* __restrict__ gmask) {
+    __shared__ float red[3][256];
+    const int bin = blockIdx.x, kk = a.k * a.k;
+    const int r = bin / kk, t = bin - r * kk;
+    const BinGeom g = bin_geom(a, off, mask, r, t);
+    float s_dy = 0.f, s_dx = 0.f, s_m = 0.f;
+    if (g.b >= 0) {
+        const T* xb = x + (size_t)g.b * a.H * a.W * a.C;
+        float* gxb = gx + (size_t)g.b * a.H * a.W * a.C;
+        const T* gyb = gy + (size_t)bin * a.C;
+        for (int c = threadIdx.x; c < a.C; c += blockDim.x) {
+            const float gc = ldf(gyb + c) / g.n;
+            const float gm = gc * g.m;
+            for (int u = g.u_lo; u < g.u_hi; ++u)
+                for (int v = g.v_lo; v < g.v_hi; ++v) {
+                    const Corner q = corner(g.y1 + u + g.dy, g.x1 + v + g.dx);
+                    const float v00 = px_or_zero(xb, a, q.y0, q.x0, c), v01 = px_or_zero(xb, a, q.y0, q.x0 + 1, c);
+                    const float v10 = px_or_zero(xb, a, q.y0 + 1, q.x0, c);
+                    const float v11 = px_or_zero(xb, a, q.y0 + 1, q.x0 + 1, c);
+                    add_if_inside(gxb, a, q.y0, q.x0, c, gm * (1.f - q.ly) * (1.f - q.lx));
+                    add_if_inside(gxb, a, q.y0, q.x0 + 1, c, gm * (1.f - q.ly) * q.lx);
+                    add_if_inside(gxb, a, q.y0 + 1, q.x0, c, gm * q.ly * (1.f - q.lx));
+                    add_if_inside(gxb, a, q.y0 + 1, q.x0 + 1, c, gm * q.ly * q.lx);
+                    s_dy += gm * ((1.f - q.lx) * (v10 - v00) + q.lx * (v11 - v01));
+                    s_dx += gm * ((1.f - q.ly) * (v01 - v00) + q.ly * (v11 - v10));
+                    s_m += gc * ((1.f - q.ly) * ((1.f - q.lx) * v00 + q.lx * v01) +
+                                 q.ly * ((1.f - q.lx) * v10 + q.lx * v11));
+                }
+        }
+    }
+    if (goff == nullptr && gmask == nullptr) return;
+    red[0][threadIdx.x] = s_dy;
+    red[1][threadIdx.x] = s_dx;
+    red[2][threadIdx.x] = s_m;
+    __syncthreads();
+    for (int st = blockDim.x / 2; st > 0; st >>= 1) {
+        if ((int)threadIdx.x < st) {
+            red[0][threadIdx.x] += red[0][threadIdx.x + st];
+            red[1][threadIdx.x] += red[1][threadIdx.x + st];
+            red[2][threadIdx.x] += red[2][threadIdx.x + st];
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        const bool live = g.b >= 0;
+        if (goff) {
+            goff[(size_t)r * 2 * kk + 2 * t] = live ? red[0][0] * a.gamma * g.h : 0.f;
+            goff[(size_t)r * 2 * kk + 2 * t + 1] = live ? red[1][0] * a.gamma * g.w : 0.f;
+        }
+        if (gmask) gmask[(size_t)r * kk + t] = live ? red[2][0] : 0.f;
+    }
+}
+
+// a power of two from 32 to 256 covering the channels (the reduction halves it)
+int block_for(int C) {
+    int t = 32;
+    while (t < C && t < 256) t *= 2;
+    return t;
+}
+
+}  // namespace
+
+cudaError_t droi_forward(const RoiArgs& a, int dtype_bf16, const void* x, const void* off, const void* mask, void* y,
+                         cudaStream_t st) {
+    const long long bins = (long long)a.R * a.k * a.k;
+    if (bins == 0) return cudaSuccess;
+    if (dtype_bf16)
+        droi_fwd_kernel<bf16><<<(unsigned)bins, block_for(a.C), 0, st>>>(a, (const bf16*)x, (const bf16*)off,
+                                                                         (const bf16*)mask, (bf16*)y);
+    else
+        droi_fwd_kernel<float><<<(unsigned)bins, block_for(a.C), 0, st>>>(a, (const float*)x, (const float*)off,
+                                                                          (const float*)mask, (float*)y);
+    return cudaGetLastError();
+}
+
+cudaError_t droi_backward(const RoiArgs& a, int dtype_bf16, const void* x, const void* off, const void* mask,
+                          const void* gy, float* gx, float* goff, float* gmask, cudaStream_t st) {
+    const long long bins = (long long)a.R * a.k * a.k;
+    if (bins == 0) return cudaSuccess;
+    if (dtype_bf16)
+        droi_bwd_kernel<bf16><<<(unsigned)bins, block_for(a.C), 0, st>>>(
+            a, (const bf16*)x, (const bf16*)off, (const bf16*)mask, (const bf16*)gy, gx, goff, gmask);
+    else
+        droi_bwd_kernel<float><<<(unsigned)bins, block_for(a.C), 0, st>>>(
+            a, (const float*)x, (const float*)off, (const float*)mask, (const float*)gy, gx, goff, gmask);
+    return cudaGetLastError();
+}
+
+}  // namespace dcn

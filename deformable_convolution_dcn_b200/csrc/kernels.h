@@ -29,6 +29,17 @@ size_t fwd_tc_static_scratch_bytes();
 cudaError_t fwd_tc_noalloc(const Shape& s, const void* x, const void* off, const void* mask, const void* w,
                            const void* bias, void* y, unsigned* status, cudaStream_t st, int* launches);
 
+// droi_pool.cu — (modulated) deformable RoI pooling, forward and backward (grad_x zeroed by the caller).
+struct RoiArgs {
+    const float* rois;  // [R, 5]: b, x1, y1, x2, y2
+    int B, H, W, C, R, k;
+    float gamma;
+};
+cudaError_t droi_forward(const RoiArgs& a, int dtype_bf16, const void* x, const void* off, const void* mask, void* y,
+                         cudaStream_t st);
+cudaError_t droi_backward(const RoiArgs& a, int dtype_bf16, const void* x, const void* off, const void* mask,
+                          const void* gy, float* gx, float* goff, float* gmask, cudaStream_t st);
+
 // pred_tc.cu — the bfloat16 stride-1 offset/mask predictor on tcgen05, sigmoid and split fused (no workspace).
 bool pred_tc_supported(const Shape& s);
 cudaError_t pred_tc(const Shape& s, const void* x, const void* w, const void* bias, void* off, void* mask,

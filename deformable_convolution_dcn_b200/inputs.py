@@ -233,6 +233,32 @@ def predictor_inputs(seed: int, s: LayerShape, dtype: str = "f32", bias: bool = 
     return {k: (None if v is None else v.to(dt).to(device)) for k, v in out.items()}
 
 
+def roi_inputs(seed: int, B: int, H: int, W: int, C: int, R: int, k: int, dtype: str = "f32", offsets: bool = True,
+               mask: bool = True, max_side: float | None = None, device="cpu"):
+    """Inputs of deformable RoI pooling: x [B, H, W, C] ~ N(0, 1); R RoIs (b, x1,
+    y1, x2, y2) float32 with corners on a 1/8-pixel grid, sides up to max_side
+    (default the map's), some reaching past the map's edges; normalised offsets
+    [R, 2k^2] ~ U(-0.3, 0.3) rounded to 1/64; masks [R, k^2] ~ U(0, 1)."""
+    g = torch.Generator().manual_seed(seed)
+    dt = torch_dtype(dtype)
+    x = torch.randn((B, C, H, W), generator=g).permute(0, 2, 3, 1).contiguous()
+    side = max_side or float(max(H, W))
+    b = torch.randint(0, B, (R,), generator=g).float()
+    cx = torch.rand(R, generator=g) * (W + 2) - 1
+    cy = torch.rand(R, generator=g) * (H + 2) - 1
+    ww = torch.rand(R, generator=g) * side
+    hh = torch.rand(R, generator=g) * side
+    q = lambda v: torch.round(v * 8) / 8
+    rois = torch.stack([b, q(cx - ww / 2), q(cy - hh / 2), q(cx + ww / 2), q(cy + hh / 2)], dim=1)
+    # offsets on a 1/64 grid: with dyadic gamma every sample position is exact in float32 and float64
+    off = (torch.round((torch.rand((R, 2 * k * k), generator=g) * 0.6 - 0.3) * 64) / 64) if offsets else None
+    m = torch.rand((R, k * k), generator=g) if mask else None
+    gy = torch.randn((R, k, k, C), generator=g)
+    out = {"x": x.to(dt), "rois": rois, "offset": None if off is None else off.to(dt),
+           "mask": None if m is None else m.to(dt), "grad_y": gy.to(dt)}
+    return {n: (None if v is None else v.to(device)) for n, v in out.items()}
+
+
 def as_f64(t):
     """numpy float64 copy of a tensor's stored values (None passes through)."""
     if t is None:

@@ -199,6 +199,45 @@ DCN_API int dcn_predict_offset_mask(const dcn_params_t* params, const void* x, c
                                     const void* b_pred, void* offset, void* mask, void* workspace,
                                     size_t workspace_bytes, void* stream);
 
+/* (Modulated) deformable RoI pooling (notes, "可变形ROI pooling"; the explainer's
+ * "可变形RoI池化" paragraph; DCNv2 section 3.2 for the per-bin modulation). The
+ * pages describe it in words only; the computation is this reading of them:
+ *   roi r = (b, x1, y1, x2, y2) in feature-map pixel coordinates, b truncated
+ *   toward zero; h = max(y2 - y1, 0), w = max(x2 - x1, 0);
+ *   bin t = i*k + j holds the integer offsets (u, v) with
+ *     floor(i*h/k) <= u < ceil((i+1)*h/k),  floor(j*w/k) <= v < ceil((j+1)*w/k),
+ *   n of them; its shift is (dy, dx) = gamma * (offset[r][2t] * h, offset[r][2t+1] * w);
+ *   y[r][i][j][c] = m / n * sum over (u, v) of x_b(y1 + u + dy, x1 + v + dx, c),
+ *   m = mask[r][t] (1 when mask is NULL), bilinear sampling whose neighbours
+ *   outside the map contribute zero (as in the layer); 0 for an empty bin or a
+ *   batch index outside [0, B).
+ * Layouts: x [B, H, W, C]; rois [R, 5] float32; offset [R, 2*k*k] (normalised;
+ * NULL: plain RoI pooling); mask [R, k*k] or NULL; y and grad_y [R, k, k, C].
+ * x, offset, mask, y and grad_y are in `dtype`; gradients are float32. The
+ * caller owns all device buffers; work is enqueued on `stream`; argument
+ * problems return before anything is enqueued. */
+typedef struct {
+    int B, H, W, C;   /* feature map x [B, H, W, C] */
+    int R, k;         /* RoIs (R >= 0) and bins per side (1 <= k <= 64) */
+    float gamma;      /* scale of the normalised offsets */
+    int dtype;        /* DCN_F32 or DCN_BF16 */
+    unsigned flags;   /* reserved, 0 */
+} dcn_roi_params_t;
+
+/* Writes y. */
+DCN_API int dcn_droi_pool_forward(const dcn_roi_params_t* params, const void* x, const float* rois,
+                                  const void* offset, const void* mask, void* y, void* stream);
+
+/* Given grad_y = dL/dy: grad_x (required, overwritten), grad_offset [R, 2*k*k]
+ * (with respect to the normalised offsets; NULL: not computed; must be NULL
+ * when offset is NULL) and grad_mask [R, k*k] (NULL: not computed; must be NULL
+ * when mask is NULL). The RoI coordinates get no gradient. The offset gradient
+ * is taken through floor(), as in the layer. grad_x is accumulated with float
+ * atomics, so its last bits may differ between runs. */
+DCN_API int dcn_droi_pool_backward(const dcn_roi_params_t* params, const void* x, const float* rois,
+                                   const void* offset, const void* mask, const void* grad_y, float* grad_x,
+                                   float* grad_offset, float* grad_mask, void* stream);
+
 /* The calling thread's last error message ("" after success). */
 DCN_API const char* dcn_last_error_string(void);
 
