@@ -12,8 +12,9 @@
 //   bilinear with neighbours outside the map contributing zero; 0 for an empty
 //   bin or a batch index outside [0, B).
 //
-// One block per (RoI, bin), threads over channels (NHWC: a warp reads 32
-// consecutive channels of one neighbour). Samples whose bilinear footprint
+// One block per (RoI, bin), threads over channels (NHWC: consecutive threads
+// read consecutive 16-byte channel vectors of one neighbour; one channel per
+// thread when C is not a multiple of 16 bytes). Samples whose bilinear footprint
 // misses the map contribute exactly zero, so the sample loops run only over the
 // rows and columns that can touch it, which also bounds them for any RoI size;
 // n still counts the whole bin. The backward scatters grad_x with float atomics
@@ -110,6 +111,90 @@ __global__ void __launch_bounds__(256) droi_fwd_kernel(RoiArgs a, const T* __res
     }
 }
 
+// 16 bytes of channels: 8 bf16 or 4 float32, widened to float
+template <typename T>
+struct Vec16 {
+    static constexpr int N = 16 / sizeof(T);
+};
+
+template <typename T>
+__device__ __forceinline__ void load16(const T* p, float (&v)[Vec16<T>::N]) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    if constexpr (sizeof(T) == 2) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[q]));
+            v[2 * q] = f.x;
+            v[2 * q + 1] = f.y;
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) v[q] = __uint_as_float(w[q]);
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ void store16(T* p, const float (&v)[Vec16<T>::N]) {
+    uint32_t w[4];
+    if constexpr (sizeof(T) == 2) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * q], v[2 * q + 1]);
+            w[q] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) w[q] = __float_as_uint(v[q]);
+    }
+    *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// As droi_fwd_kernel, 16 bytes of channels per thread (C a multiple of 16 bytes, x and y 16-byte aligned).
+template <typename T>
+__global__ void __launch_bounds__(256) droi_fwd_vec_kernel(RoiArgs a, const T* __restrict__ x,
+                                                           const T* __restrict__ off, const T* __restrict__ mask,
+                                                           T* __restrict__ y) {
+    constexpr int N = Vec16<T>::N;
+    const int bin = blockIdx.x, kk = a.k * a.k;
+    const int r = bin / kk, t = bin - r * kk;
+    const BinGeom g = bin_geom(a, off, mask, r, t);
+    T* yb = y + (size_t)bin * a.C;
+    const int nv = a.C / N;
+    if (g.b < 0) {
+        float z[N];
+#pragma unroll
+        for (int e = 0; e < N; ++e) z[e] = 0.f;
+        for (int cv = threadIdx.x; cv < nv; cv += blockDim.x) store16(yb + cv * N, z);
+        return;
+    }
+    const T* xb = x + (size_t)g.b * a.H * a.W * a.C;
+    for (int cv = threadIdx.x; cv < nv; cv += blockDim.x) {
+        const int c = cv * N;
+        float acc[N];
+#pragma unroll
+        for (int e = 0; e < N; ++e) acc[e] = 0.f;
+        for (int u = g.u_lo; u < g.u_hi; ++u)
+            for (int v = g.v_lo; v < g.v_hi; ++v) {
+                const Corner q = corner(g.y1 + u + g.dy, g.x1 + v + g.dx);
+#pragma unroll
+                for (int nb = 0; nb < 4; ++nb) {
+                    const int rr = q.y0 + (nb >> 1), cc = q.x0 + (nb & 1);
+                    if (rr < 0 || rr >= a.H || cc < 0 || cc >= a.W) continue;
+                    const float wt = ((nb >> 1) ? q.ly : 1.f - q.ly) * ((nb & 1) ? q.lx : 1.f - q.lx);
+                    float vv[N];
+                    load16(xb + ((size_t)rr * a.W + cc) * a.C + c, vv);
+#pragma unroll
+                    for (int e = 0; e < N; ++e) acc[e] += wt * vv[e];
+                }
+            }
+        const float sc = g.m / g.n;
+#pragma unroll
+        for (int e = 0; e < N; ++e) acc[e] *= sc;
+        store16(yb + c, acc);
+    }
+}
+
 __device__ __forceinline__ void add_if_inside(float* gxb, const RoiArgs& a, int r, int q, int c, float v) {
     if (r < 0 || r >= a.H || q < 0 || q >= a.W) return;
     atomicAdd(gxb + ((size_t)r * a.W + q) * a.C + c, v);
@@ -185,7 +270,16 @@ cudaError_t droi_forward(const RoiArgs& a, int dtype_bf16, const void* x, const 
                          cudaStream_t st) {
     const long long bins = (long long)a.R * a.k * a.k;
     if (bins == 0) return cudaSuccess;
-    if (dtype_bf16)
+    const int es = dtype_bf16 ? 2 : 4, n = 16 / es;
+    const bool vec = a.C % n == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0 &&
+                     (reinterpret_cast<uintptr_t>(y) & 15) == 0;
+    if (vec && dtype_bf16)
+        droi_fwd_vec_kernel<bf16><<<(unsigned)bins, block_for(a.C / n), 0, st>>>(
+            a, (const bf16*)x, (const bf16*)off, (const bf16*)mask, (bf16*)y);
+    else if (vec)
+        droi_fwd_vec_kernel<float><<<(unsigned)bins, block_for(a.C / n), 0, st>>>(
+            a, (const float*)x, (const float*)off, (const float*)mask, (float*)y);
+    else if (dtype_bf16)
         droi_fwd_kernel<bf16><<<(unsigned)bins, block_for(a.C), 0, st>>>(a, (const bf16*)x, (const bf16*)off,
                                                                          (const bf16*)mask, (bf16*)y);
     else
