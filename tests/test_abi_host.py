@@ -124,6 +124,38 @@ def test_predictor_tensor_core_path_needs_no_workspace(lib):
     assert lib.dcn_predict_offset_mask(ctypes.byref(p16), f, odd, None, f, f, None, 0, None) == EUNSUP
 
 
+def test_roi_pool_arguments(lib):
+    f = ctypes.c_void_p(1 << 20)
+
+    def RP(**kw):
+        d = dict(B=2, H=8, W=9, C=16, R=5, k=3, gamma=0.5, dtype=0, flags=0)
+        d.update(kw)
+        return dcn.RoiParams(d["B"], d["H"], d["W"], d["C"], d["R"], d["k"], d["gamma"], d["dtype"], d["flags"])
+
+    fwd = lambda p, *a: lib.dcn_droi_pool_forward(ctypes.byref(p), *a, None)
+    bwd = lambda p, *a: lib.dcn_droi_pool_backward(ctypes.byref(p), *a, None)
+    for bad, code in ((dict(k=0), EINVAL), (dict(k=65), EINVAL), (dict(R=-1), EINVAL), (dict(C=0), EINVAL),
+                      (dict(B=0), EINVAL), (dict(dtype=9), EUNSUP), (dict(gamma=float("nan")), EINVAL),
+                      (dict(gamma=float("inf")), EINVAL), (dict(B=1024, H=1024, W=1024, C=8), EUNSUP)):
+        assert fwd(RP(**bad), f, f, None, None, f) == code, bad
+        assert lib.dcn_last_error_string().decode() != ""
+    assert fwd(RP(), None, f, None, None, f) == EINVAL
+    assert "x is NULL" in lib.dcn_last_error_string().decode()
+    assert fwd(RP(), f, None, None, None, f) == EINVAL
+    assert fwd(RP(), f, f, None, None, None) == EINVAL
+    assert fwd(RP(), f, ctypes.c_void_p((1 << 20) + 2), None, None, f) == EUNSUP
+    assert fwd(RP(dtype=1), f, f, ctypes.c_void_p((1 << 20) + 1), None, f) == EUNSUP
+    # no RoIs: nothing to do, nothing enqueued
+    assert fwd(RP(R=0), f, None, None, None, None) == OK
+    # gradients of absent inputs, and the required grad_x
+    assert bwd(RP(), f, f, None, None, f, f, f, None) == EINVAL
+    assert "grad_offset needs offset" in lib.dcn_last_error_string().decode()
+    assert bwd(RP(), f, f, f, None, f, f, None, f) == EINVAL
+    assert "grad_mask needs mask" in lib.dcn_last_error_string().decode()
+    assert bwd(RP(), f, f, f, f, f, None, None, None) == EINVAL
+    assert bwd(RP(), f, f, f, f, None, f, None, None) == EINVAL
+
+
 def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     import importlib
     monkeypatch.setattr(dcn, "_lib", None)
