@@ -88,6 +88,7 @@ def _load():
         RP = ctypes.POINTER(RoiParams)
         lib.dcn_droi_pool_forward.argtypes = [RP, vp, vp, vp, vp, vp, vp]
         lib.dcn_droi_pool_backward.argtypes = [RP, vp, vp, vp, vp, vp, fp, fp, fp, vp]
+        lib.dcn_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, vp]
         lib.dcn_last_error_string.restype = ctypes.c_char_p
         lib.dcn_check_status.restype = ctypes.c_int
         lib.dcn_launch_count.restype = ctypes.c_ulonglong

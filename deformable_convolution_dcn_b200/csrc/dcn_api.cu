@@ -537,6 +537,15 @@ int dcn_check_status(void) {
     return ok();
 }
 
+int dcn_selftest_wait_timeout(unsigned long long limit_cycles, void* stream) {
+    if (limit_cycles < 1000ull || limit_cycles > 4000000000ull)
+        return fail(DCN_ERR_INVALID_ARG, "limit_cycles must be in [1e3, 4e9], got %llu", limit_cycles);
+    cudaError_t e = dcn::selftest_wait_timeout((long long)limit_cycles, (cudaStream_t)stream);
+    g_launches += 1;
+    if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+    return ok();
+}
+
 unsigned long long dcn_launch_count(void) { return g_launches.load(); }
 
 }  // extern "C"

@@ -75,6 +75,9 @@ cudaError_t bwd_data_tc(const Shape& s, const void* x, const void* off, const vo
                         const void* gy, float* gx, float* goff, float* gmask, void* ws, size_t ws_bytes,
                         unsigned* status, cudaStream_t st, int* launches);
 
+// selftest.cu — a kernel whose bounded wait can only give up (failure-detection test).
+cudaError_t selftest_wait_timeout(long long limit_cycles, cudaStream_t st);
+
 // status.cu — the device status word that bounded waits report to; SM count.
 int num_sms();
 cudaError_t status_word_ptr(unsigned int** ptr);

@@ -246,6 +246,14 @@ DCN_API const char* dcn_last_error_string(void);
  * wait since the last check. */
 DCN_API int dcn_check_status(void);
 
+/* Failure-detection self-test (no counterpart on the pages): enqueues one
+ * kernel whose bounded mbarrier wait can never complete, through the same wait
+ * every tensor-core kernel uses; after limit_cycles clock cycles (1e3 to 4e9)
+ * it gives up, records the timeout in the device status word and ends
+ * normally. The next dcn_check_status() returns DCN_ERR_TIMEOUT (and clears the
+ * word); the context stays usable. Nothing faults, traps or hangs. */
+DCN_API int dcn_selftest_wait_timeout(unsigned long long limit_cycles, void* stream);
+
 /* Number of kernels (and memsets) this library has enqueued since the process
  * started, summed over threads. */
 DCN_API unsigned long long dcn_launch_count(void);

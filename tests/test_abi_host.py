@@ -156,6 +156,12 @@ def test_roi_pool_arguments(lib):
     assert bwd(RP(), f, f, f, f, None, f, None, None) == EINVAL
 
 
+def test_selftest_rejects_out_of_range_limits(lib):
+    assert lib.dcn_selftest_wait_timeout(10, None) == EINVAL
+    assert lib.dcn_selftest_wait_timeout(5_000_000_000, None) == EINVAL
+    assert "limit_cycles" in lib.dcn_last_error_string().decode()
+
+
 def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     import importlib
     monkeypatch.setattr(dcn, "_lib", None)
