@@ -6,7 +6,7 @@ rebuilt only when a source or header is newer), then linked into
 statically, so the library does not depend on which libcudart a host process
 has already loaded.
 
-    python -m deformable_convolution_dcn_b200.build [--force] [-v]
+    python -m deformable_convolution_dcn_b200.build [--force] [-v] [--nvtx]
 """
 from __future__ import annotations
 
@@ -78,4 +78,6 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, ptxas_verbose="--ptxas" in sys.argv))
+    # --nvtx: rebuild the library with NVTX ranges around its entry points (--force goes back)
+    print(build(force="--force" in sys.argv or "--nvtx" in sys.argv, verbose="-v" in sys.argv,
+                ptxas_verbose="--ptxas" in sys.argv, defines=["DCN_NVTX"] if "--nvtx" in sys.argv else ()))

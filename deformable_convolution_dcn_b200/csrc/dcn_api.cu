@@ -11,6 +11,23 @@
 #include "dcn.h"
 #include "kernels.h"
 
+// Built with -DDCN_NVTX, every entry point that enqueues device work opens an
+// NVTX range named after itself for the duration of the call (host side: the
+// enqueue, not the kernels), so that a timeline tool shows which library call
+// launched which kernels. Header-only; no effect in the default build.
+#ifdef DCN_NVTX
+#include <nvtx3/nvToolsExt.h>
+namespace {
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+};
+}  // namespace
+#define DCN_TRACE(name) NvtxRange dcn_nvtx_range_(name)
+#else
+#define DCN_TRACE(name) ((void)0)
+#endif
+
 namespace {
 
 thread_local std::string g_err;
@@ -170,6 +187,7 @@ const char* dcn_forward_path(const dcn_params_t* params) {
 
 int dcn_forward(const dcn_params_t* params, const void* x, const void* offset, const void* mask, const void* weight,
                 const void* bias, void* y, void* workspace, size_t workspace_bytes, void* stream) {
+    DCN_TRACE("dcn_forward");
     dcn::Shape s;
     TRY(make_shape(params, s));
     size_t es = elem_size(params->dtype);
@@ -217,6 +235,7 @@ int dcn_forward(const dcn_params_t* params, const void* x, const void* offset, c
 
 int dcn_forward_noalloc(const dcn_params_t* params, const void* x, const void* offset, const void* mask,
                         const void* weight, const void* bias, void* y, void* stream) {
+    DCN_TRACE("dcn_forward_noalloc");
     dcn::Shape s;
     TRY(make_shape(params, s));
     size_t es = elem_size(params->dtype);
@@ -248,6 +267,7 @@ int dcn_forward_noalloc(const dcn_params_t* params, const void* x, const void* o
 int dcn_backward_data(const dcn_params_t* params, const void* x, const void* offset, const void* mask,
                       const void* weight, const void* grad_y, float* grad_x, float* grad_offset, float* grad_mask,
                       void* workspace, size_t workspace_bytes, void* stream) {
+    DCN_TRACE("dcn_backward_data");
     dcn::Shape s;
     TRY(make_shape(params, s));
     size_t es = elem_size(params->dtype);
@@ -293,6 +313,7 @@ int dcn_backward_data(const dcn_params_t* params, const void* x, const void* off
 int dcn_backward_input(const dcn_params_t* params, const void* x, const void* offset, const void* mask,
                        const void* weight, const void* grad_y, float* grad_x, void* workspace, size_t workspace_bytes,
                        void* stream) {
+    DCN_TRACE("dcn_backward_input");
     if (!grad_x) return fail(DCN_ERR_INVALID_ARG, "grad_x is NULL");
     return dcn_backward_data(params, x, offset, mask, weight, grad_y, grad_x, nullptr, nullptr, workspace,
                              workspace_bytes, stream);
@@ -301,6 +322,7 @@ int dcn_backward_input(const dcn_params_t* params, const void* x, const void* of
 int dcn_backward_offset_mask(const dcn_params_t* params, const void* x, const void* offset, const void* mask,
                              const void* weight, const void* grad_y, float* grad_offset, float* grad_mask,
                              void* workspace, size_t workspace_bytes, void* stream) {
+    DCN_TRACE("dcn_backward_offset_mask");
     if (!grad_offset) return fail(DCN_ERR_INVALID_ARG, "grad_offset is NULL");
     return dcn_backward_data(params, x, offset, mask, weight, grad_y, nullptr, grad_offset, grad_mask, workspace,
                              workspace_bytes, stream);
@@ -309,6 +331,7 @@ int dcn_backward_offset_mask(const dcn_params_t* params, const void* x, const vo
 int dcn_backward_weight(const dcn_params_t* params, const void* x, const void* offset, const void* mask,
                         const void* grad_y, float* grad_weight, float* grad_bias, void* workspace,
                         size_t workspace_bytes, void* stream) {
+    DCN_TRACE("dcn_backward_weight");
     dcn::Shape s;
     TRY(make_shape(params, s));
     size_t es = elem_size(params->dtype);
@@ -413,6 +436,7 @@ size_t dcn_predict_workspace_size(const dcn_params_t* params) {
 
 int dcn_predict_offset_mask(const dcn_params_t* params, const void* x, const void* w_pred, const void* b_pred,
                             void* offset, void* mask, void* workspace, size_t workspace_bytes, void* stream) {
+    DCN_TRACE("dcn_predict_offset_mask");
     PredPlan pl;
     dcn::Shape s;
     TRY(pred_plan(params, pl, s));
@@ -481,6 +505,7 @@ static int roi_args(const dcn_roi_params_t* p, dcn::RoiArgs& a, const float* roi
 
 int dcn_droi_pool_forward(const dcn_roi_params_t* params, const void* x, const float* rois, const void* offset,
                           const void* mask, void* y, void* stream) {
+    DCN_TRACE("dcn_droi_pool_forward");
     dcn::RoiArgs a;
     TRY(roi_args(params, a, rois));
     const size_t es = elem_size(params->dtype);
@@ -500,6 +525,7 @@ int dcn_droi_pool_forward(const dcn_roi_params_t* params, const void* x, const f
 int dcn_droi_pool_backward(const dcn_roi_params_t* params, const void* x, const float* rois, const void* offset,
                            const void* mask, const void* grad_y, float* grad_x, float* grad_offset, float* grad_mask,
                            void* stream) {
+    DCN_TRACE("dcn_droi_pool_backward");
     dcn::RoiArgs a;
     TRY(roi_args(params, a, rois));
     const size_t es = elem_size(params->dtype);
@@ -528,6 +554,7 @@ int dcn_droi_pool_backward(const dcn_roi_params_t* params, const void* x, const 
 const char* dcn_last_error_string(void) { return g_err.c_str(); }
 
 int dcn_check_status(void) {
+    DCN_TRACE("dcn_check_status");
     cudaError_t e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return cuda_fail(e, "synchronising before the status read");
     unsigned int st = 0;
@@ -538,6 +565,7 @@ int dcn_check_status(void) {
 }
 
 int dcn_selftest_wait_timeout(unsigned long long limit_cycles, void* stream) {
+    DCN_TRACE("dcn_selftest_wait_timeout");
     if (limit_cycles < 1000ull || limit_cycles > 4000000000ull)
         return fail(DCN_ERR_INVALID_ARG, "limit_cycles must be in [1e3, 4e9], got %llu", limit_cycles);
     cudaError_t e = dcn::selftest_wait_timeout((long long)limit_cycles, (cudaStream_t)stream);
