@@ -311,7 +311,6 @@ def run_ours(args):
     torch.cuda.synchronize()
     launches = launches_per_step * args.steps
     barrier(device)
-    clk = clocks.stop()
     dcn.check_status()
     total_ms = t0.elapsed_time(t1)
     fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
@@ -327,12 +326,18 @@ def run_ours(args):
     if do_bwd:
         per["backward_data"] = statistics.mean(bd_ms) / 1e3
         per["backward_weight"] = statistics.mean(bw_ms) / 1e3
-    rl = {k: roofline_entry(wm[k], t, pk, sustained=True) for k, t in per.items()}
-    dominant = max(per, key=per.get)
-    traffic = load_traffic(args.workload, dominant)
-    roof = dict(rl[dominant])
-    roof.update({"kernel": dominant, "traffic": traffic, "peak_source": pk_src + " (sustained bf16, HBM copy)",
-                 "share_of_step": round(per[dominant] / (total_ms / args.steps / 1e3), 3)})
+    # every pass is a sub-millisecond kernel timed inside a step well under a second: burst peak
+    rl = {k: roofline_entry(wm[k], t, pk, sustained=False) for k, t in per.items()}
+    for k in rl:
+        rl[k]["traffic"] = load_traffic(args.workload, k)
+        rl[k]["share_of_step"] = round(per[k] / (total_ms / args.steps / 1e3), 3)
+    roof = dict(rl["forward"])
+    roof.update({"kernel": "forward", "peak_source": pk_src + " (burst bf16, HBM copy)"})
+
+    per_config = None
+    if not args.no_per_config and world == 1:
+        per_config = measure_per_config(args, device, pk, pk_src, rl if do_bwd else None, per)
+    clk = clocks.stop()
 
     e2e = measure_e2e(args, s, host, device, wm) if rank == 0 else None
     cpu = None
@@ -364,6 +369,8 @@ def run_ours(args):
                         "roofline_frac": rl["forward"]["roofline_frac"]},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
         }
+        if per_config is not None:
+            line["per_config"] = per_config
         if dp:
             line["allreduce"] = {"us": round(statistics.mean(ar_ms) * 1e3, 2),
                                  "bytes": int(outs[0]["grad_wb"].numel() * 4)}
@@ -373,13 +380,131 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def load_traffic(workload, kernel):
-    """DRAM bytes per launch from a committed ncu summary, or None."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+def _source_digest(name):
+    import hashlib
     try:
-        return json.load(open(path))[workload][kernel]
+        return hashlib.sha256(open(os.path.join(ROOT, "deformable_convolution_dcn_b200", "csrc", name),
+                                   "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+
+
+def load_traffic(workload, kernel, path=None):
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
+    committed ncu summary profiles/traffic.json, or None: None as well when the
+    kernel's source file has changed since the counters were taken (each entry
+    records the source file and its digest at capture time)."""
+    path = path or os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        e = json.load(open(path))[workload][kernel]
     except Exception:
         return None
+    if isinstance(e, dict):
+        if e.get("sha") != _source_digest(e.get("source", "")):
+            return None
+        return e.get("bytes")
+    return None
+
+
+# The layer shapes timed one by one in the default run, besides the conv4 step:
+# the 224x224 RGB stem (float32; HBM-bound), the conv3 down-sampling layer and
+# the conv5 dilated, grouped layer (bfloat16).
+PER_CONFIG = ("stem", "conv3_s2", "conv5_d2g4", "conv4")
+
+
+def time_forward(w, device, seconds, per_graph=32):
+    """Forward of workload `w` alone: `per_graph` forwards over rotating input
+    sets (every set evicted from L2 before it comes round again) captured in one
+    CUDA graph through the public API, the graph replayed for about `seconds`
+    of device time with CUDA events around every replay. Returns (seconds per
+    forward, launches per forward, replays)."""
+    import torch
+
+    import deformable_convolution_dcn_b200 as dcn
+    from deformable_convolution_dcn_b200 import inputs as gen
+    s = w.shape
+    host = gen.make_inputs(w)
+    elem = host["x"].element_size()
+    set_bytes = sum(t.numel() * t.element_size() for t in host.values() if t is not None) + elem * s.P * s.Cout
+    n_sets = max(2, min(per_graph, math.ceil(3 * L2_BYTES / set_bytes) + 1))
+    sets = [{k: (None if t is None else t.to(device)) for k, t in host.items()} for _ in range(n_sets)]
+    ys = [torch.empty((s.B, s.Ho, s.Wo, s.Cout), dtype=host["x"].dtype, device=device) for _ in range(n_sets)]
+    p = dcn._params(sets[0]["x"], sets[0]["weight"], sets[0]["offset"], s.stride, s.pad, s.dil, False)
+    ws = torch.empty(max(1, dcn.workspace_size(p, dcn.OP_FORWARD)), dtype=torch.uint8, device=device)
+
+    def run(k):
+        d = sets[k % n_sets]
+        dcn.forward(d["x"], d["offset"], d["mask"], d["weight"], d["bias"], s.stride, s.pad, s.dil,
+                    out=ys[k % n_sets], workspace=ws)
+
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        for k in range(n_sets + 3):
+            run(k)
+    torch.cuda.synchronize()
+    dcn.check_status()
+    g = torch.cuda.CUDAGraph()
+    l0 = dcn.launch_count()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(g, stream=stream):
+            for k in range(per_graph):
+                run(k)
+    launches = (dcn.launch_count() - l0) / per_graph
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+        ev[0].record(stream)
+        g.replay()
+        ev[1].record(stream)
+    torch.cuda.synchronize()
+    reps = max(3, min(4000, int(seconds / max(ev[0].elapsed_time(ev[1]) / 1e3, 1e-6))))
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(int(HOLD_CYCLES_PER_STEP * min(reps, 400)))
+        for r in range(reps):
+            evs[r].record(stream)
+            g.replay()
+        evs[reps].record(stream)
+    torch.cuda.synchronize()
+    dcn.check_status()
+    ms = sorted(evs[r].elapsed_time(evs[r + 1]) for r in range(reps))
+    del g
+    return statistics.median(ms) / 1e3 / per_graph, launches, reps
+
+
+def measure_per_config(args, device, pk, pk_src, step_rl, step_per):
+    """Per-layer figures of the default run: each spec layer's forward timed
+    alone (stem, conv3_s2, conv5_d2g4, and conv4 as a cross-check of the step),
+    plus the conv4 backward passes from the timed step, each against its own
+    roofline (burst bf16 peak, measured HBM copy)."""
+    from deformable_convolution_dcn_b200 import inputs as gen
+    out = {"peak_source": pk_src + " (burst bf16, HBM copy)",
+           "timing": "per layer: 32 forwards over rotating input sets in one CUDA graph, replayed for about "
+                     "%.2f s of device time; median replay / 32" % args.config_seconds}
+    for name in PER_CONFIG:
+        w = gen.WORKLOADS[name]
+        s = w.shape
+        elem = 2 if w.dtype == "bf16" else 4
+        wm = work_model(s, elem, mask=w.mask_dist != "none")["forward"]
+        sec, launches, reps = time_forward(w, device, args.config_seconds)
+        e = roofline_entry(wm, sec, pk, sustained=False)
+        e.update({"us": round(sec * 1e6, 2), "tflops": round(wm["flops"] / sec / 1e12, 2),
+                  "gbs": round(wm["bytes"] / sec / 1e9, 1), "flops": wm["flops"], "bytes": wm["bytes"],
+                  "dtype": w.dtype, "workload": w.description, "traffic": load_traffic(name, "forward"),
+                  "launches_per_forward": launches, "replays": reps})
+        out[name + "_forward"] = e
+    if step_rl is not None:
+        for k in ("backward_data", "backward_weight"):
+            out["conv4_" + k] = dict(step_rl[k], us=round(step_per[k] * 1e6, 2))
+        tot = step_per["backward_data"] + step_per["backward_weight"]
+        s = gen.WORKLOADS["conv4"].shape
+        out["conv4_backward"] = {"us": round(tot * 1e6, 2), "tflops": round(2 * s.flops() / tot / 1e12, 2),
+                                 "frac": round(2 * s.flops() / tot / 1e12 / pk["bf16_tflops"], 4),
+                                 "bound": "tensor", "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                                 "what": "backward_data + backward_weight of the conv4 step (two contractions "
+                                         "of the forward's size)"}
+    return out
 
 
 def measure_e2e(args, s, host, device, wm):
@@ -720,6 +845,10 @@ def main(argv=None):
                     help="with several GPUs: data-parallel step (grad_weight and grad_bias all-reduced every step) "
                          "instead of independent replicas")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the per-layer forward timings (stem, conv3_s2, conv5_d2g4) of the default run")
+    ap.add_argument("--config-seconds", type=float, default=0.5,
+                    help="device time spent on each per-layer timing of the default run")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args(argv)
     if args.warmup < 3:

@@ -90,6 +90,7 @@ def _load():
         lib.dcn_droi_pool_backward.argtypes = [RP, vp, vp, vp, vp, vp, fp, fp, fp, vp]
         lib.dcn_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, vp]
         lib.dcn_last_error_string.restype = ctypes.c_char_p
+        lib.dcn_check_status.argtypes = [vp]
         lib.dcn_check_status.restype = ctypes.c_int
         lib.dcn_launch_count.restype = ctypes.c_ulonglong
         lib.dcn_forward_path.argtypes = [P]
@@ -162,8 +163,13 @@ def forward_path(p: Params) -> str:
     return _load().dcn_forward_path(ctypes.byref(p)).decode()
 
 
-def check_status():
-    _check(_load().dcn_check_status())
+def check_status(stream=None):
+    """Waits for `stream` (a torch.cuda.Stream; default: the current stream of
+    the current device) and takes the device status word, raising DcnError
+    (code -4, DCN_ERR_TIMEOUT) if a kernel of the library gave up a bounded wait
+    since the word was last taken. Other streams are not waited for."""
+    s = torch.cuda.current_stream() if stream is None else stream
+    _check(_load().dcn_check_status(ctypes.c_void_p(s.cuda_stream)))
 
 
 def launch_count() -> int:

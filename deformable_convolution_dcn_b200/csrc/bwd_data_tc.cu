@@ -428,15 +428,9 @@ cudaError_t bwd_data_tc(const Shape& s, const void* x, const void* off, const vo
     if (!encode_kmajor(&map_dy, gy, (uint64_t)s.Cout, (uint64_t)s.P, BM) ||
         !encode_kmajor(&map_wt, wt, (uint64_t)s.Cout, (uint64_t)s.KC, NT))
         return cudaErrorInvalidValue;
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static DeviceFlags attr_set;
+    cudaError_t e = max_dynamic_smem_once((const void*)dcn_bwd_data_tc_kernel, 227 * 1024, attr_set);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        e = cudaFuncSetAttribute(dcn_bwd_data_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-        if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
-    }
     int n = 0;
     dim3 tg((s.KC + 31) / 32, (s.Cout + 31) / 32);
     dcn_transpose_kernel<<<tg, dim3(32, 8), 0, st>>>((const bf16*)w, wt, s.Cout, s.KC);

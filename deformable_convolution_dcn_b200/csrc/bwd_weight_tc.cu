@@ -432,15 +432,9 @@ cudaError_t bwd_weight_tc(const Shape& s, const void* x, const void* off, const 
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static DeviceFlags attr_set;
+    cudaError_t e = max_dynamic_smem_once((const void*)dcn_bwd_weight_tc_kernel, 227 * 1024, attr_set);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        e = cudaFuncSetAttribute(dcn_bwd_weight_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-        if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
-    }
     uint4* rec = reinterpret_cast<uint4*>(ws);
     dim3 rg((pl.ppad + 255) / 256, s.G * s.K2);
     dcn_records_kernel<<<rg, 256, 0, st>>>(s, (const bf16*)off, (const bf16*)mask, rec, pl.ppad);

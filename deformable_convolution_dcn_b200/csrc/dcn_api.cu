@@ -553,12 +553,11 @@ int dcn_droi_pool_backward(const dcn_roi_params_t* params, const void* x, const 
 
 const char* dcn_last_error_string(void) { return g_err.c_str(); }
 
-int dcn_check_status(void) {
+int dcn_check_status(void* stream) {
     DCN_TRACE("dcn_check_status");
-    cudaError_t e = cudaDeviceSynchronize();
-    if (e != cudaSuccess) return cuda_fail(e, "synchronising before the status read");
     unsigned int st = 0;
-    e = dcn::read_and_clear_status(&st);
+    cudaError_t e = dcn::read_and_clear_status(&st, (cudaStream_t)stream);
+    g_launches += 1;
     if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
     if (st) return fail(DCN_ERR_TIMEOUT, "a kernel gave up a bounded wait (status 0x%x)", st);
     return ok();

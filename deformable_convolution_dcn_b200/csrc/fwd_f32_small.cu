@@ -224,14 +224,11 @@ cudaError_t launch(const Shape& s, const float* x, const float* off, const float
                    const float* bias, float* y, cudaStream_t st) {
     const int ppb = px_per_block(s);
     const size_t smem = smem_bytes(s, CIN, ppb);
-    static bool attr[64] = {false};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (smem > 48 * 1024 && dev >= 0 && dev < 64 && !attr[dev]) {
-        e = cudaFuncSetAttribute(stem_fwd_kernel<CIN>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    static DeviceFlags attr;
+    cudaError_t e = cudaSuccess;
+    if (smem > 48 * 1024) {
+        e = max_dynamic_smem_once((const void*)stem_fwd_kernel<CIN>, 200 * 1024, attr);
         if (e != cudaSuccess) return e;
-        attr[dev] = true;
     }
     dim3 grid((s.P + ppb - 1) / ppb);
     stem_fwd_kernel<CIN><<<grid, THREADS, smem, st>>>(s, x, off, mask, w, bias, y, ppb);

@@ -312,15 +312,9 @@ cudaError_t launch(const Shape& s, const float* x, const float* off, const float
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    static bool attr[64] = {false};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static DeviceFlags attr;
+    cudaError_t e = max_dynamic_smem_once((const void*)stem_tc_kernel<CIN>, 227 * 1024, attr);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64 && !attr[dev]) {
-        e = cudaFuncSetAttribute(stem_tc_kernel<CIN>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-        if (e != cudaSuccess) return e;
-        attr[dev] = true;
-    }
     Args a;
     a.s = s;
     a.x = x;

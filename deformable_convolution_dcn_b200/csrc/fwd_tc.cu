@@ -1044,15 +1044,9 @@ cudaError_t fwd_tc(const Shape& s, const void* x, const void* off, const void* m
     // one 32-byte load per neighbour slice when every slice start is 32-byte aligned
     const bool wide = s.Cin % 16 == 0 && s.Cg % 16 == 0 && (reinterpret_cast<uintptr_t>(x) & 31) == 0;
     auto kernel = wide ? dcn_fwd_tc_kernel<true> : dcn_fwd_tc_kernel<false>;
-    static bool attr_set[64][2] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static DeviceFlags attr_set[2];
+    cudaError_t e = max_dynamic_smem_once((const void*)kernel, 227 * 1024, attr_set[wide]);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64 && !attr_set[dev][wide]) {
-        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-        if (e != cudaSuccess) return e;
-        attr_set[dev][wide] = true;
-    }
     int* counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + pl.ws_counters_off);
     e = cudaMemsetAsync(counters, 0, (size_t)pl.tiles * sizeof(int), st);
     if (e != cudaSuccess) return e;

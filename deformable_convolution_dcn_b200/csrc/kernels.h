@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stddef.h>
 
+#include <atomic>
+
 #include "common.cuh"
 
 namespace dcn {
@@ -81,6 +83,16 @@ cudaError_t selftest_wait_timeout(long long limit_cycles, cudaStream_t st);
 // status.cu — the device status word that bounded waits report to; SM count.
 int num_sms();
 cudaError_t status_word_ptr(unsigned int** ptr);
-cudaError_t read_and_clear_status(unsigned int* out);
+// Waits for `st`, then atomically takes the status word (leaving 0) and returns it in *out.
+cudaError_t read_and_clear_status(unsigned int* out, cudaStream_t st);
+
+// Per-device "done" flags for one-time host set-up (one per kernel), safe to
+// test and set from several host threads at once.
+struct DeviceFlags {
+    std::atomic<bool> done[64];
+};
+// cudaFuncSetAttribute(func, MaxDynamicSharedMemorySize, bytes) once per device
+// for the current device; later calls return at once. Thread-safe.
+cudaError_t max_dynamic_smem_once(const void* func, int bytes, DeviceFlags& flags);
 
 }  // namespace dcn

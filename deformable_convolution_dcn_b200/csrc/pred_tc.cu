@@ -302,15 +302,9 @@ cudaError_t pred_tc(const Shape& s, const void* x, const void* w, const void* bi
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
-    static bool attr[64] = {false};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static DeviceFlags attr;
+    cudaError_t e = max_dynamic_smem_once((const void*)pred_tc_kernel, 227 * 1024, attr);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64 && !attr[dev]) {
-        e = cudaFuncSetAttribute(pred_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-        if (e != cudaSuccess) return e;
-        attr[dev] = true;
-    }
     PredArgs a;
     a.s = s;
     a.bias = (const bf16*)bias;

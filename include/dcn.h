@@ -60,7 +60,7 @@
 extern "C" {
 #endif
 
-#define DCN_ABI_VERSION 1
+#define DCN_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define DCN_API __attribute__((visibility("default")))
@@ -241,10 +241,16 @@ DCN_API int dcn_droi_pool_backward(const dcn_roi_params_t* params, const void* x
 /* The calling thread's last error message ("" after success). */
 DCN_API const char* dcn_last_error_string(void);
 
-/* Reads and clears the device status word of the current device (synchronises
- * the device). Returns DCN_OK, or DCN_ERR_TIMEOUT if a kernel gave up a bounded
- * wait since the last check. */
-DCN_API int dcn_check_status(void);
+/* Waits for the work enqueued on `stream` so far (and for nothing else: other
+ * streams keep running), then takes the device status word of the current
+ * device, leaving it cleared, with one atomic exchange enqueued on `stream`.
+ * The word collects the bounded-wait timeouts of every kernel of this library
+ * on the device, whichever stream launched it; a kernel still running on
+ * another stream may report after this call. Returns DCN_OK, or
+ * DCN_ERR_TIMEOUT if a kernel gave up a bounded wait since the word was last
+ * taken, or DCN_ERR_CUDA if the stream reported an error. Enqueues one kernel
+ * (counted by dcn_launch_count). */
+DCN_API int dcn_check_status(void* stream);
 
 /* Failure-detection self-test (no counterpart on the pages): enqueues one
  * kernel whose bounded mbarrier wait can never complete, through the same wait

@@ -30,7 +30,7 @@ def test_exports_every_header_symbol(lib):
             "dcn_backward_data", "dcn_workspace_size", "dcn_last_error_string"} <= set(names)
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.dcn_abi_version() == 1
+    assert lib.dcn_abi_version() == 2
 
 
 @pytest.mark.parametrize("H,W,K,stride,pad,dil,expect", [

@@ -63,8 +63,22 @@ def test_committed_traffic_figures_are_read():
         if wl.startswith("_"):
             continue
         for k, v in kernels.items():
-            assert bench.load_traffic(wl, k) == v and v > 0
+            assert v["bytes"] > 0
+            src = os.path.join(ROOT, "deformable_convolution_dcn_b200", "csrc", v["source"])
+            assert os.path.exists(src)
+            # a figure is reported only while its kernel's source is the one it was taken on
+            fresh = v["sha"] == bench._source_digest(v["source"])
+            assert bench.load_traffic(wl, k) == (v["bytes"] if fresh else None)
     assert bench.load_traffic("conv4", "no_such_kernel") is None
+
+
+def test_traffic_of_a_changed_kernel_is_dropped(tmp_path):
+    p = tmp_path / "traffic.json"
+    good = bench._source_digest("fwd_tc.cu")
+    p.write_text(json.dumps({"conv4": {"forward": {"bytes": 123, "source": "fwd_tc.cu", "sha": good},
+                                       "backward_data": {"bytes": 456, "source": "fwd_tc.cu", "sha": "0" * 16}}}))
+    assert bench.load_traffic("conv4", "forward", path=str(p)) == 123
+    assert bench.load_traffic("conv4", "backward_data", path=str(p)) is None
 
 
 def test_arguments_are_checked():
