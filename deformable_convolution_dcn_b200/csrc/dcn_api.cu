@@ -179,7 +179,7 @@ const char* dcn_forward_path(const dcn_params_t* params) {
         g_err = keep;
         return "invalid";
     }
-    if (use_fwd_tc(params, s)) return "tcgen05_gather";
+    if (use_fwd_tc(params, s)) return dcn::fwd_tc_variant(s);
     if (use_fwd_f32_tc(params, s)) return "tcgen05_tf32_split";
     if (use_fwd_small(params, s)) return "f32_small_channels";
     return "generic";

@@ -1,0 +1,405 @@
+// Persistent float32 forward for stem-like layers (Cin <= 3, one group,
+// K*K <= 9, Cout a multiple of 32 up to 128) on tcgen05 tensor cores with split
+// tf32 operands, as in fwd_f32_tc.cu:
+//
+//   Col * W^T  ~=  Col_hi * W_hi^T + Col_hi * W_lo^T + Col_lo * W_hi^T,
+//
+// x_hi the nearest tf32 value of x and x_lo = x - x_hi. Such a layer moves far
+// more bytes (offsets, mask, and above all the float32 output) than it does
+// arithmetic, so the kernel is laid out to keep reads and writes in flight
+// together: one CTA per SM walks its share of the 128-pixel tiles with two A
+// buffers and two TMEM accumulators.
+//
+//   * warps 4-15 (three threads per tile row, each a third of the taps): load
+//     the NEXT tile's offsets and mask into registers, gather the current
+//     tile's modulated samples (bilinear, a neighbour outside the map
+//     contributing zero), split them and write both parts into the tile's A
+//     buffer; one of them issues the tile's twelve kind::tf32 MMAs;
+//   * warps 0-3: read the previous tile's accumulator from TMEM, add the bias,
+//     write the rows into a swizzled staging tile and hand it to TMA tensor
+//     stores, which drain while the next tiles are gathered.
+#include "kernels.h"
+#include "tc_ptx.cuh"
+#include "fwd_common.cuh"
+
+namespace dcn {
+namespace {
+
+constexpr int S_BM = 128;          // output pixels per tile (UMMA M)
+constexpr int S_KP = 32;           // padded contraction depth: one 128-byte swizzle row of float32
+constexpr int S_PARTS = 3;         // gather threads per tile row
+constexpr int S_TAPS_PER_PART = 3;
+constexpr int S_MAX_TAPS = 9;
+constexpr int S_EPI_THREADS = 128;                 // warps 0-3
+constexpr int S_GATHER0 = S_EPI_THREADS;           // first gather thread
+constexpr int S_THREADS = S_EPI_THREADS + S_PARTS * S_BM;
+constexpr int S_MAX_COUT = 128;
+constexpr uint32_t S_TILE = S_BM * 128;            // one [128 x 32] float32 swizzled tile (16 KB)
+constexpr int BAR_GATHER = 1, BAR_EPI = 2;         // named barriers (0 is __syncthreads)
+
+struct StemArgs {
+    Shape s;
+    const float* x;
+    const float* off;
+    const float* mask;
+    const float* w;
+    const float* bias;
+    unsigned* status;
+    int tiles;           // ceil(P / 128)
+    int w_bulk;          // weights 16-byte aligned and a whole number of 16-byte units
+    uint32_t a_off, st_off, b_off, w_off, bias_off, bar_off;
+    int acc_cols;        // columns per accumulator (Cout)
+    int tmem_cols;
+};
+
+__device__ __forceinline__ uint32_t sw_off(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
+
+template <int CIN>
+__global__ void __launch_bounds__(S_THREADS, 1)
+    stem_persistent_kernel(const __grid_constant__ CUtensorMap tmap_y, const StemArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const Shape& s = a.s;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int KC = s.K2 * CIN;
+    const uint32_t bsz = (uint32_t)s.Cout * 128;   // one B tile (hi or lo)
+    float* s_w = reinterpret_cast<float*>(smem + a.w_off);
+    float* s_bias = reinterpret_cast<float*>(smem + a.bias_off);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + a.bar_off);
+    uint64_t* wbar = bars;              // raw weights landed
+    uint64_t* mma_bar = bars + 1;       // [2] the MMAs of the tile in buffer b completed
+    uint64_t* acc_empty = bars + 3;     // [2] the epilogue read accumulator b
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 5);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+    const uint32_t wbytes = (uint32_t)s.Cout * KC * 4;
+    // this CTA's tiles: blockIdx.x, blockIdx.x + gridDim.x, ...
+    const int ntl = a.tiles > (int)blockIdx.x ? (a.tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+
+    if (tid == 0) {
+        ptx::mbar_init(ptx::smem_u32(wbar), 1);
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(ptx::smem_u32(&mma_bar[i]), 1);
+            ptx::mbar_init(ptx::smem_u32(&acc_empty[i]), 4);
+        }
+        *s_abort = 0;
+        ptx::fence_mbar_init();
+        if (a.w_bulk) {
+            ptx::mbar_arrive_expect_tx(ptx::smem_u32(wbar), wbytes);
+            for (uint32_t o = 0; o < wbytes; o += 16384u)
+                ptx::bulk_load(ptx::smem_u32(smem + a.w_off) + o, reinterpret_cast<const uint8_t*>(a.w) + o,
+                               min(16384u, wbytes - o), ptx::smem_u32(wbar));
+        }
+    }
+    if (warp == 0) {
+        ptx::tmem_alloc(ptx::smem_u32(s_tmem), (uint32_t)a.tmem_cols);
+        ptx::tmem_relinquish();
+    }
+    for (int i = tid; i < s.Cout; i += S_THREADS) s_bias[i] = a.bias ? __ldg(a.bias + i) : 0.f;
+
+    // ---- gather threads: this thread's row and taps, and the first tile's offsets in flight
+    const int gt = tid - S_GATHER0;
+    const int row = gt & (S_BM - 1), part = gt >> 7;
+    const int tp_lo = s.K2 * part / S_PARTS, tp_hi = s.K2 * (part + 1) / S_PARTS;
+    const int plane = s.Ho * s.Wo;
+    float cur[3 * S_TAPS_PER_PART], nxt[3 * S_TAPS_PER_PART];
+    // offsets and mask of tile-local row `row` of this CTA's i-th tile, for this thread's taps
+    auto fetch = [&](int i, float (&v)[3 * S_TAPS_PER_PART]) {
+        const int p = ((int)blockIdx.x + i * (int)gridDim.x) * S_BM + row;
+        const bool pv = i < ntl && p < s.P;
+        int bb = 0, pix = 0;
+        if (pv) {
+            bb = p / plane;
+            pix = p - bb * plane;
+        }
+        const float* offp = a.off + (size_t)bb * 2 * s.K2 * plane + pix;
+        const float* mp = a.mask ? a.mask + (size_t)bb * s.K2 * plane + pix : nullptr;
+#pragma unroll
+        for (int j = 0; j < S_TAPS_PER_PART; ++j) {
+            const int t = tp_lo + j;
+            v[3 * j] = v[3 * j + 1] = 0.f;
+            v[3 * j + 2] = 1.f;
+            if (pv && t < tp_hi) {
+                v[3 * j] = __ldg(offp + (size_t)(2 * t) * plane);
+                v[3 * j + 1] = __ldg(offp + (size_t)(2 * t + 1) * plane);
+                if (mp) v[3 * j + 2] = __ldg(mp + (size_t)t * plane);
+            }
+        }
+    };
+    if (gt >= 0) fetch(0, cur);
+
+    // ---- weights into the two B tiles: row n = output channel, k = tap*Cin + c, zero for k >= KC
+    __syncthreads();  // barriers initialised, TMEM allocated, bias staged
+    bool ok = true;
+    if (a.w_bulk) ok = ptx::mbar_wait(ptx::smem_u32(wbar), 0, s_abort, a.status, WAIT_LIMIT);
+    uint8_t* sB = smem + a.b_off;
+    for (int e = tid; e < s.Cout * (S_KP / 4); e += S_THREADS) {
+        const int n = e >> 3, c = e & 7;
+        float v[4], hi[4], lo[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int k = 4 * c + j;
+            v[j] = k >= KC ? 0.f : (a.w_bulk ? s_w[n * KC + k] : __ldg(a.w + (size_t)n * KC + k));
+            hi[j] = ptx::to_tf32(v[j]);
+            lo[j] = v[j] - hi[j];
+        }
+        const uint32_t o = ptx::smem_u32(sB) + sw_off(n, c);
+        ptx::sts_v4(o, make_uint4(__float_as_uint(hi[0]), __float_as_uint(hi[1]), __float_as_uint(hi[2]),
+                                  __float_as_uint(hi[3])));
+        ptx::sts_v4(o + bsz, make_uint4(__float_as_uint(lo[0]), __float_as_uint(lo[1]), __float_as_uint(lo[2]),
+                                        __float_as_uint(lo[3])));
+    }
+    ptx::fence_proxy_async_smem();
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+
+    if (gt >= 0) {
+        // ------------------------------------------------------------ gather --
+        const float* xb0 = a.x;
+        for (int i = 0; i < ntl && ok; ++i) {
+            const int buf = i & 1;
+            const uint32_t arow = ptx::smem_u32(smem + a.a_off) + (uint32_t)buf * 2 * S_TILE + (uint32_t)row * 128;
+            if (i + 1 < ntl) fetch(i + 1, nxt);
+            // the MMAs of tile i - 2 have read this A buffer
+            if (i >= 2 && !ptx::mbar_wait(ptx::smem_u32(&mma_bar[buf]), ((i >> 1) - 1) & 1, s_abort, a.status,
+                                          WAIT_LIMIT)) {
+                ok = false;
+                break;
+            }
+            const int p = ((int)blockIdx.x + i * (int)gridDim.x) * S_BM + row;
+            const bool pv = p < s.P;
+            int bb = 0, oy = 0, ox = 0;
+            if (pv) {
+                bb = p / plane;
+                const int pix = p - bb * plane;
+                const int ho = pix / s.Wo, wo = pix - ho * s.Wo;
+                oy = ho * s.stride - s.pad;
+                ox = wo * s.stride - s.pad;
+            }
+            const float* xb = xb0 + (size_t)bb * s.H * s.W * CIN;
+#pragma unroll
+            for (int j = 0; j < S_TAPS_PER_PART; ++j) {
+                const int t = tp_lo + j;
+                if (t >= tp_hi) break;
+                float col[CIN];
+#pragma unroll
+                for (int c = 0; c < CIN; ++c) col[c] = 0.f;
+                if (pv) {
+                    const int ti = t / s.K, tj = t - ti * s.K;
+                    int y0, x0;
+                    float ly, lx;
+                    split_coord(oy + ti * s.dil, cur[3 * j], y0, ly);
+                    split_coord(ox + tj * s.dil, cur[3 * j + 1], x0, lx);
+                    float wt[4], v[4][CIN];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int r = y0 + (q >> 1), cc = x0 + (q & 1);
+                        wt[q] = 0.f;
+#pragma unroll
+                        for (int c = 0; c < CIN; ++c) v[q][c] = 0.f;
+                        if (!inside(s, r, cc)) continue;
+                        wt[q] = ((q >> 1) ? ly : 1.f - ly) * ((q & 1) ? lx : 1.f - lx) * cur[3 * j + 2];
+                        const float* pc = xb + ((size_t)r * s.W + cc) * CIN;
+#pragma unroll
+                        for (int c = 0; c < CIN; ++c) v[q][c] = __ldg(pc + c);
+                    }
+#pragma unroll
+                    for (int c = 0; c < CIN; ++c)
+                        col[c] = wt[0] * v[0][c] + wt[1] * v[1][c] + wt[2] * v[2][c] + wt[3] * v[3][c];
+                }
+#pragma unroll
+                for (int c = 0; c < CIN; ++c) {
+                    const int k = t * CIN + c;
+                    const float hi = ptx::to_tf32(col[c]);
+                    const uint32_t o = arow + ((((k >> 2) ^ (row & 7)) << 4) | ((k & 3) << 2));
+                    ptx::sts_f32(o, hi);
+                    ptx::sts_f32(o + S_TILE, col[c] - hi);
+                }
+            }
+            if (part == S_PARTS - 1) {
+                for (int k = KC; k < S_KP; ++k) {
+                    const uint32_t o = arow + ((((k >> 2) ^ (row & 7)) << 4) | ((k & 3) << 2));
+                    ptx::sts_f32(o, 0.f);
+                    ptx::sts_f32(o + S_TILE, 0.f);
+                }
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::tc_fence_before();
+            ptx::bar_sync_named(BAR_GATHER, S_PARTS * S_BM);
+            if (gt == 0) {
+                // accumulator `buf` was read by the epilogue of tile i - 2
+                if (i >= 2 && !ptx::mbar_wait(ptx::smem_u32(&acc_empty[buf]), ((i >> 1) - 1) & 1, s_abort, a.status,
+                                              WAIT_LIMIT)) {
+                    ok = false;
+                } else {
+                    ptx::tc_fence_after();
+                    const uint32_t idesc = ptx::idesc_tf32_f32(S_BM, s.Cout);
+                    const uint32_t a0 = arow - (uint32_t)row * 128, b0 = ptx::smem_u32(sB);
+                    const uint32_t d = tmem + (uint32_t)(buf * a.acc_cols);
+                    // small terms first; each K step of 8 tf32 is 32 bytes along the swizzled row
+#pragma unroll
+                    for (int kk = 0; kk < S_KP / 8; ++kk)
+                        ptx::mma_tf32(d, ptx::sw128_desc(a0 + S_TILE + kk * 32), ptx::sw128_desc(b0 + kk * 32), idesc,
+                                      kk > 0 ? 1u : 0u);
+#pragma unroll
+                    for (int kk = 0; kk < S_KP / 8; ++kk)
+                        ptx::mma_tf32(d, ptx::sw128_desc(a0 + kk * 32), ptx::sw128_desc(b0 + bsz + kk * 32), idesc,
+                                      1u);
+#pragma unroll
+                    for (int kk = 0; kk < S_KP / 8; ++kk)
+                        ptx::mma_tf32(d, ptx::sw128_desc(a0 + kk * 32), ptx::sw128_desc(b0 + kk * 32), idesc, 1u);
+                    ptx::mma_commit(ptx::smem_u32(&mma_bar[buf]));
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 3 * S_TAPS_PER_PART; ++j) cur[j] = nxt[j];
+        }
+    } else {
+        // ---------------------------------------------------------- epilogue --
+        const uint32_t taddr0 = tmem + ((uint32_t)(warp * 32) << 16);
+        const uint32_t stg = ptx::smem_u32(smem + a.st_off);
+        for (int i = 0; i < ntl && ok; ++i) {
+            const int buf = i & 1;
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(ptx::smem_u32(&mma_bar[buf]), (i >> 1) & 1, s_abort, a.status,
+                                                        WAIT_LIMIT))) {
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after();
+            // the previous tile's stores have finished reading the staging tile
+            if (tid == 0) ptx::bulk_wait_group_read0();
+            ptx::bar_sync_named(BAR_EPI, S_EPI_THREADS);
+            for (int cb = 0; cb < s.Cout / 32; ++cb) {
+                float v[32];
+                ptx::tmem_ld32(taddr0 + (uint32_t)(buf * a.acc_cols) + cb * 32, v);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] += s_bias[cb * 32 + j];
+                const uint32_t o = stg + cb * S_TILE;
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    ptx::sts_v4(o + sw_off(tid, c), make_uint4(__float_as_uint(v[4 * c]), __float_as_uint(v[4 * c + 1]),
+                                                               __float_as_uint(v[4 * c + 2]),
+                                                               __float_as_uint(v[4 * c + 3])));
+            }
+            // accumulator `buf` is free for the tile after next
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&acc_empty[buf]));
+            ptx::fence_proxy_async_smem();
+            ptx::bar_sync_named(BAR_EPI, S_EPI_THREADS);
+            if (tid == 0) {
+                const int tile = (int)blockIdx.x + i * (int)gridDim.x;
+                for (int cb = 0; cb < s.Cout / 32; ++cb)
+                    ptx::tma_store_2d(&tmap_y, stg + cb * S_TILE, cb * 32, tile * S_BM);
+                ptx::bulk_commit_group();
+            }
+        }
+        if (tid == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");  // stores complete
+    }
+
+    // ------------------------------------------------------------ teardown --
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (!ok && tid == 0) {
+        // MMAs may still be in flight: let them finish (bounded) before TMEM is released
+        volatile int dummy = 0;
+        for (int b = 0; b < 2; ++b) {
+            const int last = ((ntl - 1 - b) >= 0) ? (ntl - 1 - b) : -1;
+            if (last >= 0) ptx::mbar_wait(ptx::smem_u32(&mma_bar[last & 1]), (last >> 1) & 1, &dummy, nullptr,
+                                          WAIT_LIMIT);
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, (uint32_t)a.tmem_cols);
+    }
+}
+
+struct StemPlan {
+    uint32_t a_off, st_off, b_off, w_off, bias_off, bar_off, smem_bytes;
+    int tmem_cols;
+};
+
+StemPlan make_stem_plan(const Shape& s) {
+    StemPlan pl;
+    pl.a_off = 0;                                              // two buffers of (hi, lo) A tiles
+    pl.st_off = 4 * S_TILE;                                    // output staging: Cout / 32 tiles
+    pl.b_off = pl.st_off + (uint32_t)(s.Cout / 32) * S_TILE;   // B hi, lo
+    pl.w_off = pl.b_off + 2u * (uint32_t)s.Cout * 128;
+    pl.bias_off = pl.w_off + (((uint32_t)s.Cout * s.K2 * s.Cin * 4 + 15) & ~15u);
+    pl.bar_off = pl.bias_off + (uint32_t)s.Cout * 4;
+    pl.smem_bytes = pl.bar_off + 64 + 1024;
+    int cols = 32;
+    while (cols < 2 * s.Cout) cols *= 2;
+    pl.tmem_cols = cols;
+    return pl;
+}
+
+template <int CIN>
+cudaError_t launch_stem(const Shape& s, const float* x, const float* off, const float* mask, const float* w,
+                        const float* bias, float* y, unsigned* status, cudaStream_t st) {
+    const StemPlan pl = make_stem_plan(s);
+    auto encode = get_encode();
+    if (!encode) return cudaErrorNotSupported;
+    CUtensorMap map;
+    cuuint64_t dims[2] = {(cuuint64_t)s.Cout, (cuuint64_t)s.P};
+    cuuint64_t strides[1] = {(cuuint64_t)s.Cout * 4};
+    cuuint32_t box[2] = {32, (cuuint32_t)S_BM};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, y, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    static DeviceFlags attr;
+    cudaError_t e = max_dynamic_smem_once((const void*)stem_persistent_kernel<CIN>, 227 * 1024, attr);
+    if (e != cudaSuccess) return e;
+    StemArgs a;
+    a.s = s;
+    a.x = x;
+    a.off = off;
+    a.mask = mask;
+    a.w = w;
+    a.bias = bias;
+    a.status = status;
+    a.tiles = (s.P + S_BM - 1) / S_BM;
+    a.w_bulk = ((reinterpret_cast<uintptr_t>(w) & 15) == 0 && ((size_t)s.Cout * s.K2 * s.Cin * 4) % 16 == 0) ? 1 : 0;
+    a.a_off = pl.a_off;
+    a.st_off = pl.st_off;
+    a.b_off = pl.b_off;
+    a.w_off = pl.w_off;
+    a.bias_off = pl.bias_off;
+    a.bar_off = pl.bar_off;
+    a.acc_cols = s.Cout;
+    a.tmem_cols = pl.tmem_cols;
+    const int grid = std::min(a.tiles, num_sms());
+    stem_persistent_kernel<CIN><<<grid, S_THREADS, pl.smem_bytes, st>>>(map, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// Cin <= 3 with one group, K*K <= 9, Cout a multiple of 32 up to 128, and index
+// ranges within 32 bits (y 16-byte aligned: TMA stores).
+bool fwd_f32_stem_supported(const Shape& s) {
+    if (s.Cin > 3 || s.G != 1 || s.K2 > S_MAX_TAPS || s.K2 * s.Cin > S_KP) return false;
+    if (s.Cout % 32 || s.Cout < 32 || s.Cout > S_MAX_COUT) return false;
+    if ((long long)s.B * 2 * s.K2 * s.Ho * s.Wo >= (1LL << 31) || (long long)s.B * s.H * s.W * s.Cin >= (1LL << 31))
+        return false;
+    return make_stem_plan(s).smem_bytes <= 227 * 1024;
+}
+
+cudaError_t fwd_f32_stem(const Shape& s, const void* x, const void* off, const void* mask, const void* w,
+                         const void* bias, void* y, unsigned* status, cudaStream_t st) {
+    const float *xf = (const float*)x, *of = (const float*)off, *mf = (const float*)mask, *wf = (const float*)w,
+                *bf = (const float*)bias;
+    float* yf = (float*)y;
+    switch (s.Cin) {
+        case 1: return launch_stem<1>(s, xf, of, mf, wf, bf, yf, status, st);
+        case 2: return launch_stem<2>(s, xf, of, mf, wf, bf, yf, status, st);
+        default: return launch_stem<3>(s, xf, of, mf, wf, bf, yf, status, st);
+    }
+}
+
+}  // namespace dcn

@@ -1,0 +1,677 @@
+// Forward DCNv2 on sm_100a tensor cores, bfloat16 in / float32 accumulate, with
+// the gathered operand in tensor memory (layers with Cout <= 256).
+//
+// Y[P x Cout] = Col[P x K*K*Cin] * W^T as in fwd_tc.cu (the im2col view of the
+// deformable convolution: the "Deformable ConvNets" notes, im2col appendix and
+// the y(p0) equations), but the producers write each gathered A chunk (128
+// output pixels x 64 channels of one tap) into TMEM with tcgen05.st, and the
+// MMA reads A from TMEM (tcgen05.mma ... [a-tmem], b-desc). The gathered tile
+// never passes through shared memory: shared memory holds only the weight ring,
+// the sampling records and the epilogue's staging, which leaves the rest of the
+// SM's 256 KB to the L1 cache the gather hits in, and no shared-memory
+// bandwidth goes to writing A or to the tensor cores reading it.
+//
+//   * 8 producer warps, two per TMEM lane quarter (a warp may only reach the
+//     32 lanes of its index mod 4). Each warp owns 16 rows (pixels) of every
+//     chunk; lane l gathers row (l / 4) and row (l / 4) + 8, 16 channels
+//     (32 bytes) of each, l % 4 picking which 16 of the chunk's 64. The blended
+//     rows go to TMEM with one tcgen05.st.16x256b.x4, whose fixed thread-to-
+//     column map places channel c = 16j + 4n + e (j = l % 4) at K position
+//     k = 16n + 4j + e of the chunk. The weights are read in that same order:
+//     a pre-pass permutes W = [Cout, K*K*Cin] into the workspace as
+//     W' = [Cout, units x 64], unit u's 64 columns in K order k (zero where the
+//     group has no channel), so the product sums the same terms.
+//   * 1 TMA warp loads the [N x 64] tiles of W' into a shared-memory ring.
+//   * 1 MMA warp issues tcgen05.mma.kind::f16 (M=128, N=Cout tile, K=16) with A
+//     from TMEM into a TMEM accumulator, and commits each stage's release.
+//   * 4 epilogue warps build the sampling records one (tile, group) epoch ahead
+//     and read the accumulator back (stream-K combine as in fwd_tc.cu).
+//
+// TMEM (512 columns): accumulators at column 0 (one of <= 256 columns, or two
+// of <= 128), the A ring of 8 stages x 32 columns at column 256.
+#include "fwd_common.cuh"
+
+namespace dcn {
+namespace {
+
+constexpr int NUM_PROD_WARPS = 8;
+constexpr int TMA_WARP = 4, MMA_WARP = 5, PROD_WARP0 = 6;  // warps 0-3: records and epilogue
+constexpr int NUM_THREADS = (PROD_WARP0 + NUM_PROD_WARPS) * 32;
+constexpr int A_STAGES = 8;                  // TMEM A ring
+constexpr int A_COL = 256;                   // first TMEM column of the A ring
+constexpr int A_STAGE_COLS = BK / 2;         // 64 bf16 per row = 32 columns
+constexpr int MAX_B_STAGES = 4;
+constexpr int SLICE_CH = 16;                 // channels one lane gathers per sample (32 bytes)
+#ifndef DCN_FWD_TS_B_STAGES
+#define DCN_FWD_TS_B_STAGES 3
+#endif
+
+// Sixteen 32-bit registers per thread into 16 TMEM lanes x 32 columns
+// (16x256b shape, 4 repetitions): thread t writes lanes t/4 and t/4 + 8,
+// columns 8n + 2(t%4) and 8n + 2(t%4) + 1 of repetition n.
+__device__ __forceinline__ void tmem_st_16x256b_x4(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x256b.x4.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, bf16 x bf16 -> f32 (A read from TMEM lanes 0..127).
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+struct TsArgs {
+    FwdArgs f;
+    int b_stages;
+    uint32_t idle_bytes;  // shared memory free after the last MMA (the weight ring)
+};
+
+// ------------------------------------------------------------ pre-pass --
+// W' [Cout][U*64] from W [Cout][K*K*Cin]: unit u = (g, q, tap) (taps innermost),
+// K position k of the unit holds channel c = 16*((k >> 2) & 3) + 4*(k >> 4) + (k & 3)
+// of chunk q of group g at tap `tap` (zero past the group's channels). One
+// thread per 8 outputs (16 bytes); also clears the stream-K tile counters.
+__global__ void __launch_bounds__(256) dcn_wperm_kernel(const bf16* __restrict__ w, bf16* __restrict__ wp, Shape s,
+                                                        int nq, int U, int* counters, int tiles) {
+    const long long n8 = (long long)s.Cout * U * 8;
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < tiles) counters[i] = 0;
+    if (i >= n8) return;
+    const int k8 = (int)(i & 7);
+    const long long ou = i >> 3;
+    const int u = (int)(ou % U);
+    const int o = (int)(ou / U);
+    const int g = u / (nq * s.K2), q = (u / s.K2) % nq, tap = u % s.K2;
+    uint2 v[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int kb = 2 * k8 + h;                  // 4-element block of k
+        const int c = 16 * (kb & 3) + 4 * (kb >> 2);  // its first channel within the chunk
+        const int cg = q * BK + c;
+        v[h] = make_uint2(0u, 0u);
+        if (cg < s.Cg)
+            v[h] = *reinterpret_cast<const uint2*>(w + (size_t)o * s.KC + (size_t)tap * s.Cin + (size_t)g * s.Cg + cg);
+    }
+    *reinterpret_cast<uint4*>(wp + ((size_t)o * U + u) * BK + 8 * k8) = make_uint4(v[0].x, v[0].y, v[1].x, v[1].y);
+}
+
+// --------------------------------------------------------------- kernel --
+// WIDE: x is 32-byte aligned and Cin, Cg are multiples of 16, so a lane's
+// 16-channel slice is one 32-byte load.
+template <bool WIDE>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    dcn_fwd_ts_kernel(const __grid_constant__ CUtensorMap tmap_w, const TsArgs ta) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const FwdArgs& a = ta.f;
+    const Shape& s = a.s;
+
+    uint8_t* sB = smem;  // weight ring: b_stages x [N x 128 B], 128-byte swizzle
+    TapRec* s_rec = reinterpret_cast<TapRec*>(smem + a.info_off);  // two buffers of BM * K2 records
+    int2* s_tap = reinterpret_cast<int2*>(smem + a.row_off);        // per tap: (i*dil, j*dil)
+    long long* s_starts = reinterpret_cast<long long*>(s_tap + 32);   // [ctas + 1] first unit of each CTA
+    float* s_bias = reinterpret_cast<float*>(s_starts + MAX_CTAS + 2);  // [2][512] bias of a tile's columns
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + a.bar_off);
+    uint64_t* a_full = bars;                      // [A_STAGES] every producer warp stored the chunk
+    uint64_t* a_empty = a_full + A_STAGES;        // [A_STAGES] the MMAs reading the stage completed
+    uint64_t* b_full = a_empty + A_STAGES;        // [MAX_B_STAGES] weight tile landed
+    uint64_t* b_empty = b_full + MAX_B_STAGES;    // [MAX_B_STAGES] the MMAs reading it completed
+    uint64_t* acc_full = b_empty + MAX_B_STAGES;  // [2]
+    uint64_t* acc_empty = acc_full + 2;           // [2]
+    uint64_t* drain = acc_empty + 2;
+    uint64_t* tail_bar = drain + 1;               // bulk copy of other CTAs' partials for the last segment
+    uint64_t* rec_full = tail_bar + 1;            // [2] records of an epoch built
+    uint64_t* rec_empty = rec_full + 2;           // [2] every producer warp done with an epoch's records
+    uint64_t* rec0_bar = rec_empty + 2;           // the first epoch's records, built by all warps
+    uint64_t* epi_bar = rec0_bar + 1;
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(epi_bar + 1);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+    volatile int* s_last = s_abort + 1;  // [2], by segment parity
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < A_STAGES; ++i) {
+            ptx::mbar_init(ptx::smem_u32(&a_full[i]), NUM_PROD_WARPS);
+            ptx::mbar_init(ptx::smem_u32(&a_empty[i]), 1);
+        }
+        for (int i = 0; i < MAX_B_STAGES; ++i) {
+            ptx::mbar_init(ptx::smem_u32(&b_full[i]), 1);
+            ptx::mbar_init(ptx::smem_u32(&b_empty[i]), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(ptx::smem_u32(&acc_full[i]), 1);
+            ptx::mbar_init(ptx::smem_u32(&acc_empty[i]), 4);
+        }
+        ptx::mbar_init(ptx::smem_u32(drain), 1);
+        ptx::mbar_init(ptx::smem_u32(tail_bar), 1);
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(ptx::smem_u32(&rec_full[i]), 4);
+            ptx::mbar_init(ptx::smem_u32(&rec_empty[i]), NUM_PROD_WARPS);
+        }
+        ptx::mbar_init(ptx::smem_u32(rec0_bar), NUM_PROD_WARPS + 4);
+        ptx::mbar_init(ptx::smem_u32(epi_bar), 4);
+        *s_abort = 0;
+        s_last[0] = s_last[1] = 0;
+        ptx::fence_mbar_init();
+    }
+    if (threadIdx.x < s.K2) {
+        const int i = threadIdx.x / s.K;
+        s_tap[threadIdx.x] = make_int2(i * s.dil, (threadIdx.x - i * s.K) * s.dil);
+    }
+    for (int c = threadIdx.x; c <= a.ctas; c += NUM_THREADS) s_starts[c] = unit_begin(c, a);
+    if (warp == MMA_WARP) {
+        ptx::tmem_alloc(ptx::smem_u32(s_tmem), 512u);
+        ptx::tmem_relinquish();
+    }
+    if (warp == TMA_WARP && lane == 0) ptx::prefetch_tmap(&tmap_w);
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = *s_tmem;
+
+    const int cta = blockIdx.x;
+    const long long ubeg = s_starts[cta], uend = s_starts[cta + 1];
+    const SegList L = seg_list(ubeg, uend, a.U);
+    if (warp >= PROD_WARP0) {
+        // ------------------------------------------------------ producers --
+        const int ptid = threadIdx.x - PROD_WARP0 * 32;
+        const int rb = 32 * (warp & 3) + 16 * ((warp - PROD_WARP0) >> 2);  // this warp's 16 TMEM lanes (rows)
+        const int j4 = lane & 3;
+        const int r0 = rb + (lane >> 2), r1 = r0 + 8;
+        const uint32_t t_row = tmem_base + ((uint32_t)rb << 16) + (uint32_t)A_COL;
+        const long long cin2 = (long long)s.Cin * 2, rp2 = (long long)s.W * cin2;
+        const uint8_t* zb = reinterpret_cast<const uint8_t*>(g_zero_slice);
+        bool ok = true;
+        // the first epoch's records are built by all warps together
+        if (L.ns > 0) {
+            const Seg s0 = seg_at(L, 0);
+            build_records(a, s0.t / a.n_tiles, s0.k0 / (a.nq * s.K2), ptid & (BM - 1), 1 + (ptid >> 7), s_rec, s_tap);
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(rec0_bar));
+            ok = __all_sync(0xffffffffu, ptx::mbar_wait(ptx::smem_u32(rec0_bar), 0, s_abort, a.status, WAIT_LIMIT));
+        }
+        int isi = 0, ik = 0, ik1 = 0, icur_g = -1, iepoch = 0;
+        Chunk ich{0, 0, 0};
+        const TapRec* irecs = s_rec;
+        if (L.ns > 0) {
+            const Seg s0 = seg_at(L, 0);
+            ik = s0.k0;
+            ik1 = s0.k1;
+            ich = chunk_of(ik, a);
+            icur_g = ich.g;
+        }
+        // loads of row `row` of the cursor chunk into v, its weights into w
+        auto issue = [&](uint32_t(&v)[4][8], uint32_t(&w)[2], int row) {
+            const int cg = ich.q * BK + j4 * SLICE_CH;
+            const uint32_t cmask = cg < s.Cg ? 0xFu : 0u;
+            const bool hi_ok = cg + 8 < s.Cg;  // upper 8 channels present (narrow loads only)
+            const uint8_t* xc = reinterpret_cast<const uint8_t*>(a.x + ich.g * s.Cg + cg);
+            const TapRec rc = irecs[row * s.K2 + ich.tap];
+            w[0] = rc.w01_00;
+            w[1] = rc.w11_10;
+            const uint32_t vm = rc.vmask & cmask;
+            const uint8_t* p = xc + (long long)rc.base * cin2;
+            const uint8_t* pc[4] = {p, p + cin2, p + rp2, p + rp2 + cin2};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const bool rd = (vm >> c) & 1u;
+                load_slice<WIDE>(v[c], rd ? pc[c] : zb, (rd && hi_ok) ? pc[c] + 16 : zb);
+            }
+        };
+        auto advance = [&]() -> bool {
+            ++ik;
+            if (++ich.tap == s.K2) {
+                ich.tap = 0;
+                if (++ich.q == a.nq) {
+                    ich.q = 0;
+                    ++ich.g;
+                }
+            }
+            if (ik == ik1) {
+                const Seg sn = seg_at(L, ++isi);
+                ik = sn.k0;
+                ik1 = sn.k1;
+                ich = chunk_of(ik, a);
+                icur_g = -1;
+            }
+            if (ich.g != icur_g) {
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&rec_empty[iepoch & 1]));
+                ++iepoch;
+                const int b = iepoch & 1;
+                const uint32_t par = (uint32_t)(b ? (iepoch >> 1) : ((iepoch >> 1) - 1)) & 1u;
+                // warp-uniform outcome: the tcgen05.st below is warp-collective
+                if (!__all_sync(0xffffffffu, ptx::mbar_wait(ptx::smem_u32(&rec_full[b]), par, s_abort, a.status,
+                                                            WAIT_LIMIT)))
+                    return false;
+                irecs = s_rec + b * BM * s.K2;
+                icur_g = ich.g;
+            }
+            return true;
+        };
+        const long long total = uend - ubeg;  // chunks of this CTA
+        uint32_t va[4][8], vb[4][8], wa[2], wb[2];
+        if (ok && total > 0) {
+            issue(va, wa, r0);
+            issue(vb, wb, r1);
+        }
+        int stage = 0, prev = -1;
+        uint32_t phase = 0;
+        for (long long n = 0; n < total && ok; ++n) {
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(ptx::smem_u32(&a_empty[stage]), phase ^ 1, s_abort, a.status,
+                                                        WAIT_LIMIT))) {
+                ok = false;
+                break;
+            }
+            const bool more = n + 1 < total;
+            uint32_t r[16];
+            {
+                uint32_t t[8];
+                blend16(t, va, wa[0], wa[1]);
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    r[4 * m] = t[2 * m];
+                    r[4 * m + 1] = t[2 * m + 1];
+                }
+            }
+            if (more) {
+                if (!advance()) {
+                    ok = false;
+                    break;
+                }
+                issue(va, wa, r0);
+            }
+            {
+                uint32_t t[8];
+                blend16(t, vb, wb[0], wb[1]);
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    r[4 * m + 2] = t[2 * m];
+                    r[4 * m + 3] = t[2 * m + 1];
+                }
+            }
+            if (more) issue(vb, wb, r1);
+            // the previous chunk's store has had this chunk's blend to land: publish it
+            if (prev >= 0) {
+                tmem_wait_st();
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&a_full[prev]));
+            }
+            tmem_st_16x256b_x4(t_row + (uint32_t)(stage * A_STAGE_COLS), r);
+            prev = stage;
+            if (++stage == A_STAGES) {
+                stage = 0;
+                phase ^= 1;
+            }
+        }
+        tmem_wait_st();
+        if (ok && prev >= 0) {
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&a_full[prev]));
+        }
+    } else if (warp == TMA_WARP) {
+        // ------------------------------------------------------- weights --
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued = 0, issued_par = 0;  // per stage: a load was issued / parity of the last one
+            const uint32_t bytes = (uint32_t)(a.box_rows * BK * 2);
+            bool ok = true;
+            for (int si = 0; si < L.ns && ok; ++si) {
+                const Seg sg = seg_at(L, si);
+                const int n0 = (sg.t % a.n_tiles) * a.bn_total;
+                for (int k = sg.k0; k < sg.k1; ++k) {
+                    if (!ptx::mbar_wait(ptx::smem_u32(&b_empty[stage]), phase ^ 1, s_abort, a.status, WAIT_LIMIT)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = ptx::smem_u32(&b_full[stage]);
+                    ptx::mbar_arrive_expect_tx(fb, bytes);
+                    ptx::tma_load_2d(ptx::smem_u32(sB + stage * a.b_stage_bytes), &tmap_w, fb, k * BK, n0);
+                    issued |= 1u << stage;
+                    issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+                    if (++stage == ta.b_stages) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+            if (*s_abort) {
+                // wait (bounded) for loads still in flight before shared memory is released
+                volatile int dummy = 0;
+                for (int i = 0; i < ta.b_stages; ++i)
+                    if ((issued >> i) & 1u)
+                        ptx::mbar_wait(ptx::smem_u32(&b_full[i]), (issued_par >> i) & 1u, &dummy, nullptr,
+                                       WAIT_LIMIT);
+            }
+        }
+        __syncwarp();
+    } else if (warp == MMA_WARP) {
+        // ----------------------------------------------------------- MMA --
+        if (lane == 0) {
+            int as = 0, bs = 0;
+            uint32_t aph = 0, bph = 0;
+            const uint32_t idesc = ptx::idesc_bf16_f32(BM, a.bn_total);
+            const uint32_t b0 = ptx::smem_u32(sB);
+            bool ok = true;
+            for (int seg = 0; seg < L.ns && ok; ++seg) {
+                const Seg sg = seg_at(L, seg);
+                const int abuf = a.acc_cols ? (seg & 1) : 0;
+                const uint32_t accph = a.acc_cols ? ((seg >> 1) & 1) : (seg & 1);
+                if (!ptx::mbar_wait(ptx::smem_u32(&acc_empty[abuf]), accph ^ 1, s_abort, a.status, WAIT_LIMIT)) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                const uint32_t d = tmem_base + (uint32_t)(abuf * a.acc_cols);
+                for (int k = sg.k0; k < sg.k1; ++k) {
+                    if (!ptx::mbar_wait(ptx::smem_u32(&a_full[as]), aph, s_abort, a.status, WAIT_LIMIT) ||
+                        !ptx::mbar_wait(ptx::smem_u32(&b_full[bs]), bph, s_abort, a.status, WAIT_LIMIT)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t at = tmem_base + (uint32_t)(A_COL + as * A_STAGE_COLS);
+                    const uint32_t bsm = b0 + bs * a.b_stage_bytes;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        mma_bf16_ts(d, at + kk * 8, ptx::sw128_desc(bsm + kk * 32), idesc,
+                                    (k > sg.k0 || kk > 0) ? 1u : 0u);
+                    ptx::mma_commit(ptx::smem_u32(&a_empty[as]));
+                    ptx::mma_commit(ptx::smem_u32(&b_empty[bs]));
+                    if (++as == A_STAGES) {
+                        as = 0;
+                        aph ^= 1;
+                    }
+                    if (++bs == ta.b_stages) {
+                        bs = 0;
+                        bph ^= 1;
+                    }
+                }
+                if (!ok) break;
+                ptx::mma_commit(ptx::smem_u32(&acc_full[abuf]));
+            }
+            // all MMAs issued by this thread complete before TMEM is released
+            ptx::mma_commit(ptx::smem_u32(drain));
+            volatile int dummy = 0;
+            ptx::mbar_wait(ptx::smem_u32(drain), 0, &dummy, a.status, WAIT_LIMIT);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------- records and epilogue --
+        // As in fwd_tc.cu: the records are built one epoch ahead of the
+        // producers in two buffers; building epoch e waits only for the
+        // producers to release epoch e - 2, which needs no epilogue of this
+        // segment, so the order cannot deadlock.
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const int per_g = a.nq * s.K2;
+        uint32_t ephase = 0;
+        int rec_epoch = 0;
+        int rseg = 0, rk = L.ns > 0 ? seg_at(L, 0).k0 : 0;
+        bool ok = true;
+        for (int seg = 0; seg < L.ns && ok; ++seg) {
+            const Seg sg = seg_at(L, seg);
+            const int t = sg.t;
+            while (rseg < L.ns && (rseg <= seg || (rseg == seg + 1 && rk == seg_at(L, rseg).k0))) {
+                const Seg rs = seg_at(L, rseg);
+                const int b = rec_epoch & 1;
+                if (rec_epoch >= 2 && !ptx::mbar_wait(ptx::smem_u32(&rec_empty[b]), ((rec_epoch - 2) >> 1) & 1, s_abort,
+                                                      a.status, WAIT_LIMIT)) {
+                    ok = false;
+                    break;
+                }
+                const int rg = rk / per_g;
+                build_records(a, rs.t / a.n_tiles, rg, row, rec_epoch == 0 ? 0 : -1, s_rec + b * BM * s.K2, s_tap);
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(rec_epoch == 0 ? rec0_bar : &rec_full[b]));
+                rk = min((rg + 1) * per_g, rs.k1);
+                if (rk >= rs.k1 && ++rseg < L.ns) rk = seg_at(L, rseg).k0;
+                ++rec_epoch;
+            }
+            if (!ok) break;
+
+            const int abuf = a.acc_cols ? (seg & 1) : 0;
+            const uint32_t accph = a.acc_cols ? ((seg >> 1) & 1) : (seg & 1);
+            const bool full = (sg.k0 == 0 && sg.k1 == a.U);
+            const bool last_proc = seg == L.ns - 1;  // the pipeline is idle after this segment's accumulator
+            const long long tu0 = (long long)t * a.U;
+            int c_lo = cta, c_hi = cta;
+            if (!full) {
+                c_lo = cta_of_unit(tu0, s_starts, a.ctas);
+                c_hi = cta_of_unit(tu0 + a.U - 1, s_starts, a.ctas);
+            }
+            int cnt = -1;
+            if (!full && threadIdx.x == 0) cnt = ptx::ld_relaxed_gpu(a.counters + t);
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(ptx::smem_u32(&acc_full[abuf]), accph, s_abort, a.status,
+                                                        WAIT_LIMIT))) {
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after();
+            const int mt = t / a.n_tiles, n0 = (t % a.n_tiles) * a.bn_total;
+            const int ncols = min(a.bn_total, s.Cout - n0);
+            if (threadIdx.x == 0) {
+                int last = full ? 1 : 0;
+                if (!full) {
+                    if (cnt != c_hi - c_lo && last_proc) cnt = ptx::ld_relaxed_gpu(a.counters + t);
+                    last = cnt == c_hi - c_lo;
+                    if (last) ptx::fence_acq_rel_gpu();  // the partials read below follow the counter
+                }
+                s_last[seg & 1] = last;
+            }
+            float* sbias = s_bias + (seg & 1) * 512;
+            if (a.bias)
+                for (int i = threadIdx.x; i < ncols; i += 4 * 32) sbias[i] = __bfloat162float(a.bias[n0 + i]);
+            if (!epi_sync(epi_bar, ephase, s_abort, a.status)) {
+                ok = false;
+                break;
+            }
+            const float* sb = a.bias ? sbias : nullptr;
+            const int p = strip_to_raster(mt * BM + row, a);
+            const uint32_t taddr = tmem_base + (uint32_t)(abuf * a.acc_cols) + ((uint32_t)(quarter * 32) << 16);
+            bf16* ycol0 = a.y + n0;
+            if (s_last[seg & 1]) {
+                const uint32_t tile_bytes = (uint32_t)BM * a.bn_total * 4;
+                const bool staged = !full && last_proc && (uint32_t)(c_hi - c_lo) * tile_bytes <= ta.idle_bytes;
+                if (staged) {
+                    if (threadIdx.x == 0) {
+                        ptx::fence_proxy_async_all();
+                        const uint32_t tb = ptx::smem_u32(tail_bar);
+                        ptx::mbar_arrive_expect_tx(tb, (uint32_t)(c_hi - c_lo) * tile_bytes);
+                        uint32_t dst = ptx::smem_u32(smem);
+                        for (int c = c_lo; c <= c_hi; ++c) {
+                            if (c == cta) continue;
+                            const uint8_t* src = reinterpret_cast<const uint8_t*>(partial_base(a, s_starts, c, tu0, 0));
+                            for (uint32_t o = 0; o < tile_bytes; o += 16384u)
+                                ptx::bulk_load(dst + o, src + o, min(16384u, tile_bytes - o), tb);
+                            dst += tile_bytes;
+                        }
+                    }
+                    if (!__all_sync(0xffffffffu, ptx::mbar_wait(ptx::smem_u32(tail_bar), 0, s_abort, a.status,
+                                                                WAIT_LIMIT))) {
+                        ok = false;
+                        break;
+                    }
+                }
+                const uint32_t yoff = staged ? (uint32_t)(c_hi - c_lo) * tile_bytes : 0u;
+                const uint32_t ybuf =
+                    (last_proc && yoff + 4 * 4096 <= ta.idle_bytes) ? ptx::smem_u32(smem + yoff) + quarter * 4096 : 0u;
+                combine_rows(taddr, ncols, c_lo, c_hi, cta, staged, [&](int c) -> const float* {
+                    if (staged) return reinterpret_cast<const float*>(smem + (size_t)(c - c_lo - (c > cta)) * tile_bytes) + row * 4;
+                    return partial_base(a, s_starts, c, tu0, row);
+                }, sb, ybuf, ycol0, p, s.Cout);
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&acc_empty[abuf]));
+                if (!full && threadIdx.x == 0) a.counters[t] = 0;
+            } else {
+                float* dst = const_cast<float*>(partial_base(a, s_starts, cta, tu0, row));
+                tmem_rows<true>(taddr, a.bn_total, [&](uint32_t(&r)[32], int cc) {
+                    float* b = dst + (size_t)(cc >> 5) * 8 * BM * 4;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        *reinterpret_cast<uint4*>(b + q * BM * 4) = make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+                });
+                __threadfence();
+                if (!epi_sync(epi_bar, ephase, s_abort, a.status)) {
+                    ok = false;
+                    break;
+                }
+                if (threadIdx.x == 0) s_last[seg & 1] = (atomicAdd(a.counters + t, 1) == c_hi - c_lo) ? 1 : 0;
+                if (!epi_sync(epi_bar, ephase, s_abort, a.status)) {
+                    ok = false;
+                    break;
+                }
+                if (s_last[seg & 1]) {
+                    __threadfence();
+                    combine_rows(taddr, ncols, c_lo, c_hi, cta, false, [&](int c) -> const float* {
+                        return partial_base(a, s_starts, c, tu0, row);
+                    }, sb, 0u, ycol0, p, s.Cout);
+                    if (threadIdx.x == 0) a.counters[t] = 0;
+                }
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&acc_empty[abuf]));
+            }
+        }
+    }
+
+    // ------------------------------------------------------------ teardown --
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == MMA_WARP) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem_base, 512u);
+    }
+}
+
+// ------------------------------------------------------------------- host --
+
+struct TsPlan {
+    bool ok;
+    StreamK k;
+    int bn_total, b_stages, acc_cols;
+    uint32_t b_stage_bytes, info_off, row_off, bar_off, smem_bytes, idle_bytes;
+    size_t ws_partials, ws_counters_off, ws_wperm_off, ws_bytes;
+};
+
+TsPlan make_ts_plan(const Shape& s, int sms) {
+    TsPlan pl{};
+    pl.ok = false;
+    if (s.Cin % 8 || s.Cg % 8 || s.Cout % 8 || s.K2 > 25 || s.Cout > 256) return pl;
+    pl.bn_total = (s.Cout + 31) / 32 * 32;
+    pl.k = plan_stream_k(s, pl.bn_total, sms);
+    // two accumulators of <= 128 columns, or one of <= 256, below the A ring at column 256
+    pl.acc_cols = pl.bn_total <= 128 ? 128 : 0;
+    pl.b_stage_bytes = (uint32_t)pl.bn_total * 128;
+    pl.b_stages = std::min(DCN_FWD_TS_B_STAGES, MAX_B_STAGES);
+    const uint32_t ring = (uint32_t)pl.b_stages * pl.b_stage_bytes;
+    const uint32_t info_bytes = (uint32_t)(2 * BM * s.K2 * sizeof(TapRec));
+    pl.info_off = ring;
+    pl.row_off = pl.info_off + info_bytes;
+    pl.bar_off = pl.row_off + (uint32_t)(32 * sizeof(int2) + (MAX_CTAS + 2) * sizeof(long long) + 2 * 512 * sizeof(float));
+    pl.smem_bytes = pl.bar_off + (2 * A_STAGES + 2 * MAX_B_STAGES + 16) * 8 + 16 + 1024;
+    pl.idle_bytes = ring;
+    if (pl.smem_bytes > 227 * 1024) return pl;
+    pl.ws_partials = (size_t)pl.k.ctas * 2 * BM * pl.bn_total * sizeof(float);
+    pl.ws_counters_off = (pl.ws_partials + 255) & ~(size_t)255;
+    pl.ws_wperm_off = (pl.ws_counters_off + (size_t)pl.k.tiles * sizeof(int) + 255) & ~(size_t)255;
+    pl.ws_bytes = pl.ws_wperm_off + (size_t)s.Cout * pl.k.U * BK * 2;
+    pl.ok = true;
+    return pl;
+}
+
+}  // namespace
+
+bool fwd_ts_supported(const Shape& s) { return make_ts_plan(s, num_sms()).ok; }
+
+size_t fwd_ts_workspace(const Shape& s) {
+    const TsPlan pl = make_ts_plan(s, num_sms());
+    return pl.ok ? pl.ws_bytes : 0;
+}
+
+cudaError_t fwd_ts(const Shape& s, const void* x, const void* off, const void* mask, const void* w, const void* bias,
+                   void* y, void* ws, size_t ws_bytes, unsigned* status, cudaStream_t st, int* launches) {
+    const TsPlan pl = make_ts_plan(s, num_sms());
+    if (!pl.ok || ws_bytes < pl.ws_bytes || !ws) return cudaErrorInvalidValue;
+    auto encode = get_encode();
+    if (!encode) return cudaErrorNotSupported;
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    int* counters = reinterpret_cast<int*>(wsb + pl.ws_counters_off);
+    bf16* wperm = reinterpret_cast<bf16*>(wsb + pl.ws_wperm_off);
+    CUtensorMap map;
+    cuuint64_t dims[2] = {(cuuint64_t)pl.k.U * BK, (cuuint64_t)s.Cout};
+    cuuint64_t strides[1] = {(cuuint64_t)pl.k.U * BK * 2};
+    cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)pl.bn_total};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, wperm, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    const bool wide = s.Cin % 16 == 0 && s.Cg % 16 == 0 && (reinterpret_cast<uintptr_t>(x) & 31) == 0;
+    auto kernel = wide ? dcn_fwd_ts_kernel<true> : dcn_fwd_ts_kernel<false>;
+    static DeviceFlags attr_set[2];
+    cudaError_t e = max_dynamic_smem_once((const void*)kernel, 227 * 1024, attr_set[wide]);
+    if (e != cudaSuccess) return e;
+    {
+        const long long n = std::max<long long>((long long)s.Cout * pl.k.U * 8, pl.k.tiles);
+        dcn_wperm_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>((const bf16*)w, wperm, s, pl.k.nq, pl.k.U,
+                                                                       counters, pl.k.tiles);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    TsArgs ta;
+    FwdArgs& a = ta.f;
+    a = FwdArgs{};
+    a.s = s;
+    a.x = (const bf16*)x;
+    a.off = (const bf16*)off;
+    a.mask = (const bf16*)mask;
+    a.bias = (const bf16*)bias;
+    a.y = (bf16*)y;
+    a.partials = reinterpret_cast<float*>(ws);
+    a.counters = counters;
+    a.status = status;
+    a.n_tiles = pl.k.n_tiles;
+    a.tiles = pl.k.tiles;
+    a.U = pl.k.U;
+    a.nq = pl.k.nq;
+    a.sw = pl.k.sw;
+    a.nf = pl.k.nf;
+    a.wl = pl.k.wl;
+    a.ctas = pl.k.ctas;
+    a.total_units = pl.k.total_units;
+    a.snap = pl.k.snap;
+    a.bn_total = pl.bn_total;
+    a.nsub = 1;
+    a.box_rows = pl.bn_total;
+    a.stages = A_STAGES;
+    a.acc_cols = pl.acc_cols;
+    a.tmem_cols = 512;
+    a.b_off = 0;
+    a.info_off = pl.info_off;
+    a.row_off = pl.row_off;
+    a.bar_off = pl.bar_off;
+    a.b_stage_bytes = pl.b_stage_bytes;
+    ta.b_stages = pl.b_stages;
+    ta.idle_bytes = pl.idle_bytes;
+    kernel<<<pl.k.ctas, NUM_THREADS, pl.smem_bytes, st>>>(map, ta);
+    if (launches) *launches += 2;
+    return cudaGetLastError();
+}
+
+}  // namespace dcn

@@ -26,6 +26,15 @@ size_t fwd_tc_workspace(const Shape& s);
 cudaError_t fwd_tc(const Shape& s, const void* x, const void* off, const void* mask, const void* w, const void* bias,
                    void* y, void* ws, size_t ws_bytes, unsigned* status, cudaStream_t st, int* launches);
 
+// fwd_tc_ts.cu — the same forward with the gathered operand in tensor memory (Cout <= 256);
+// fwd_tc() dispatches to it where it applies.
+bool fwd_ts_supported(const Shape& s);
+size_t fwd_ts_workspace(const Shape& s);
+cudaError_t fwd_ts(const Shape& s, const void* x, const void* off, const void* mask, const void* w, const void* bias,
+                   void* y, void* ws, size_t ws_bytes, unsigned* status, cudaStream_t st, int* launches);
+// Which of the two fwd_tc() runs for this shape ("tcgen05_gather_tmem" or "tcgen05_gather").
+const char* fwd_tc_variant(const Shape& s);
+
 // Same forward with its scratch in a static device array instead of a caller workspace.
 size_t fwd_tc_static_scratch_bytes();
 cudaError_t fwd_tc_noalloc(const Shape& s, const void* x, const void* off, const void* mask, const void* w,
@@ -58,6 +67,12 @@ cudaError_t predict_split(int dtype_bf16, const void* y, void* off, void* mask, 
 bool fwd_f32_tc_supported(const Shape& s);
 cudaError_t fwd_f32_tc(const Shape& s, const void* x, const void* off, const void* mask, const void* w,
                        const void* bias, void* y, unsigned* status, cudaStream_t st);
+
+// fwd_f32_stem.cu — the same float32 layers with Cout <= 128 on a persistent, double-buffered
+// kernel (one CTA per SM over the 128-pixel tiles); fwd_f32_tc() dispatches to it where it applies.
+bool fwd_f32_stem_supported(const Shape& s);
+cudaError_t fwd_f32_stem(const Shape& s, const void* x, const void* off, const void* mask, const void* w,
+                         const void* bias, void* y, unsigned* status, cudaStream_t st);
 
 // fwd_f32_small.cu — float32 forward for layers with Cin <= 8 (CUDA cores, HBM-bound).
 bool fwd_f32_small_supported(const Shape& s);
