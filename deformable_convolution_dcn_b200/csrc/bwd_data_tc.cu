@@ -451,6 +451,17 @@ cudaError_t bwd_data_tc(const Shape& s, const void* x, const void* off, const vo
         if ((e = cudaMemsetAsync(gmask, 0, sizeof(float) * (size_t)s.P * s.G * s.K2, st)) != cudaSuccess) return e;
         ++n;
     }
+    // grad_x through the shared-memory window kernel where it applies; this
+    // file's kernel then computes only grad_offset and grad_mask
+    if (gx && bwd_gx_supported(s)) {
+        e = bwd_gx_tc(s, gy, wt, rec, pl.ppad, gx, status, st, &n);
+        if (e != cudaSuccess) return e;
+        gx = nullptr;
+        if (!goff && !gmask) {
+            if (launches) *launches += n;
+            return cudaSuccess;
+        }
+    }
     BdArgs a;
     a.s = s;
     a.x = (const bf16*)x;

@@ -284,7 +284,8 @@ __device__ __forceinline__ void tmem_rows(uint32_t taddr, int ncols, F&& f) {
     }
 }
 
-// y rows = bias + the tile's partial sums in contributor order c_lo..c_hi,
+// y rows = bias + the tile's partial sums in contributor order c_lo..c_hi
+// (columns [cc_begin, cc_end) of them),
 // this CTA's own taken from its TMEM accumulator and every other one from
 // `part(c)` (a row pointer in partial_base layout; in_smem: staged in shared
 // memory). The fixed order makes the result independent of which CTA finishes
@@ -297,10 +298,10 @@ __device__ __forceinline__ void tmem_rows(uint32_t taddr, int ncols, F&& f) {
 template <typename P>
 __device__ __forceinline__ void combine_rows(uint32_t taddr, int ncols, int c_lo, int c_hi, int cta, bool in_smem,
                                              P&& part, const float* sb, uint32_t ybuf, bf16* ycol0, int pr,
-                                             int ldy) {
+                                             int ldy, int cc_begin = 0, int cc_end = 1 << 30) {
     const int lane = threadIdx.x & 31;
-    const bool coalesce = ybuf != 0 && (ncols & 63) == 0;
-    for (int cc = 0; cc < ncols; cc += 32) {
+    const bool coalesce = ybuf != 0 && (ncols & 63) == 0;  // cc_begin must then be a multiple of 64
+    for (int cc = cc_begin; cc < min(ncols, cc_end); cc += 32) {
         uint32_t acc[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) acc[e] = 0u;

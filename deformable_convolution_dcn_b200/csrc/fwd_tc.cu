@@ -596,7 +596,10 @@ cudaError_t fwd_tc(const Shape& s, const void* x, const void* off, const void* m
     const bool wide = s.Cin % 16 == 0 && s.Cg % 16 == 0 && (reinterpret_cast<uintptr_t>(x) & 31) == 0;
     auto kernel = wide ? dcn_fwd_tc_kernel<true> : dcn_fwd_tc_kernel<false>;
     static DeviceFlags attr_set[2];
+    static DeviceCarveout carve[2];
     cudaError_t e = max_dynamic_smem_once((const void*)kernel, 227 * 1024, attr_set[wide]);
+    if (e != cudaSuccess) return e;
+    e = smem_carveout_for((const void*)kernel, pl.smem_bytes, carve[wide]);
     if (e != cudaSuccess) return e;
     int* counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + pl.ws_counters_off);
     e = cudaMemsetAsync(counters, 0, (size_t)pl.tiles * sizeof(int), st);

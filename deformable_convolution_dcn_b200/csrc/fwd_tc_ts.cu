@@ -45,6 +45,11 @@ constexpr int SLICE_CH = 16;                 // channels one lane gathers per sa
 #ifndef DCN_FWD_TS_B_STAGES
 #define DCN_FWD_TS_B_STAGES 3
 #endif
+// Each producer row also asks L1 for its neighbours this many chunks ahead
+// (same epoch only); 0: no prefetch.
+#ifndef DCN_FWD_TS_PREFETCH
+#define DCN_FWD_TS_PREFETCH 2
+#endif
 
 // Sixteen 32-bit registers per thread into 16 TMEM lanes x 32 columns
 // (16x256b shape, 4 repetitions): thread t writes lanes t/4 and t/4 + 8,
@@ -136,9 +141,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint64_t* rec_empty = rec_full + 2;           // [2] every producer warp done with an epoch's records
     uint64_t* rec0_bar = rec_empty + 2;           // the first epoch's records, built by all warps
     uint64_t* epi_bar = rec0_bar + 1;
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(epi_bar + 1);
+    uint64_t* fin_go = epi_bar + 1;  // the last segment's combine plan is known (producers may help)
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(fin_go + 1);
     volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
     volatile int* s_last = s_abort + 1;  // [2], by segment parity
+    volatile int* s_help = s_last + 2;   // [2]: producers share the final combine; partials staged in smem
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < A_STAGES; ++i) {
@@ -161,8 +168,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         ptx::mbar_init(ptx::smem_u32(rec0_bar), NUM_PROD_WARPS + 4);
         ptx::mbar_init(ptx::smem_u32(epi_bar), 4);
+        ptx::mbar_init(ptx::smem_u32(fin_go), 1);
         *s_abort = 0;
         s_last[0] = s_last[1] = 0;
+        s_help[0] = s_help[1] = 0;
         ptx::fence_mbar_init();
     }
     if (threadIdx.x < s.K2) {
@@ -227,6 +236,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int c = 0; c < 4; ++c) {
                 const bool rd = (vm >> c) & 1u;
                 load_slice<WIDE>(v[c], rd ? pc[c] : zb, (rd && hi_ok) ? pc[c] + 16 : zb);
+            }
+            if (DCN_FWD_TS_PREFETCH > 0) {
+                // the same row's neighbours DCN_FWD_TS_PREFETCH chunks on, if still in this epoch
+                int tp = ich.tap + DCN_FWD_TS_PREFETCH, qq = ich.q;
+                while (tp >= s.K2) {
+                    tp -= s.K2;
+                    ++qq;
+                }
+                const int cg2 = qq * BK + j4 * SLICE_CH;
+                if (qq < a.nq && cg2 < s.Cg) {
+                    const TapRec rp = irecs[row * s.K2 + tp];
+                    const uint8_t* q0 = reinterpret_cast<const uint8_t*>(a.x + ich.g * s.Cg + cg2) +
+                                        (long long)rp.base * cin2;
+                    if (rp.vmask & 1u) ptx::prefetch_l1(q0);
+                    if (rp.vmask & 2u) ptx::prefetch_l1(q0 + cin2);
+                    if (rp.vmask & 4u) ptx::prefetch_l1(q0 + rp2);
+                    if (rp.vmask & 8u) ptx::prefetch_l1(q0 + rp2 + cin2);
+                }
             }
         };
         auto advance = [&]() -> bool {
@@ -321,6 +348,46 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&a_full[prev]));
+        }
+        // The CTA's last segment: when this CTA finishes a shared tile there, the
+        // three warps of each TMEM lane quarter (its epilogue warp and two
+        // producers) split the combine of that tile by 64-column pairs.
+        if (ok && L.ns > 0 &&
+            __all_sync(0xffffffffu, ptx::mbar_wait(ptx::smem_u32(fin_go), 0, s_abort, a.status, WAIT_LIMIT)) &&
+            s_help[0]) {
+            const int seg = L.ns - 1;
+            const Seg sg = seg_at(L, seg);
+            const int t = sg.t;
+            const int abuf = a.acc_cols ? (seg & 1) : 0;
+            const uint32_t accph = a.acc_cols ? ((seg >> 1) & 1) : (seg & 1);
+            const bool staged = s_help[1] != 0;
+            const long long tu0 = (long long)t * a.U;
+            const int c_lo = cta_of_unit(tu0, s_starts, a.ctas), c_hi = cta_of_unit(tu0 + a.U - 1, s_starts, a.ctas);
+            const uint32_t tile_bytes = (uint32_t)BM * a.bn_total * 4;
+            bool go = __all_sync(0xffffffffu, ptx::mbar_wait(ptx::smem_u32(&acc_full[abuf]), accph, s_abort, a.status,
+                                                             WAIT_LIMIT));
+            if (go && staged)
+                go = __all_sync(0xffffffffu, ptx::mbar_wait(ptx::smem_u32(tail_bar), 0, s_abort, a.status, WAIT_LIMIT));
+            if (go) {
+                ptx::tc_fence_after();
+                const int mt = t / a.n_tiles, n0 = (t % a.n_tiles) * a.bn_total;
+                const int ncols = min(a.bn_total, s.Cout - n0);
+                const int qd = warp & 3, role = 1 + ((warp - PROD_WARP0) >> 2);
+                const int row = qd * 32 + lane;
+                const int p = strip_to_raster(mt * BM + row, a);
+                const uint32_t taddr = tmem_base + (uint32_t)(abuf * a.acc_cols) + ((uint32_t)(qd * 32) << 16);
+                const float* sb = a.bias ? s_bias + (seg & 1) * 512 : nullptr;
+                const uint32_t yoff = staged ? (uint32_t)(c_hi - c_lo) * tile_bytes : 0u;
+                const uint32_t ybuf = (yoff + 12 * 4096 <= ta.idle_bytes)
+                                          ? ptx::smem_u32(smem + yoff) + (uint32_t)(warp - PROD_WARP0 + 4) * 4096u
+                                          : 0u;
+                for (int pr2 = role; pr2 * 64 < ncols; pr2 += 3)
+                    combine_rows(taddr, ncols, c_lo, c_hi, cta, staged, [&](int c) -> const float* {
+                        if (staged)
+                            return reinterpret_cast<const float*>(smem + (size_t)(c - c_lo - (c > cta)) * tile_bytes) + row * 4;
+                        return partial_base(a, s_starts, c, tu0, row);
+                    }, sb, ybuf, a.y + n0, p, s.Cout, pr2 * 64, pr2 * 64 + 64);
+            }
         }
     } else if (warp == TMA_WARP) {
         // ------------------------------------------------------- weights --
@@ -508,17 +575,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     }
                 }
                 const uint32_t yoff = staged ? (uint32_t)(c_hi - c_lo) * tile_bytes : 0u;
+                // in the last segment the producers take two thirds of the columns (64-column pairs)
+                const bool help = last_proc && (ncols & 63) == 0 && yoff + 12 * 4096 <= ta.idle_bytes;
+                if (last_proc && threadIdx.x == 0) {
+                    s_help[1] = staged ? 1 : 0;
+                    s_help[0] = help ? 1 : 0;
+                    ptx::mbar_arrive(ptx::smem_u32(fin_go));
+                }
                 const uint32_t ybuf =
                     (last_proc && yoff + 4 * 4096 <= ta.idle_bytes) ? ptx::smem_u32(smem + yoff) + quarter * 4096 : 0u;
-                combine_rows(taddr, ncols, c_lo, c_hi, cta, staged, [&](int c) -> const float* {
+                auto part = [&](int c) -> const float* {
                     if (staged) return reinterpret_cast<const float*>(smem + (size_t)(c - c_lo - (c > cta)) * tile_bytes) + row * 4;
                     return partial_base(a, s_starts, c, tu0, row);
-                }, sb, ybuf, ycol0, p, s.Cout);
+                };
+                if (help) {
+                    for (int pr2 = 0; pr2 * 64 < ncols; pr2 += 3)
+                        combine_rows(taddr, ncols, c_lo, c_hi, cta, staged, part, sb, ybuf, ycol0, p, s.Cout, pr2 * 64,
+                                     pr2 * 64 + 64);
+                } else {
+                    combine_rows(taddr, ncols, c_lo, c_hi, cta, staged, part, sb, ybuf, ycol0, p, s.Cout);
+                }
                 ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&acc_empty[abuf]));
                 if (!full && threadIdx.x == 0) a.counters[t] = 0;
             } else {
+                if (last_proc && threadIdx.x == 0) {  // the producers have nothing to add here
+                    s_help[0] = 0;
+                    ptx::mbar_arrive(ptx::smem_u32(fin_go));
+                }
                 float* dst = const_cast<float*>(partial_base(a, s_starts, cta, tu0, row));
                 tmem_rows<true>(taddr, a.bn_total, [&](uint32_t(&r)[32], int cc) {
                     float* b = dst + (size_t)(cc >> 5) * 8 * BM * 4;
@@ -584,7 +669,7 @@ TsPlan make_ts_plan(const Shape& s, int sms) {
     pl.info_off = ring;
     pl.row_off = pl.info_off + info_bytes;
     pl.bar_off = pl.row_off + (uint32_t)(32 * sizeof(int2) + (MAX_CTAS + 2) * sizeof(long long) + 2 * 512 * sizeof(float));
-    pl.smem_bytes = pl.bar_off + (2 * A_STAGES + 2 * MAX_B_STAGES + 16) * 8 + 16 + 1024;
+    pl.smem_bytes = pl.bar_off + (2 * A_STAGES + 2 * MAX_B_STAGES + 17) * 8 + 32 + 1024;
     pl.idle_bytes = ring;
     if (pl.smem_bytes > 227 * 1024) return pl;
     pl.ws_partials = (size_t)pl.k.ctas * 2 * BM * pl.bn_total * sizeof(float);
@@ -625,7 +710,11 @@ cudaError_t fwd_ts(const Shape& s, const void* x, const void* off, const void* m
     const bool wide = s.Cin % 16 == 0 && s.Cg % 16 == 0 && (reinterpret_cast<uintptr_t>(x) & 31) == 0;
     auto kernel = wide ? dcn_fwd_ts_kernel<true> : dcn_fwd_ts_kernel<false>;
     static DeviceFlags attr_set[2];
+    static DeviceCarveout carve[2];
     cudaError_t e = max_dynamic_smem_once((const void*)kernel, 227 * 1024, attr_set[wide]);
+    if (e != cudaSuccess) return e;
+    // the gather hits in L1: give it everything the kernel's shared memory does not need
+    e = smem_carveout_for((const void*)kernel, pl.smem_bytes, carve[wide]);
     if (e != cudaSuccess) return e;
     {
         const long long n = std::max<long long>((long long)s.Cout * pl.k.U * 8, pl.k.tiles);

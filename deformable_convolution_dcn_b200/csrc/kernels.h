@@ -92,6 +92,12 @@ cudaError_t bwd_data_tc(const Shape& s, const void* x, const void* off, const vo
                         const void* gy, float* gx, float* goff, float* gmask, void* ws, size_t ws_bytes,
                         unsigned* status, cudaStream_t st, int* launches);
 
+// bwd_gx_tc.cu — grad_x alone on tcgen05 with the scatter summed in a shared-memory window
+// (groups of whole 32-channel slices); uses the data-backward pre-pass's records and W^T.
+bool bwd_gx_supported(const Shape& s);
+cudaError_t bwd_gx_tc(const Shape& s, const void* gy, const void* wt, const void* rec, int ppad, float* gx,
+                      unsigned* status, cudaStream_t st, int* launches);
+
 // selftest.cu — a kernel whose bounded wait can only give up (failure-detection test).
 cudaError_t selftest_wait_timeout(long long limit_cycles, cudaStream_t st);
 
@@ -109,5 +115,14 @@ struct DeviceFlags {
 // cudaFuncSetAttribute(func, MaxDynamicSharedMemorySize, bytes) once per device
 // for the current device; later calls return at once. Thread-safe.
 cudaError_t max_dynamic_smem_once(const void* func, int bytes, DeviceFlags& flags);
+// Per-device cache of the last shared-memory carveout set for one kernel.
+struct DeviceCarveout {
+    std::atomic<int> pct[64];  // 0: not set yet, else percentage + 1
+};
+// Asks for the smallest shared-memory carveout that holds `smem_bytes` of
+// dynamic shared memory for `func` on the current device, leaving the rest of
+// the SM's unified L1 / shared memory to the L1 cache (re-set only when the
+// needed percentage changes). Thread-safe.
+cudaError_t smem_carveout_for(const void* func, uint32_t smem_bytes, DeviceCarveout& cache);
 
 }  // namespace dcn

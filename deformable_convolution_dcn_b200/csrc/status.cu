@@ -62,6 +62,25 @@ cudaError_t max_dynamic_smem_once(const void* func, int bytes, DeviceFlags& flag
     return e;
 }
 
+cudaError_t smem_carveout_for(const void* func, uint32_t smem_bytes, DeviceCarveout& cache) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    int per_sm = 0;
+    e = cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+    if (e != cudaSuccess || per_sm <= 0) return e != cudaSuccess ? e : cudaErrorInvalidValue;
+    // the block's dynamic shared memory plus the 1 KB the system reserves per block
+    int pct = (int)(((long long)smem_bytes + 1024) * 100 / per_sm) + 1;
+    pct = pct > 100 ? 100 : pct;
+    if (cache.pct[dev].load(std::memory_order_acquire) == pct + 1) return cudaSuccess;
+    std::lock_guard<std::mutex> lock(g_setup_mu);
+    if (cache.pct[dev].load(std::memory_order_relaxed) == pct + 1) return cudaSuccess;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributePreferredSharedMemoryCarveout, pct);
+    if (e == cudaSuccess) cache.pct[dev].store(pct + 1, std::memory_order_release);
+    return e;
+}
+
 int num_sms() {
     static std::atomic<int> cached[64];
     int dev = 0;
