@@ -39,6 +39,11 @@ constexpr int MAX_STAGES = 4;
 constexpr uint32_t A_BYTES = BM * BK * 2;   // 16 KB
 constexpr uint32_t B_BYTES = NT * BK * 2;   // 32 KB
 constexpr int TPITCH = 36;                  // floats per row of an epilogue warp's 32x32 transpose buffer
+// grad_x through bwd_gx_tc.cu's shared-memory window (1) or this file's
+// per-sample vector atomics (0, faster on the shapes measured so far)
+#ifndef DCN_BWD_GX_WINDOW
+#define DCN_BWD_GX_WINDOW 0
+#endif
 
 struct BdArgs {
     Shape s;
@@ -451,9 +456,10 @@ cudaError_t bwd_data_tc(const Shape& s, const void* x, const void* off, const vo
         if ((e = cudaMemsetAsync(gmask, 0, sizeof(float) * (size_t)s.P * s.G * s.K2, st)) != cudaSuccess) return e;
         ++n;
     }
-    // grad_x through the shared-memory window kernel where it applies; this
-    // file's kernel then computes only grad_offset and grad_mask
-    if (gx && bwd_gx_supported(s)) {
+    // grad_x through the shared-memory window kernel where it applies (and
+    // DCN_BWD_GX_WINDOW is on); this file's kernel then computes only
+    // grad_offset and grad_mask
+    if (DCN_BWD_GX_WINDOW && gx && bwd_gx_supported(s)) {
         e = bwd_gx_tc(s, gy, wt, rec, pl.ppad, gx, status, st, &n);
         if (e != cudaSuccess) return e;
         gx = nullptr;

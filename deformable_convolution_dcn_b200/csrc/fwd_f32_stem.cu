@@ -7,11 +7,12 @@
 // x_hi the nearest tf32 value of x and x_lo = x - x_hi. Such a layer moves far
 // more bytes (offsets, mask, and above all the float32 output) than it does
 // arithmetic, so the kernel is laid out to keep reads and writes in flight
-// together: one CTA per SM walks its share of the 128-pixel tiles with two A
-// buffers and two TMEM accumulators.
+// together: one CTA per SM walks an equal share of the output rows (whole
+// groups of 8), in tiles of up to 128 pixels, with two A buffers and two TMEM
+// accumulators.
 //
 //   * warps 4-15 (three threads per tile row, each a third of the taps): load
-//     the NEXT tile's offsets and mask into registers, gather the current
+//     the next tile's offsets and mask into registers, gather the current
 //     tile's modulated samples (bilinear, a neighbour outside the map
 //     contributing zero), split them and write both parts into the tile's A
 //     buffer; one of them issues the tile's twelve kind::tf32 MMAs;
@@ -56,7 +57,8 @@ __device__ __forceinline__ uint32_t sw_off(int r, int c) { return (uint32_t)(r *
 
 template <int CIN>
 __global__ void __launch_bounds__(S_THREADS, 1)
-    stem_persistent_kernel(const __grid_constant__ CUtensorMap tmap_y, const StemArgs a) {
+    stem_persistent_kernel(const __grid_constant__ CUtensorMap tmap_y, const __grid_constant__ CUtensorMap tmap_y8,
+                           const StemArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const Shape& s = a.s;
@@ -72,8 +74,13 @@ __global__ void __launch_bounds__(S_THREADS, 1)
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 5);
     volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
     const uint32_t wbytes = (uint32_t)s.Cout * KC * 4;
-    // this CTA's tiles: blockIdx.x, blockIdx.x + gridDim.x, ...
-    const int ntl = a.tiles > (int)blockIdx.x ? (a.tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    // This CTA's output pixels: an equal share [rbeg, rend) of the P rows of y,
+    // cut at multiples of 8 rows, walked in tiles of up to 128 rows.
+    const long long p8 = (s.P + 7) / 8;
+    const int rbeg = (int)(8 * (p8 * blockIdx.x / gridDim.x));
+    const int rend = blockIdx.x + 1 == gridDim.x ? s.P : (int)(8 * (p8 * (blockIdx.x + 1) / gridDim.x));
+    const int ntl = rend > rbeg ? (rend - rbeg + S_BM - 1) / S_BM : 0;
+    auto tile_end = [&](int i) { return min(rbeg + (i + 1) * S_BM, rend); };
 
     if (tid == 0) {
         ptx::mbar_init(ptx::smem_u32(wbar), 1);
@@ -101,11 +108,12 @@ __global__ void __launch_bounds__(S_THREADS, 1)
     const int row = gt & (S_BM - 1), part = gt >> 7;
     const int tp_lo = s.K2 * part / S_PARTS, tp_hi = s.K2 * (part + 1) / S_PARTS;
     const int plane = s.Ho * s.Wo;
-    float cur[3 * S_TAPS_PER_PART], nxt[3 * S_TAPS_PER_PART];
     // offsets and mask of tile-local row `row` of this CTA's i-th tile, for this thread's taps
+    // (two register sets in turn: a tile's values are requested while the tile before it is gathered)
+    float S0[3 * S_TAPS_PER_PART], S1[3 * S_TAPS_PER_PART];
     auto fetch = [&](int i, float (&v)[3 * S_TAPS_PER_PART]) {
-        const int p = ((int)blockIdx.x + i * (int)gridDim.x) * S_BM + row;
-        const bool pv = i < ntl && p < s.P;
+        const int p = rbeg + i * S_BM + row;
+        const bool pv = i < ntl && p < tile_end(i);
         int bb = 0, pix = 0;
         if (pv) {
             bb = p / plane;
@@ -125,7 +133,10 @@ __global__ void __launch_bounds__(S_THREADS, 1)
             }
         }
     };
-    if (gt >= 0) fetch(0, cur);
+    if (gt >= 0) {
+        fetch(0, S0);
+        fetch(1, S1);
+    }
 
     // ---- weights into the two B tiles: row n = output channel, k = tap*Cin + c, zero for k >= KC
     __syncthreads();  // barriers initialised, TMEM allocated, bias staged
@@ -157,18 +168,16 @@ __global__ void __launch_bounds__(S_THREADS, 1)
     if (gt >= 0) {
         // ------------------------------------------------------------ gather --
         const float* xb0 = a.x;
-        for (int i = 0; i < ntl && ok; ++i) {
+        // tile i of this CTA from the offsets in `cur`
+        auto gather_tile = [&](int i, const float (&cur)[3 * S_TAPS_PER_PART]) {
             const int buf = i & 1;
             const uint32_t arow = ptx::smem_u32(smem + a.a_off) + (uint32_t)buf * 2 * S_TILE + (uint32_t)row * 128;
-            if (i + 1 < ntl) fetch(i + 1, nxt);
-            // the MMAs of tile i - 2 have read this A buffer
-            if (i >= 2 && !ptx::mbar_wait(ptx::smem_u32(&mma_bar[buf]), ((i >> 1) - 1) & 1, s_abort, a.status,
-                                          WAIT_LIMIT)) {
-                ok = false;
-                break;
-            }
-            const int p = ((int)blockIdx.x + i * (int)gridDim.x) * S_BM + row;
-            const bool pv = p < s.P;
+            // the MMAs of tile i - 2 have read this A buffer (a thread that gives up still
+            // reaches the barrier below, where all decide together)
+            const bool w_ok = i < 2 || ptx::mbar_wait(ptx::smem_u32(&mma_bar[buf]), ((i >> 1) - 1) & 1, s_abort,
+                                                      a.status, WAIT_LIMIT);
+            const int p = rbeg + i * S_BM + row;
+            const bool pv = w_ok && p < tile_end(i);
             int bb = 0, oy = 0, ox = 0;
             if (pv) {
                 bb = p / plane;
@@ -226,7 +235,10 @@ __global__ void __launch_bounds__(S_THREADS, 1)
             }
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
-            ptx::bar_sync_named(BAR_GATHER, S_PARTS * S_BM);
+            if (ptx::bar_or_named(BAR_GATHER, S_PARTS * S_BM, !w_ok || *s_abort)) {
+                ok = false;
+                return;
+            }
             if (gt == 0) {
                 // accumulator `buf` was read by the epilogue of tile i - 2
                 if (i >= 2 && !ptx::mbar_wait(ptx::smem_u32(&acc_empty[buf]), ((i >> 1) - 1) & 1, s_abort, a.status,
@@ -252,8 +264,14 @@ __global__ void __launch_bounds__(S_THREADS, 1)
                     ptx::mma_commit(ptx::smem_u32(&mma_bar[buf]));
                 }
             }
-#pragma unroll
-            for (int j = 0; j < 3 * S_TAPS_PER_PART; ++j) cur[j] = nxt[j];
+        };
+        for (int i = 0; i < ntl && ok; i += 2) {
+            gather_tile(i, S0);
+            fetch(i + 2, S0);
+            if (i + 1 < ntl && ok) {
+                gather_tile(i + 1, S1);
+                fetch(i + 3, S1);
+            }
         }
     } else {
         // ---------------------------------------------------------- epilogue --
@@ -261,15 +279,14 @@ __global__ void __launch_bounds__(S_THREADS, 1)
         const uint32_t stg = ptx::smem_u32(smem + a.st_off);
         for (int i = 0; i < ntl && ok; ++i) {
             const int buf = i & 1;
-            if (!__all_sync(0xffffffffu, ptx::mbar_wait(ptx::smem_u32(&mma_bar[buf]), (i >> 1) & 1, s_abort, a.status,
-                                                        WAIT_LIMIT))) {
-                ok = false;
-                break;
-            }
+            const bool w_ok = ptx::mbar_wait(ptx::smem_u32(&mma_bar[buf]), (i >> 1) & 1, s_abort, a.status, WAIT_LIMIT);
             ptx::tc_fence_after();
             // the previous tile's stores have finished reading the staging tile
             if (tid == 0) ptx::bulk_wait_group_read0();
-            ptx::bar_sync_named(BAR_EPI, S_EPI_THREADS);
+            if (ptx::bar_or_named(BAR_EPI, S_EPI_THREADS, !w_ok || *s_abort)) {  // one decision for all four warps
+                ok = false;
+                break;
+            }
             for (int cb = 0; cb < s.Cout / 32; ++cb) {
                 float v[32];
                 ptx::tmem_ld32(taddr0 + (uint32_t)(buf * a.acc_cols) + cb * 32, v);
@@ -289,9 +306,17 @@ __global__ void __launch_bounds__(S_THREADS, 1)
             ptx::fence_proxy_async_smem();
             ptx::bar_sync_named(BAR_EPI, S_EPI_THREADS);
             if (tid == 0) {
-                const int tile = (int)blockIdx.x + i * (int)gridDim.x;
-                for (int cb = 0; cb < s.Cout / 32; ++cb)
-                    ptx::tma_store_2d(&tmap_y, stg + cb * S_TILE, cb * 32, tile * S_BM);
+                // a whole tile in 128-row boxes; a CTA's shorter last tile in 8-row boxes
+                // (its share ends on a multiple of 8 rows, or at the end of y)
+                const int p0 = rbeg + i * S_BM, nrow = tile_end(i) - p0;
+                for (int cb = 0; cb < s.Cout / 32; ++cb) {
+                    if (nrow == S_BM) {
+                        ptx::tma_store_2d(&tmap_y, stg + cb * S_TILE, cb * 32, p0);
+                    } else {
+                        for (int r8 = 0; r8 < nrow; r8 += 8)
+                            ptx::tma_store_2d(&tmap_y8, stg + cb * S_TILE + (uint32_t)r8 * 128, cb * 32, p0 + r8);
+                    }
+                }
                 ptx::bulk_commit_group();
             }
         }
@@ -352,6 +377,11 @@ cudaError_t launch_stem(const Shape& s, const float* x, const float* off, const 
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    CUtensorMap map8;  // the same, in boxes of 8 rows
+    cuuint32_t box8[2] = {32, 8};
+    r = encode(&map8, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, y, dims, strides, box8, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     static DeviceFlags attr;
     cudaError_t e = max_dynamic_smem_once((const void*)stem_persistent_kernel<CIN>, 227 * 1024, attr);
     if (e != cudaSuccess) return e;
@@ -373,8 +403,9 @@ cudaError_t launch_stem(const Shape& s, const float* x, const float* off, const 
     a.bar_off = pl.bar_off;
     a.acc_cols = s.Cout;
     a.tmem_cols = pl.tmem_cols;
-    const int grid = std::min(a.tiles, num_sms());
-    stem_persistent_kernel<CIN><<<grid, S_THREADS, pl.smem_bytes, st>>>(map, a);
+    // one CTA per SM, each an equal share of the rows (a whole number of 8-row groups)
+    const int grid = (int)std::min<long long>(num_sms(), ((long long)s.P + 7) / 8);
+    stem_persistent_kernel<CIN><<<grid, S_THREADS, pl.smem_bytes, st>>>(map, map8, a);
     return cudaGetLastError();
 }
 

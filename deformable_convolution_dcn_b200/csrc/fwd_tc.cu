@@ -578,7 +578,11 @@ size_t fwd_tc_workspace(const Shape& s) {
 
 cudaError_t fwd_tc(const Shape& s, const void* x, const void* off, const void* mask, const void* w, const void* bias,
                    void* y, void* ws, size_t ws_bytes, unsigned* status, cudaStream_t st, int* launches) {
-    if (fwd_ts_supported(s)) return fwd_ts(s, x, off, mask, w, bias, y, ws, ws_bytes, status, st, launches);
+    if (fwd_ts_supported(s)) {
+        const cudaError_t e = fwd_ts(s, x, off, mask, w, bias, y, ws, ws_bytes, status, st, launches);
+        if (e != cudaErrorNotSupported) return e;
+        (void)cudaGetLastError();  // the build's register layout does not fit that kernel: run this one
+    }
     Plan pl = make_plan(s, num_sms());
     if (!pl.ok || ws_bytes < pl.ws_bytes || !ws) return cudaErrorInvalidValue;
     auto encode = get_encode();

@@ -45,11 +45,6 @@ constexpr int SLICE_CH = 16;                 // channels one lane gathers per sa
 #ifndef DCN_FWD_TS_B_STAGES
 #define DCN_FWD_TS_B_STAGES 3
 #endif
-// Each producer row also asks L1 for its neighbours this many chunks ahead
-// (same epoch only); 0: no prefetch.
-#ifndef DCN_FWD_TS_PREFETCH
-#define DCN_FWD_TS_PREFETCH 2
-#endif
 
 // Sixteen 32-bit registers per thread into 16 TMEM lanes x 32 columns
 // (16x256b shape, 4 repetitions): thread t writes lanes t/4 and t/4 + 8,
@@ -236,24 +231,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int c = 0; c < 4; ++c) {
                 const bool rd = (vm >> c) & 1u;
                 load_slice<WIDE>(v[c], rd ? pc[c] : zb, (rd && hi_ok) ? pc[c] + 16 : zb);
-            }
-            if (DCN_FWD_TS_PREFETCH > 0) {
-                // the same row's neighbours DCN_FWD_TS_PREFETCH chunks on, if still in this epoch
-                int tp = ich.tap + DCN_FWD_TS_PREFETCH, qq = ich.q;
-                while (tp >= s.K2) {
-                    tp -= s.K2;
-                    ++qq;
-                }
-                const int cg2 = qq * BK + j4 * SLICE_CH;
-                if (qq < a.nq && cg2 < s.Cg) {
-                    const TapRec rp = irecs[row * s.K2 + tp];
-                    const uint8_t* q0 = reinterpret_cast<const uint8_t*>(a.x + ich.g * s.Cg + cg2) +
-                                        (long long)rp.base * cin2;
-                    if (rp.vmask & 1u) ptx::prefetch_l1(q0);
-                    if (rp.vmask & 2u) ptx::prefetch_l1(q0 + cin2);
-                    if (rp.vmask & 4u) ptx::prefetch_l1(q0 + rp2);
-                    if (rp.vmask & 8u) ptx::prefetch_l1(q0 + rp2 + cin2);
-                }
             }
         };
         auto advance = [&]() -> bool {

@@ -311,6 +311,21 @@ __device__ __forceinline__ void bar_sync_named(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Named barrier over nthreads threads that also ORs `v` across them: every
+// participant returns the same value, so a decision taken on it is uniform.
+__device__ __forceinline__ bool bar_or_named(int id, int nthreads, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
+
 __device__ __forceinline__ uint4 ldg_v4(const void* p) {
     uint4 v;
     asm("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
