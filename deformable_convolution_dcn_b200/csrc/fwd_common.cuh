@@ -295,10 +295,13 @@ __device__ __forceinline__ void tmem_rows(uint32_t taddr, int ncols, F&& f) {
 // 16-byte chunks swizzled by row) and a tile width that is a multiple of 64,
 // every 64 columns of the warp's 32 rows go through it and leave as full
 // 128-byte row segments, eight lanes per row; otherwise each lane stores its row.
+// own_in_part: this CTA's own contribution is read back from part(cta) as
+// well (its accumulator has already been released).
 template <typename P>
 __device__ __forceinline__ void combine_rows(uint32_t taddr, int ncols, int c_lo, int c_hi, int cta, bool in_smem,
                                              P&& part, const float* sb, uint32_t ybuf, bf16* ycol0, int pr,
-                                             int ldy, int cc_begin = 0, int cc_end = 1 << 30) {
+                                             int ldy, int cc_begin = 0, int cc_end = 1 << 30,
+                                             bool own_in_part = false) {
     const int lane = threadIdx.x & 31;
     const bool coalesce = ybuf != 0 && (ncols & 63) == 0;  // cc_begin must then be a multiple of 64
     for (int cc = cc_begin; cc < min(ncols, cc_end); cc += 32) {
@@ -309,7 +312,9 @@ __device__ __forceinline__ void combine_rows(uint32_t taddr, int ncols, int c_lo
             if (in_smem) add_partial32_smem(acc, part(c), cc);
             else add_partial32(acc, part(c), cc);
         }
-        {
+        if (own_in_part) {
+            add_partial32(acc, part(cta), cc);
+        } else {
             uint32_t r[32];
             ptx::tmem_ld32_issue(taddr + cc, r);
             ptx::tmem_wait_ld(r);
@@ -379,6 +384,38 @@ __device__ __forceinline__ Chunk chunk_of(int u, const FwdArgs& a) {
     c.q = r / a.s.K2;
     c.tap = r - c.q * a.s.K2;
     return c;
+}
+
+// The sampling record of tile row `row`, tap `tp`, group g of m-tile mt (as
+// build_records below computes it), for a pre-pass that writes all of them.
+__device__ __forceinline__ TapRec record_at(const FwdArgs& a, int mt, int g, int row, int tp) {
+    const Shape& s = a.s;
+    const int plane = s.Ho * s.Wo;
+    const int pr = strip_to_raster(mt * BM + row, a);
+    TapRec rc;
+    rc.w01_00 = rc.w11_10 = 0u;
+    rc.base = 0;
+    rc.vmask = 0u;
+    if (pr < 0) return rc;
+    const int bb = pr / plane, pix = pr - bb * plane;
+    const int ho = pix / s.Wo, wo = pix - ho * s.Wo;
+    const int i = tp / s.K, j = tp - i * s.K;
+    const bf16* offp = a.off + ((size_t)bb * 2 * s.G * s.K2 + (size_t)g * 2 * s.K2 + 2 * tp) * plane + pix;
+    const float dy = __bfloat162float(offp[0]), dx = __bfloat162float(offp[plane]);
+    const float mk = a.mask ? __bfloat162float(a.mask[((size_t)bb * s.G * s.K2 + (size_t)g * s.K2 + tp) * plane + pix])
+                            : 1.f;
+    int y0, x0;
+    float ly, lx;
+    split_coord(ho * s.stride - s.pad + i * s.dil, dy, y0, ly);
+    split_coord(wo * s.stride - s.pad + j * s.dil, dx, x0, lx);
+    const bool v00 = inside(s, y0, x0), v01 = inside(s, y0, x0 + 1);
+    const bool v10 = inside(s, y0 + 1, x0), v11 = inside(s, y0 + 1, x0 + 1);
+    rc.w01_00 = pack_bf16(v00 ? (1.f - ly) * (1.f - lx) * mk : 0.f, v01 ? (1.f - ly) * lx * mk : 0.f);
+    rc.w11_10 = pack_bf16(v10 ? ly * (1.f - lx) * mk : 0.f, v11 ? ly * lx * mk : 0.f);
+    if (v00 | v01 | v10 | v11) rc.base = (bb * s.H + y0) * s.W + x0;
+    rc.vmask = ((rc.w01_00 & 0x7FFFu) ? 1u : 0u) | ((rc.w01_00 & 0x7FFF0000u) ? 2u : 0u) |
+               ((rc.w11_10 & 0x7FFFu) ? 4u : 0u) | ((rc.w11_10 & 0x7FFF0000u) ? 8u : 0u);
+    return rc;
 }
 
 // Sampling records of tile row `row` for the taps of `part` (0..2: a third of

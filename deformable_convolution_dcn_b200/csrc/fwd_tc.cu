@@ -652,7 +652,7 @@ cudaError_t fwd_tc(const Shape& s, const void* x, const void* off, const void* m
 // process exits; all calls share it.
 namespace {
 
-constexpr size_t kStaticScratchBytes = 40ull << 20;  // 40 MiB
+constexpr size_t kStaticScratchBytes = 48ull << 20;  // 48 MiB
 static __device__ __align__(256) unsigned char g_fwd_scratch[kStaticScratchBytes];
 
 // Device address of g_fwd_scratch on the current device, looked up once per

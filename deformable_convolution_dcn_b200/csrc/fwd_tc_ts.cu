@@ -73,20 +73,37 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
 
 struct TsArgs {
     FwdArgs f;
+    const TapRec* recs;   // [m tiles][G][K*K][BM] sampling records (workspace), tap-major
     int b_stages;
     uint32_t idle_bytes;  // shared memory free after the last MMA (the weight ring)
 };
 
 // ------------------------------------------------------------ pre-pass --
-// W' [Cout][U*64] from W [Cout][K*K*Cin]: unit u = (g, q, tap) (taps innermost),
-// K position k of the unit holds channel c = 16*((k >> 2) & 3) + 4*(k >> 4) + (k & 3)
-// of chunk q of group g at tap `tap` (zero past the group's channels). One
-// thread per 8 outputs (16 bytes); also clears the stream-K tile counters.
-__global__ void __launch_bounds__(256) dcn_wperm_kernel(const bf16* __restrict__ w, bf16* __restrict__ wp, Shape s,
-                                                        int nq, int U, int* counters, int tiles) {
+// The pre-pass of a call. (1) W' [Cout][U*64] from W [Cout][K*K*Cin]: unit
+// u = (g, q, tap) (taps innermost), K position k of the unit holds channel
+// c = 16*((k >> 2) & 3) + 4*(k >> 4) + (k & 3) of chunk q of group g at tap
+// `tap` (zero past the group's channels), one thread per 8 outputs (16 bytes);
+// (2) the sampling record of every (m tile, group, tap, tile row), tap-major so
+// that one (tile, group) epoch is one contiguous block; (3) the stream-K tile
+// counters cleared. Blocks [0, wblocks) do (1) and (3), the rest (2).
+__global__ void __launch_bounds__(256) dcn_fwd_prepass_kernel(const bf16* __restrict__ w, bf16* __restrict__ wp,
+                                                              TapRec* __restrict__ recs, const FwdArgs a, int wblocks,
+                                                              long long nrec) {
+    const Shape& s = a.s;
+    if ((int)blockIdx.x >= wblocks) {
+        const long long r = (long long)(blockIdx.x - wblocks) * blockDim.x + threadIdx.x;
+        if (r >= nrec) return;
+        const int row = (int)(r % BM);
+        const long long e = r / BM;  // (mt * G + g) * K2 + tap
+        const int tp = (int)(e % s.K2);
+        const long long mg = e / s.K2;
+        recs[r] = record_at(a, (int)(mg / s.G), (int)(mg % s.G), row, tp);
+        return;
+    }
+    const int nq = a.nq, U = a.U;
     const long long n8 = (long long)s.Cout * U * 8;
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i < tiles) counters[i] = 0;
+    if (i < a.tiles) a.counters[i] = 0;
     if (i >= n8) return;
     const int k8 = (int)(i & 7);
     const long long ou = i >> 3;
@@ -132,10 +149,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint64_t* acc_empty = acc_full + 2;           // [2]
     uint64_t* drain = acc_empty + 2;
     uint64_t* tail_bar = drain + 1;               // bulk copy of other CTAs' partials for the last segment
-    uint64_t* rec_full = tail_bar + 1;            // [2] records of an epoch built
+    uint64_t* rec_full = tail_bar + 1;            // [2] an epoch's records copied in
     uint64_t* rec_empty = rec_full + 2;           // [2] every producer warp done with an epoch's records
-    uint64_t* rec0_bar = rec_empty + 2;           // the first epoch's records, built by all warps
-    uint64_t* epi_bar = rec0_bar + 1;
+    uint64_t* epi_bar = rec_empty + 2;
     uint64_t* fin_go = epi_bar + 1;  // the last segment's combine plan is known (producers may help)
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(fin_go + 1);
     volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
@@ -158,10 +174,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ptx::mbar_init(ptx::smem_u32(drain), 1);
         ptx::mbar_init(ptx::smem_u32(tail_bar), 1);
         for (int i = 0; i < 2; ++i) {
-            ptx::mbar_init(ptx::smem_u32(&rec_full[i]), 4);
+            ptx::mbar_init(ptx::smem_u32(&rec_full[i]), 1);
             ptx::mbar_init(ptx::smem_u32(&rec_empty[i]), NUM_PROD_WARPS);
         }
-        ptx::mbar_init(ptx::smem_u32(rec0_bar), NUM_PROD_WARPS + 4);
         ptx::mbar_init(ptx::smem_u32(epi_bar), 4);
         ptx::mbar_init(ptx::smem_u32(fin_go), 1);
         *s_abort = 0;
@@ -197,14 +212,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const long long cin2 = (long long)s.Cin * 2, rp2 = (long long)s.W * cin2;
         const uint8_t* zb = reinterpret_cast<const uint8_t*>(g_zero_slice);
         bool ok = true;
-        // the first epoch's records are built by all warps together
-        if (L.ns > 0) {
-            const Seg s0 = seg_at(L, 0);
-            build_records(a, s0.t / a.n_tiles, s0.k0 / (a.nq * s.K2), ptid & (BM - 1), 1 + (ptid >> 7), s_rec, s_tap);
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(rec0_bar));
-            ok = __all_sync(0xffffffffu, ptx::mbar_wait(ptx::smem_u32(rec0_bar), 0, s_abort, a.status, WAIT_LIMIT));
-        }
+        // the first epoch's records (copied in by the epilogue side)
+        if (L.ns > 0)
+            ok = __all_sync(0xffffffffu, ptx::mbar_wait(ptx::smem_u32(&rec_full[0]), 0, s_abort, a.status, WAIT_LIMIT));
         int isi = 0, ik = 0, ik1 = 0, icur_g = -1, iepoch = 0;
         Chunk ich{0, 0, 0};
         const TapRec* irecs = s_rec;
@@ -221,7 +231,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint32_t cmask = cg < s.Cg ? 0xFu : 0u;
             const bool hi_ok = cg + 8 < s.Cg;  // upper 8 channels present (narrow loads only)
             const uint8_t* xc = reinterpret_cast<const uint8_t*>(a.x + ich.g * s.Cg + cg);
-            const TapRec rc = irecs[row * s.K2 + ich.tap];
+            const TapRec rc = irecs[ich.tap * BM + row];
             w[0] = rc.w01_00;
             w[1] = rc.w11_10;
             const uint32_t vm = rc.vmask & cmask;
@@ -254,7 +264,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&rec_empty[iepoch & 1]));
                 ++iepoch;
                 const int b = iepoch & 1;
-                const uint32_t par = (uint32_t)(b ? (iepoch >> 1) : ((iepoch >> 1) - 1)) & 1u;
+                const uint32_t par = (uint32_t)(iepoch >> 1) & 1u;
                 // warp-uniform outcome: the tcgen05.st below is warp-collective
                 if (!__all_sync(0xffffffffu, ptx::mbar_wait(ptx::smem_u32(&rec_full[b]), par, s_abort, a.status,
                                                             WAIT_LIMIT)))
@@ -473,15 +483,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             while (rseg < L.ns && (rseg <= seg || (rseg == seg + 1 && rk == seg_at(L, rseg).k0))) {
                 const Seg rs = seg_at(L, rseg);
                 const int b = rec_epoch & 1;
-                if (rec_epoch >= 2 && !ptx::mbar_wait(ptx::smem_u32(&rec_empty[b]), ((rec_epoch - 2) >> 1) & 1, s_abort,
-                                                      a.status, WAIT_LIMIT)) {
-                    ok = false;
-                    break;
-                }
                 const int rg = rk / per_g;
-                build_records(a, rs.t / a.n_tiles, rg, row, rec_epoch == 0 ? 0 : -1, s_rec + b * BM * s.K2, s_tap);
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(rec_epoch == 0 ? rec0_bar : &rec_full[b]));
+                if (threadIdx.x == 0) {
+                    // buffer b is free once every producer warp has left epoch rec_epoch - 2
+                    if (rec_epoch >= 2 && !ptx::mbar_wait(ptx::smem_u32(&rec_empty[b]), ((rec_epoch - 2) >> 1) & 1,
+                                                          s_abort, a.status, WAIT_LIMIT)) {
+                        ok = false;
+                    } else {
+                        ptx::fence_proxy_async_smem();  // the producers' reads before the copy's writes
+                        const uint32_t bytes = (uint32_t)(BM * s.K2 * sizeof(TapRec));
+                        const uint32_t fb = ptx::smem_u32(&rec_full[b]);
+                        ptx::mbar_arrive_expect_tx(fb, bytes);
+                        ptx::bulk_load(ptx::smem_u32(s_rec + b * BM * s.K2),
+                                       ta.recs + ((size_t)(rs.t / a.n_tiles) * s.G + rg) * s.K2 * BM, bytes, fb);
+                    }
+                }
+                if (warp == 0) ok = __shfl_sync(0xffffffffu, ok, 0);  // warp 0 stays convergent
+                if (!ok) break;
                 rk = min((rg + 1) * per_g, rs.k1);
                 if (rk >= rs.k1 && ++rseg < L.ns) rk = seg_at(L, rseg).k0;
                 ++rec_epoch;
@@ -588,6 +606,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     for (int q = 0; q < 8; ++q)
                         *reinterpret_cast<uint4*>(b + q * BM * 4) = make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
                 });
+                // the accumulator is in the workspace now: hand it to the next segment's MMAs
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&acc_empty[abuf]));
                 __threadfence();
                 if (!epi_sync(epi_bar, ephase, s_abort, a.status)) {
                     ok = false;
@@ -599,15 +621,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     break;
                 }
                 if (s_last[seg & 1]) {
+                    // every contributor's partial, this CTA's included, is in the workspace
                     __threadfence();
                     combine_rows(taddr, ncols, c_lo, c_hi, cta, false, [&](int c) -> const float* {
                         return partial_base(a, s_starts, c, tu0, row);
-                    }, sb, 0u, ycol0, p, s.Cout);
+                    }, sb, 0u, ycol0, p, s.Cout, 0, 1 << 30, true);
                     if (threadIdx.x == 0) a.counters[t] = 0;
                 }
-                ptx::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&acc_empty[abuf]));
             }
         }
     }
@@ -628,7 +648,8 @@ struct TsPlan {
     StreamK k;
     int bn_total, b_stages, acc_cols;
     uint32_t b_stage_bytes, info_off, row_off, bar_off, smem_bytes, idle_bytes;
-    size_t ws_partials, ws_counters_off, ws_wperm_off, ws_bytes;
+    size_t ws_partials, ws_counters_off, ws_wperm_off, ws_recs_off, ws_bytes;
+    long long nrec;
 };
 
 TsPlan make_ts_plan(const Shape& s, int sms) {
@@ -652,7 +673,9 @@ TsPlan make_ts_plan(const Shape& s, int sms) {
     pl.ws_partials = (size_t)pl.k.ctas * 2 * BM * pl.bn_total * sizeof(float);
     pl.ws_counters_off = (pl.ws_partials + 255) & ~(size_t)255;
     pl.ws_wperm_off = (pl.ws_counters_off + (size_t)pl.k.tiles * sizeof(int) + 255) & ~(size_t)255;
-    pl.ws_bytes = pl.ws_wperm_off + (size_t)s.Cout * pl.k.U * BK * 2;
+    pl.ws_recs_off = (pl.ws_wperm_off + (size_t)s.Cout * pl.k.U * BK * 2 + 255) & ~(size_t)255;
+    pl.nrec = (long long)pl.k.m_tiles * s.G * s.K2 * BM;
+    pl.ws_bytes = pl.ws_recs_off + (size_t)pl.nrec * sizeof(TapRec);
     pl.ok = true;
     return pl;
 }
@@ -693,13 +716,6 @@ cudaError_t fwd_ts(const Shape& s, const void* x, const void* off, const void* m
     // the gather hits in L1: give it everything the kernel's shared memory does not need
     e = smem_carveout_for((const void*)kernel, pl.smem_bytes, carve[wide]);
     if (e != cudaSuccess) return e;
-    {
-        const long long n = std::max<long long>((long long)s.Cout * pl.k.U * 8, pl.k.tiles);
-        dcn_wperm_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>((const bf16*)w, wperm, s, pl.k.nq, pl.k.U,
-                                                                       counters, pl.k.tiles);
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-    }
     TsArgs ta;
     FwdArgs& a = ta.f;
     a = FwdArgs{};
@@ -735,6 +751,17 @@ cudaError_t fwd_ts(const Shape& s, const void* x, const void* off, const void* m
     a.b_stage_bytes = pl.b_stage_bytes;
     ta.b_stages = pl.b_stages;
     ta.idle_bytes = pl.idle_bytes;
+    TapRec* recs = reinterpret_cast<TapRec*>(wsb + pl.ws_recs_off);
+    ta.recs = recs;
+    {
+        const long long nw = std::max<long long>((long long)s.Cout * pl.k.U * 8, pl.k.tiles);
+        const int wblocks = (int)((nw + 255) / 256);
+        const long long rblocks = (pl.nrec + 255) / 256;
+        dcn_fwd_prepass_kernel<<<(unsigned)(wblocks + rblocks), 256, 0, st>>>((const bf16*)w, wperm, recs, a, wblocks,
+                                                                             pl.nrec);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
     kernel<<<pl.k.ctas, NUM_THREADS, pl.smem_bytes, st>>>(map, ta);
     if (launches) *launches += 2;
     return cudaGetLastError();

@@ -153,9 +153,10 @@ DCN_API int dcn_backward_weight(const dcn_params_t* params, const void* x, const
  * during steady-state work because cudaMalloc can synchronize the device.
  *
  * Same arguments, layouts and results as dcn_forward, without workspace. Where
- * the forward needs scratch (the tensor-core path keeps float32 partial tiles
- * and per-tile counters there), it uses one static device array of
- * 40 MiB (41943040 bytes) compiled into the library; every GPU that loads the
+ * the forward needs scratch (the tensor-core path keeps float32 partial tiles,
+ * per-tile counters, a reordered copy of the weights and the sampling records
+ * there), it uses one static device array of
+ * 48 MiB (50331648 bytes) compiled into the library; every GPU that loads the
  * library holds that array until the process exits. Shapes whose scratch
  * would exceed it are rejected with DCN_ERR_WORKSPACE and a message giving
  * both sizes, before anything is enqueued. The tile counters are cleared on

@@ -81,9 +81,9 @@ def test_noalloc_refuses_shapes_beyond_its_scratch():
     s = gen.WORKLOADS["conv5_d2g4"].shape          # 512 output channels: about 78 MB of partial tiles
     d = _dev(gen.make_inputs(gen.WORKLOADS["conv5_d2g4"]))
     p = dcn._params(d["x"], d["weight"], d["offset"], s.stride, s.pad, s.dil, False)
-    if dcn.workspace_size(p, dcn.OP_FORWARD) <= 40 << 20:
+    if dcn.workspace_size(p, dcn.OP_FORWARD) <= 48 << 20:
         pytest.skip("this GPU's plan for the layer fits the static scratch")
     y = torch.empty((s.B, s.Ho, s.Wo, s.Cout), dtype=torch.bfloat16, device="cuda")
     assert _noalloc(lib, s, d, y) == DCN_ERR_WORKSPACE
     msg = lib.dcn_last_error_string().decode()
-    assert "static array holds 41943040" in msg, msg
+    assert "static array holds 50331648" in msg, msg
