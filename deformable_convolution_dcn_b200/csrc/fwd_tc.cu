@@ -145,7 +145,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // issue cursor: the chunk whose loads are issued next
         int isi = 0, ik = 0, ik1 = 0, icur_g = -1, iepoch = 0;
         Chunk ich{0, 0, 0};
-        const TapRec* irecs = s_rec;
+        // shared-memory address of the current epoch's records: read with ld.shared,
+        // which does not queue behind the gathers in the global-load path
+        uint32_t irecs = ptx::smem_u32(s_rec);
         if (L.ns > 0) {
             const Seg s0 = seg_at(L, 0);
             ik = s0.k0;
@@ -159,11 +161,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint32_t cmask = cg < s.Cg ? 0xFu : 0u;
             const bool hi_ok = cg + 8 < s.Cg;      // upper 8 channels present (narrow loads only)
             const uint8_t* xc = reinterpret_cast<const uint8_t*>(a.x + ich.g * s.Cg + cg);
-            const TapRec rc = irecs[row * s.K2 + ich.tap];
-            w[0] = rc.w01_00;
-            w[1] = rc.w11_10;
-            const uint32_t vm = rc.vmask & cmask;
-            const uint8_t* p = xc + (long long)rc.base * cin2;
+            const uint4 rc = ptx::lds_v4(irecs + (uint32_t)((row * s.K2 + ich.tap) * (int)sizeof(TapRec)));
+            w[0] = rc.x;  // TapRec::w01_00
+            w[1] = rc.y;  // TapRec::w11_10
+            const uint32_t vm = rc.w & cmask;  // TapRec::vmask
+            const uint8_t* p = xc + (long long)(int)rc.z * cin2;  // TapRec::base
             const uint8_t* pc[4] = {p, p + cin2, p + rp2, p + rp2 + cin2};
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -196,7 +198,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const int b = iepoch & 1;
                 const uint32_t par = (uint32_t)(b ? (iepoch >> 1) : ((iepoch >> 1) - 1)) & 1u;
                 if (!ptx::mbar_wait(ptx::smem_u32(&rec_full[b]), par, s_abort, a.status, WAIT_LIMIT)) return false;
-                irecs = s_rec + b * BM * s.K2;
+                irecs = ptx::smem_u32(s_rec + b * BM * s.K2);
                 icur_g = ich.g;
             }
             return true;

@@ -276,6 +276,11 @@ def _tf32_split_applies(s):
     (gen.LayerShape(B=2, Cin=2, H=6, W=9, Cout=16, K=3, stride=1, pad=1, G=2), True),
     (gen.LayerShape(B=3, Cin=6, H=8, W=8, Cout=128, K=1, stride=1, pad=0, G=3), True),
     (gen.LayerShape(B=1, Cin=4, H=31, W=17, Cout=64, K=3, stride=2, pad=0), True),
+    # input rows staged in shared memory (a map row a whole number of 16 bytes), CTAs spanning two images
+    (gen.LayerShape(B=2, Cin=3, H=40, W=32, Cout=64, K=3, stride=1, pad=1), True),
+    (gen.LayerShape(B=1, Cin=3, H=12, W=16, Cout=64, K=3, stride=2, pad=1), True),
+    # more than three 128-row tiles per CTA: several rounds
+    (gen.LayerShape(B=1, Cin=1, H=250, W=240, Cout=32, K=3, stride=1, pad=1), True),
 ], ids=lambda v: v if isinstance(v, bool) else "C%dx%dK%ds%dd%dG%d" % (v.Cin, v.Cout, v.K, v.stride, v.dil, v.G))
 def test_small_channel_f32_layers(shape, mask, kernel):
     """Float32 layers with few input channels, compared in full: the split-tf32
