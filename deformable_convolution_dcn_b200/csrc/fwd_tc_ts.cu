@@ -90,6 +90,8 @@ __global__ void __launch_bounds__(256) dcn_fwd_prepass_kernel(const bf16* __rest
                                                               TapRec* __restrict__ recs, const FwdArgs a, int wblocks,
                                                               long long nrec) {
     const Shape& s = a.s;
+    // the main kernel may be scheduled now; it waits for this grid's completion before reading its outputs
+    asm volatile("griddepcontrol.launch_dependents;");
     if ((int)blockIdx.x >= wblocks) {
         const long long r = (long long)(blockIdx.x - wblocks) * blockDim.x + threadIdx.x;
         if (r >= nrec) return;
@@ -198,13 +200,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = *s_tmem;
+    // Launched as a programmatic dependent of the pre-pass: everything above
+    // (barriers, TMEM, the stream-K plan) overlapped its tail; the records, W'
+    // and the tile counters it writes are read only after this point.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     const int cta = blockIdx.x;
     const long long ubeg = s_starts[cta], uend = s_starts[cta + 1];
     const SegList L = seg_list(ubeg, uend, a.U);
     if (warp >= PROD_WARP0) {
         // ------------------------------------------------------ producers --
-        const int ptid = threadIdx.x - PROD_WARP0 * 32;
         const int rb = 32 * (warp & 3) + 16 * ((warp - PROD_WARP0) >> 2);  // this warp's 16 TMEM lanes (rows)
         const int j4 = lane & 3;
         const int r0 = rb + (lane >> 2), r1 = r0 + 8;
@@ -764,7 +769,18 @@ cudaError_t fwd_ts(const Shape& s, const void* x, const void* off, const void* m
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    kernel<<<pl.k.ctas, NUM_THREADS, pl.smem_bytes, st>>>(map, ta);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)pl.k.ctas);
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = pl.smem_bytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kernel, map, ta);
+    if (e != cudaSuccess) return e;
     if (launches) *launches += 2;
     return cudaGetLastError();
 }
