@@ -285,6 +285,49 @@ __global__ void __launch_bounds__(256) bias_grad_kernel(Shape s, const T* __rest
     atomicAdd(gb + o, acc);
 }
 
+// grad_bias with 16-byte loads: a block takes a slice of pixels; its threads
+// form rows x groups, each thread one group of V = 16 / sizeof(T) channels and
+// every rows-th pixel of the slice; the rows are summed in shared memory and
+// one atomic per channel and block adds the slice into grad_bias.
+template <typename T>
+__global__ void __launch_bounds__(256) bias_grad_vec_kernel(Shape s, const T* __restrict__ gy, float* __restrict__ gb,
+                                                            int pix_per_block) {
+    constexpr int V = 16 / (int)sizeof(T);
+    __shared__ float red[256 * V];
+    const int groups = s.Cout / V, rows = 256 / groups;
+    const int t = threadIdx.x, g = t % groups, pr = t / groups;
+    const int pbeg = blockIdx.x * pix_per_block, pend = min(s.P, pbeg + pix_per_block);
+    float acc[V];
+#pragma unroll
+    for (int v = 0; v < V; ++v) acc[v] = 0.f;
+    if (pr < rows) {
+        for (int p = pbeg + pr; p < pend; p += rows) {
+            const uint4 q = __ldg(reinterpret_cast<const uint4*>(gy + (size_t)p * s.Cout) + g);
+            if constexpr (sizeof(T) == 2) {
+                const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    acc[2 * i] += __uint_as_float(w[i] << 16);
+                    acc[2 * i + 1] += __uint_as_float(w[i] & 0xFFFF0000u);
+                }
+            } else {
+                acc[0] += __uint_as_float(q.x);
+                acc[1] += __uint_as_float(q.y);
+                acc[2] += __uint_as_float(q.z);
+                acc[3] += __uint_as_float(q.w);
+            }
+        }
+#pragma unroll
+        for (int v = 0; v < V; ++v) red[pr * s.Cout + g * V + v] = acc[v];
+    }
+    __syncthreads();
+    for (int o = t; o < s.Cout; o += 256) {
+        float sum = 0.f;
+        for (int r = 0; r < rows; ++r) sum += red[r * s.Cout + o];
+        atomicAdd(gb + o, sum);
+    }
+}
+
 // ------------------------------------------------------------- launchers --
 
 static int splits_for(int P, int tiles, int per_block_min) {
@@ -347,6 +390,17 @@ cudaError_t generic_backward_weight(const Shape& s, int dtype, const void* x, co
 }
 
 cudaError_t bias_grad(const Shape& s, int dtype, const void* gy, float* gb, cudaStream_t st) {
+    const int esz = dtype == 0 ? 4 : 2, V = 16 / esz;
+    if ((reinterpret_cast<uintptr_t>(gy) & 15) == 0 && s.Cout % V == 0 && s.Cout / V <= 256 && s.P > 0) {
+        const int blocks = std::min<long long>(2 * 148, s.P);
+        const int per_block = (int)((s.P + blocks - 1) / blocks);
+        const int nb = (int)((s.P + per_block - 1) / per_block);
+        if (dtype == 0)
+            bias_grad_vec_kernel<float><<<nb, 256, 0, st>>>(s, (const float*)gy, gb, per_block);
+        else
+            bias_grad_vec_kernel<bf16><<<nb, 256, 0, st>>>(s, (const bf16*)gy, gb, per_block);
+        return cudaGetLastError();
+    }
     const int per = 64;
     dim3 g2((s.Cout + 255) / 256, (s.P + per - 1) / per);
     if (dtype == 0)
