@@ -29,7 +29,12 @@ __all__ = [
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-_LIB_PATH = os.path.join(_PKG, "libdcn_b200.so")
+# DCN_B200_LIB names another build of the library to load instead (e.g. the
+# range-checked libdcn_b200_checked.so); it must sit in this package directory.
+_LIB_NAME = os.environ.get("DCN_B200_LIB", "libdcn_b200.so")
+if os.path.basename(_LIB_NAME) != _LIB_NAME or not _LIB_NAME.startswith("libdcn_b200"):
+    raise ImportError("DCN_B200_LIB must name a libdcn_b200*.so file of the package directory, got %r" % _LIB_NAME)
+_LIB_PATH = os.path.join(_PKG, _LIB_NAME)
 _HEADER = os.path.join(os.path.dirname(_PKG), "include", "dcn.h")
 _lock = threading.Lock()
 _lib = None
@@ -37,6 +42,7 @@ _lib = None
 DCN_F32, DCN_BF16 = 0, 1
 DCN_FLAG_GENERIC = 0x1
 DCN_FLAG_NO_TF32 = 0x2
+DCN_ERR_TIMEOUT, DCN_ERR_RANGE = -4, -6
 OP_FORWARD, OP_BACKWARD_DATA, OP_BACKWARD_WEIGHT = 0, 1, 2
 _DTYPES = {torch.float32: DCN_F32, torch.bfloat16: DCN_BF16}
 
@@ -167,7 +173,9 @@ def check_status(stream=None):
     """Waits for `stream` (a torch.cuda.Stream; default: the current stream of
     the current device) and takes the device status word, raising DcnError
     (code -4, DCN_ERR_TIMEOUT) if a kernel of the library gave up a bounded wait
-    since the word was last taken. Other streams are not waited for."""
+    since the word was last taken, or (range-checked build) code -6,
+    DCN_ERR_RANGE, if a checked access fell outside its buffer. Other streams
+    are not waited for."""
     s = torch.cuda.current_stream() if stream is None else stream
     _check(_load().dcn_check_status(ctypes.c_void_p(s.cuda_stream)))
 

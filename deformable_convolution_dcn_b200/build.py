@@ -77,7 +77,24 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
     return LIBOUT
 
 
+CHECKED_LIB = os.path.join(os.path.dirname(LIB), "libdcn_b200_checked.so")
+CHECKED_BUILD = os.path.join(BUILD, "checked")
+
+
+def build_checked(force: bool = False, verbose: bool = False) -> str:
+    """The range-checked build (DCN_CHECKED): every indexed global access of the
+    gather and scatter paths is checked against its buffer before it is made; an
+    access outside is skipped (a load reads zeros) and recorded in the device
+    status word, which dcn_check_status reports as DCN_ERR_RANGE. Load it with
+    DCN_B200_LIB=libdcn_b200_checked.so."""
+    return build(force=force, verbose=verbose, defines=["DCN_CHECKED"], out=CHECKED_LIB, build_dir=CHECKED_BUILD)
+
+
 if __name__ == "__main__":
     # --nvtx: rebuild the library with NVTX ranges around its entry points (--force goes back)
-    print(build(force="--force" in sys.argv or "--nvtx" in sys.argv, verbose="-v" in sys.argv,
-                ptxas_verbose="--ptxas" in sys.argv, defines=["DCN_NVTX"] if "--nvtx" in sys.argv else ()))
+    # --checked: build libdcn_b200_checked.so (range-checked accesses) beside the library
+    if "--checked" in sys.argv:
+        print(build_checked(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    else:
+        print(build(force="--force" in sys.argv or "--nvtx" in sys.argv, verbose="-v" in sys.argv,
+                    ptxas_verbose="--ptxas" in sys.argv, defines=["DCN_NVTX"] if "--nvtx" in sys.argv else ()))

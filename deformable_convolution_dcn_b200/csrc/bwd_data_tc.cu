@@ -196,6 +196,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int plane = s.Ho * s.Wo;
         float* tb = reinterpret_cast<float*>(smem + a.stages * stage_bytes + 1024) + warp * 32 * TPITCH;
         const int pq = lane >> 3, cj = lane & 7;  // pixel within a group of 4, 4-channel slot
+#ifdef DCN_CHECKED
+        const size_t xbytes = (size_t)s.B * s.H * s.W * s.Cin * sizeof(bf16);  // range-checked build
+        const size_t gxbytes = (size_t)s.B * s.H * s.W * s.Cin * sizeof(float);
+#endif
         int seg = 0;
         bool ok = true;
         for (long long u = ubeg; u < uend && ok; ++u, ++seg) {
@@ -250,11 +254,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const float4 Gv = *reinterpret_cast<const float4*>(tb + src * TPITCH + 4 * cj);
                     const long long o00 = base + cc + 4 * cj;
                     const long long o01 = o00 + s.Cin, o10 = o00 + (long long)s.W * s.Cin, o11 = o10 + s.Cin;
+#ifdef DCN_CHECKED
+                    uint32_t flc = fl;
+                    {
+                        const long long oc[4] = {o00, o01, o10, o11};
+                        for (int c = 0; c < 4; ++c)
+                            if (((flc >> c) & 1u) &&
+                                !(ptx::in_range(a.x + oc[c], 8, a.x, xbytes, a.status) &&
+                                  (!a.gx || ptx::in_range(a.gx + oc[c], 16, a.gx, gxbytes, a.status))))
+                                flc &= ~(1u << c);
+                    }
+#else
+                    const uint32_t flc = fl;
+#endif
                     const uint2 z = make_uint2(0, 0);
-                    const uint2 v00 = (fl & 1u) ? ptx::ldg_v2(a.x + o00) : z;
-                    const uint2 v01 = (fl & 2u) ? ptx::ldg_v2(a.x + o01) : z;
-                    const uint2 v10 = (fl & 4u) ? ptx::ldg_v2(a.x + o10) : z;
-                    const uint2 v11 = (fl & 8u) ? ptx::ldg_v2(a.x + o11) : z;
+                    const uint2 v00 = (flc & 1u) ? ptx::ldg_v2(a.x + o00) : z;
+                    const uint2 v01 = (flc & 2u) ? ptx::ldg_v2(a.x + o01) : z;
+                    const uint2 v10 = (flc & 4u) ? ptx::ldg_v2(a.x + o10) : z;
+                    const uint2 v11 = (flc & 8u) ? ptx::ldg_v2(a.x + o11) : z;
                     const float w00 = (1.f - ly) * (1.f - lx), w01 = (1.f - ly) * lx, w10 = ly * (1.f - lx), w11 = ly * lx;
                     const float Gc[4] = {Gv.x, Gv.y, Gv.z, Gv.w};
                     float r00[4], r01[4], r10[4], r11[4];
@@ -275,10 +292,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         r11[h] = gmc * w11;
                     }
                     if (a.gx) {
-                        if (fl & 1u) ptx::red_add_v4(a.gx + o00, r00[0], r00[1], r00[2], r00[3]);
-                        if (fl & 2u) ptx::red_add_v4(a.gx + o01, r01[0], r01[1], r01[2], r01[3]);
-                        if (fl & 4u) ptx::red_add_v4(a.gx + o10, r10[0], r10[1], r10[2], r10[3]);
-                        if (fl & 8u) ptx::red_add_v4(a.gx + o11, r11[0], r11[1], r11[2], r11[3]);
+                        if (flc & 1u) ptx::red_add_v4(a.gx + o00, r00[0], r00[1], r00[2], r00[3]);
+                        if (flc & 2u) ptx::red_add_v4(a.gx + o01, r01[0], r01[1], r01[2], r01[3]);
+                        if (flc & 4u) ptx::red_add_v4(a.gx + o10, r10[0], r10[1], r10[2], r10[3]);
+                        if (flc & 8u) ptx::red_add_v4(a.gx + o11, r11[0], r11[1], r11[2], r11[3]);
                     }
                 }
             }

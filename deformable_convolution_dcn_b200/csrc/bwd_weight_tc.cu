@@ -176,6 +176,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         uint32_t m = ((r[i].x & 0xFFFFu) ? 1u : 0u) | ((r[i].x >> 16) ? 2u : 0u) |
                                      ((r[i].y & 0xFFFFu) ? 4u : 0u) | ((r[i].y >> 16) ? 8u : 0u);
                         if (!cval) m = 0;
+#ifdef DCN_CHECKED
+                        {  // range-checked build: a neighbour load outside x is skipped (zeros) and recorded
+                            const size_t xbytes = (size_t)s.B * s.H * s.W * s.Cin * sizeof(bf16);
+                            const bf16* q[4] = {pb, pb + s.Cin, pb + rowpitch, pb + rowpitch + s.Cin};
+                            for (int c = 0; c < 4; ++c)
+                                if (((m >> c) & 1u) && !ptx::in_range(q[c], 16, a.x, xbytes, a.status)) m &= ~(1u << c);
+                        }
+#endif
                         ptx::ldg4_pred(v[i], pb, pb + s.Cin, pb + rowpitch, pb + rowpitch + s.Cin, m);
                     }
 #pragma unroll

@@ -559,6 +559,8 @@ int dcn_check_status(void* stream) {
     cudaError_t e = dcn::read_and_clear_status(&st, (cudaStream_t)stream);
     g_launches += 1;
     if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+    if (st & 2u)  // kStatusRange
+        return fail(DCN_ERR_RANGE, "a device access fell outside its buffer and was skipped (status 0x%x)", st);
     if (st) return fail(DCN_ERR_TIMEOUT, "a kernel gave up a bounded wait (status 0x%x)", st);
     return ok();
 }

@@ -133,6 +133,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t swz1 = (uint32_t)(((2 * j4 + 1) ^ (r0 & 7)) << 4);  // chunk 2*j4 + 1
         const long long cin2 = (long long)s.Cin * 2, rp2 = (long long)s.W * cin2;
         const uint8_t* zb = reinterpret_cast<const uint8_t*>(g_zero_slice);
+#ifdef DCN_CHECKED
+        const size_t xbytes = (size_t)s.B * s.H * s.W * s.Cin * sizeof(bf16);  // range-checked build
+#endif
         bool ok = true;
         // the first epoch's records are built by all warps together
         if (L.ns > 0) {
@@ -169,7 +172,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint8_t* pc[4] = {p, p + cin2, p + rp2, p + rp2 + cin2};
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
+#ifdef DCN_CHECKED
+                const bool rd = ((vm >> c) & 1u) &&
+                                ptx::in_range(pc[c], (WIDE || hi_ok) ? 32 : 16, a.x, xbytes, a.status);
+#else
                 const bool rd = (vm >> c) & 1u;
+#endif
                 load_slice<WIDE>(v[c], rd ? pc[c] : zb, (rd && hi_ok) ? pc[c] + 16 : zb);
             }
         };

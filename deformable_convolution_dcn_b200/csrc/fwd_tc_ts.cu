@@ -216,6 +216,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t t_row = tmem_base + ((uint32_t)rb << 16) + (uint32_t)A_COL;
         const long long cin2 = (long long)s.Cin * 2, rp2 = (long long)s.W * cin2;
         const uint8_t* zb = reinterpret_cast<const uint8_t*>(g_zero_slice);
+#ifdef DCN_CHECKED
+        const size_t xbytes = (size_t)s.B * s.H * s.W * s.Cin * sizeof(bf16);  // range-checked build
+#endif
         bool ok = true;
         // the first epoch's records (copied in by the epilogue side)
         if (L.ns > 0)
@@ -246,7 +249,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint8_t* pc[4] = {p, p + cin2, p + rp2, p + rp2 + cin2};
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
+#ifdef DCN_CHECKED
+                const bool rd = ((vm >> c) & 1u) &&
+                                ptx::in_range(pc[c], (WIDE || hi_ok) ? 32 : 16, a.x, xbytes, a.status);
+#else
                 const bool rd = (vm >> c) & 1u;
+#endif
                 load_slice<WIDE>(v[c], rd ? pc[c] : zb, (rd && hi_ok) ? pc[c] + 16 : zb);
             }
         };

@@ -12,8 +12,22 @@
 namespace dcn {
 namespace ptx {
 
-// Status bits recorded in the device status word when a bounded wait gives up.
+// Status bits recorded in the device status word: a bounded wait gave up; an
+// access of the range-checked build (DCN_CHECKED) fell outside its buffer.
 constexpr unsigned kStatusTimeout = 1u;
+constexpr unsigned kStatusRange = 2u;
+
+// Range check of the DCN_CHECKED build: true when [p, p + bytes) lies inside
+// [base, base + size); otherwise records kStatusRange and returns false, so
+// that the caller skips the access (or reads a zero slice instead). Without
+// DCN_CHECKED it is not compiled in and every call site reduces to the access.
+__device__ __forceinline__ bool in_range(const void* p, size_t bytes, const void* base, size_t size,
+                                         unsigned* status) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p), b = reinterpret_cast<uintptr_t>(base);
+    const bool ok = a >= b && a + bytes <= b + size;
+    if (!ok && status) atomicOr(status, kStatusRange);
+    return ok;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -80,6 +80,8 @@ typedef enum {
 #define DCN_ERR_CUDA (-3)        /* a CUDA call or launch failed; the message names it */
 #define DCN_ERR_TIMEOUT (-4)     /* a bounded device wait ran out (reported by dcn_check_status) */
 #define DCN_ERR_WORKSPACE (-5)   /* workspace NULL or smaller than dcn_workspace_size() */
+#define DCN_ERR_RANGE (-6)       /* range-checked build only: a device access fell outside its buffer and was
+                                    skipped (reported by dcn_check_status) */
 
 /* dcn_params_t.flags */
 #define DCN_FLAG_GENERIC 0x1u    /* use the generic CUDA-core kernels even where a specialised kernel exists */
@@ -249,8 +251,10 @@ DCN_API const char* dcn_last_error_string(void);
  * on the device, whichever stream launched it; a kernel still running on
  * another stream may report after this call. Returns DCN_OK, or
  * DCN_ERR_TIMEOUT if a kernel gave up a bounded wait since the word was last
- * taken, or DCN_ERR_CUDA if the stream reported an error. Enqueues one kernel
- * (counted by dcn_launch_count). */
+ * taken, or (range-checked build only, see DCN_ERR_RANGE) DCN_ERR_RANGE if a
+ * checked device access fell outside its buffer and was skipped, or
+ * DCN_ERR_CUDA if the stream reported an error. Enqueues one kernel (counted
+ * by dcn_launch_count). */
 DCN_API int dcn_check_status(void* stream);
 
 /* Failure-detection self-test (no counterpart on the pages): enqueues one

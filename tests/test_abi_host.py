@@ -33,6 +33,29 @@ def test_exports_every_header_symbol(lib):
     assert lib.dcn_abi_version() == 2
 
 
+def test_checked_build_exports_every_header_symbol():
+    """The range-checked build (DCN_CHECKED) is the same library with checks
+    compiled into its gather and scatter accesses: same entry points, same ABI."""
+    import os
+    from deformable_convolution_dcn_b200 import build
+    path = build.build_checked()
+    assert os.path.basename(path) == "libdcn_b200_checked.so"
+    chk = ctypes.CDLL(path)
+    for n in dcn.header_symbols():
+        assert hasattr(chk, n), n
+    chk.dcn_abi_version.restype = ctypes.c_int
+    assert chk.dcn_abi_version() == 2
+
+
+def test_library_override_is_restricted_to_package_builds():
+    import subprocess
+    import sys
+    for bad in ("../evil.so", "/tmp/libdcn_b200.so", "libother.so"):
+        r = subprocess.run([sys.executable, "-c", "import deformable_convolution_dcn_b200"], capture_output=True,
+                           text=True, env={**__import__("os").environ, "DCN_B200_LIB": bad})
+        assert r.returncode != 0 and "DCN_B200_LIB" in r.stderr, bad
+
+
 @pytest.mark.parametrize("H,W,K,stride,pad,dil,expect", [
     (224, 224, 3, 1, 1, 1, (224, 224)), (200, 200, 3, 2, 1, 1, (100, 100)), (25, 25, 3, 1, 2, 2, (25, 25)),
     (50, 50, 3, 1, 1, 1, (50, 50)), (7, 5, 5, 2, 0, 1, (2, 1)), (1, 1, 3, 1, 1, 1, (1, 1)), (6, 6, 2, 1, 0, 1, (5, 5)),
