@@ -71,9 +71,17 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
         : "memory");
 }
 
+// Records epochs: a layer with at most ALL_TAPS taps keeps all taps of one
+// (tile, group) in a record buffer (one epoch = the group's nq * K*K chunks);
+// a larger kernel (K = 6, 7) keeps one row of K taps (one epoch = K chunks).
+constexpr int ALL_TAPS = 25;
+constexpr int MAX_TAPS_TS = 49;
+constexpr int TAP_TABLE = 64;  // entries of the shared-memory tap table
+
 struct TsArgs {
     FwdArgs f;
     const TapRec* recs;   // [m tiles][G][K*K][BM] sampling records (workspace), tap-major
+    int ep_len, ep_taps;  // chunks per records epoch, taps held per record buffer
     int b_stages;
     uint32_t idle_bytes;  // shared memory free after the last MMA (the weight ring)
 };
@@ -140,7 +148,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint8_t* sB = smem;  // weight ring: b_stages x [N x 128 B], 128-byte swizzle
     TapRec* s_rec = reinterpret_cast<TapRec*>(smem + a.info_off);  // two buffers of BM * K2 records
     int2* s_tap = reinterpret_cast<int2*>(smem + a.row_off);        // per tap: (i*dil, j*dil)
-    long long* s_starts = reinterpret_cast<long long*>(s_tap + 32);   // [ctas + 1] first unit of each CTA
+    long long* s_starts = reinterpret_cast<long long*>(s_tap + TAP_TABLE);  // [ctas + 1] first unit of each CTA
     float* s_bias = reinterpret_cast<float*>(s_starts + MAX_CTAS + 2);  // [2][512] bias of a tile's columns
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + a.bar_off);
     uint64_t* a_full = bars;                      // [A_STAGES] every producer warp stored the chunk
@@ -223,7 +231,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // the first epoch's records (copied in by the epilogue side)
         if (L.ns > 0)
             ok = __all_sync(0xffffffffu, ptx::mbar_wait(ptx::smem_u32(&rec_full[0]), 0, s_abort, a.status, WAIT_LIMIT));
-        int isi = 0, ik = 0, ik1 = 0, icur_g = -1, iepoch = 0;
+        int isi = 0, ik = 0, ik1 = 0, iepoch = 0;
+        int ileft = 0, irb = 0;  // chunks left in the records epoch; first tap held by the record buffer
         Chunk ich{0, 0, 0};
         // shared-memory address of the current epoch's records: read with ld.shared,
         // which does not queue behind the gathers in the global-load path
@@ -233,7 +242,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ik = s0.k0;
             ik1 = s0.k1;
             ich = chunk_of(ik, a);
-            icur_g = ich.g;
+            ileft = ta.ep_len - ik % ta.ep_len;
+            irb = ta.ep_taps == s.K2 ? 0 : ich.tap - ich.tap % s.K;
         }
         // loads of row `row` of the cursor chunk into v, its weights into w
         auto issue = [&](uint32_t(&v)[4][8], uint32_t(&w)[2], int row) {
@@ -241,7 +251,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint32_t cmask = cg < s.Cg ? 0xFu : 0u;
             const bool hi_ok = cg + 8 < s.Cg;  // upper 8 channels present (narrow loads only)
             const uint8_t* xc = reinterpret_cast<const uint8_t*>(a.x + ich.g * s.Cg + cg);
-            const uint4 rc = ptx::lds_v4(irecs + (uint32_t)((ich.tap * BM + row) * (int)sizeof(TapRec)));
+            const uint4 rc = ptx::lds_v4(irecs + (uint32_t)(((ich.tap - irb) * BM + row) * (int)sizeof(TapRec)));
             w[0] = rc.x;  // TapRec::w01_00
             w[1] = rc.y;  // TapRec::w11_10
             const uint32_t vm = rc.w & cmask;  // TapRec::vmask
@@ -267,14 +277,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     ++ich.g;
                 }
             }
+            bool new_epoch = --ileft == 0;
             if (ik == ik1) {
                 const Seg sn = seg_at(L, ++isi);
                 ik = sn.k0;
                 ik1 = sn.k1;
                 ich = chunk_of(ik, a);
-                icur_g = -1;
+                ileft = ta.ep_len - ik % ta.ep_len;
+                new_epoch = true;
+            } else if (new_epoch) {
+                ileft = ta.ep_len;
             }
-            if (ich.g != icur_g) {
+            if (new_epoch) {
+                irb = ta.ep_taps == s.K2 ? 0 : ich.tap - ich.tap % s.K;
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&rec_empty[iepoch & 1]));
                 ++iepoch;
@@ -284,8 +299,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 if (!__all_sync(0xffffffffu, ptx::mbar_wait(ptx::smem_u32(&rec_full[b]), par, s_abort, a.status,
                                                             WAIT_LIMIT)))
                     return false;
-                irecs = ptx::smem_u32(s_rec + b * BM * s.K2);
-                icur_g = ich.g;
+                irecs = ptx::smem_u32(s_rec + b * BM * ta.ep_taps);
             }
             return true;
         };
@@ -487,7 +501,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // segment, so the order cannot deadlock.
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
-        const int per_g = a.nq * s.K2;
+        const int per_g = a.nq * s.K2;  // chunks per group within a tile
         uint32_t ephase = 0;
         int rec_epoch = 0;
         int rseg = 0, rk = L.ns > 0 ? seg_at(L, 0).k0 : 0;
@@ -498,7 +512,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             while (rseg < L.ns && (rseg <= seg || (rseg == seg + 1 && rk == seg_at(L, rseg).k0))) {
                 const Seg rs = seg_at(L, rseg);
                 const int b = rec_epoch & 1;
-                const int rg = rk / per_g;
+                const int re = rk / ta.ep_len;  // epoch within the tile
+                const int rg = (re * ta.ep_len) / per_g, rt = ta.ep_taps == s.K2 ? 0 : ((re * ta.ep_len) % s.K2);
                 if (threadIdx.x == 0) {
                     // buffer b is free once every producer warp has left epoch rec_epoch - 2
                     if (rec_epoch >= 2 && !ptx::mbar_wait(ptx::smem_u32(&rec_empty[b]), ((rec_epoch - 2) >> 1) & 1,
@@ -506,16 +521,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         ok = false;
                     } else {
                         ptx::fence_proxy_async_smem();  // the producers' reads before the copy's writes
-                        const uint32_t bytes = (uint32_t)(BM * s.K2 * sizeof(TapRec));
+                        const uint32_t bytes = (uint32_t)(BM * ta.ep_taps * sizeof(TapRec));
                         const uint32_t fb = ptx::smem_u32(&rec_full[b]);
                         ptx::mbar_arrive_expect_tx(fb, bytes);
-                        ptx::bulk_load(ptx::smem_u32(s_rec + b * BM * s.K2),
-                                       ta.recs + ((size_t)(rs.t / a.n_tiles) * s.G + rg) * s.K2 * BM, bytes, fb);
+                        ptx::bulk_load(ptx::smem_u32(s_rec + b * BM * ta.ep_taps),
+                                       ta.recs + (((size_t)(rs.t / a.n_tiles) * s.G + rg) * s.K2 + rt) * BM, bytes, fb);
                     }
                 }
                 if (warp == 0) ok = __shfl_sync(0xffffffffu, ok, 0);  // warp 0 stays convergent
                 if (!ok) break;
-                rk = min((rg + 1) * per_g, rs.k1);
+                rk = min((re + 1) * ta.ep_len, rs.k1);
                 if (rk >= rs.k1 && ++rseg < L.ns) rk = seg_at(L, rseg).k0;
                 ++rec_epoch;
             }
@@ -661,7 +676,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 struct TsPlan {
     bool ok;
     StreamK k;
-    int bn_total, b_stages, acc_cols;
+    int bn_total, b_stages, acc_cols, ep_len, ep_taps;
     uint32_t b_stage_bytes, info_off, row_off, bar_off, smem_bytes, idle_bytes;
     size_t ws_partials, ws_counters_off, ws_wperm_off, ws_recs_off, ws_bytes;
     long long nrec;
@@ -670,7 +685,7 @@ struct TsPlan {
 TsPlan make_ts_plan(const Shape& s, int sms) {
     TsPlan pl{};
     pl.ok = false;
-    if (s.Cin % 8 || s.Cg % 8 || s.Cout % 8 || s.K2 > 25 || s.Cout > 256) return pl;
+    if (s.Cin % 8 || s.Cg % 8 || s.Cout % 8 || s.K2 > MAX_TAPS_TS || s.Cout > 256) return pl;
     pl.bn_total = (s.Cout + 31) / 32 * 32;
     pl.k = plan_stream_k(s, pl.bn_total, sms);
     // two accumulators of <= 128 columns, or one of <= 256, below the A ring at column 256
@@ -678,10 +693,13 @@ TsPlan make_ts_plan(const Shape& s, int sms) {
     pl.b_stage_bytes = (uint32_t)pl.bn_total * 128;
     pl.b_stages = std::min(DCN_FWD_TS_B_STAGES, MAX_B_STAGES);
     const uint32_t ring = (uint32_t)pl.b_stages * pl.b_stage_bytes;
-    const uint32_t info_bytes = (uint32_t)(2 * BM * s.K2 * sizeof(TapRec));
+    pl.ep_taps = s.K2 <= ALL_TAPS ? s.K2 : s.K;
+    pl.ep_len = s.K2 <= ALL_TAPS ? pl.k.nq * s.K2 : s.K;
+    const uint32_t info_bytes = (uint32_t)(2 * BM * pl.ep_taps * sizeof(TapRec));
     pl.info_off = ring;
     pl.row_off = pl.info_off + info_bytes;
-    pl.bar_off = pl.row_off + (uint32_t)(32 * sizeof(int2) + (MAX_CTAS + 2) * sizeof(long long) + 2 * 512 * sizeof(float));
+    pl.bar_off = pl.row_off + (uint32_t)(TAP_TABLE * sizeof(int2) + (MAX_CTAS + 2) * sizeof(long long) +
+                                         2 * 512 * sizeof(float));
     pl.smem_bytes = pl.bar_off + (2 * A_STAGES + 2 * MAX_B_STAGES + 17) * 8 + 32 + 1024;
     pl.idle_bytes = ring;
     if (pl.smem_bytes > 227 * 1024) return pl;
@@ -766,6 +784,8 @@ cudaError_t fwd_ts(const Shape& s, const void* x, const void* off, const void* m
     a.b_stage_bytes = pl.b_stage_bytes;
     ta.b_stages = pl.b_stages;
     ta.idle_bytes = pl.idle_bytes;
+    ta.ep_len = pl.ep_len;
+    ta.ep_taps = pl.ep_taps;
     TapRec* recs = reinterpret_cast<TapRec*>(wsb + pl.ws_recs_off);
     ta.recs = recs;
     {

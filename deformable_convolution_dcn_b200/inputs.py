@@ -95,6 +95,9 @@ WORKLOADS = {
     "conv4_k5": Workload(
         "conv4_k5", LayerShape(B=8, Cin=256, H=50, W=50, Cout=256, K=5, pad=2), "bf16", seed=7,
         description="conv4-sized 5x5 DCNv2 forward bf16 (50 offset channels), B8 Cin=Cout=256 50x50 K5 s1 p2 G1"),
+    "conv4_k7": Workload(
+        "conv4_k7", LayerShape(B=8, Cin=256, H=50, W=50, Cout=256, K=7, pad=3), "bf16", seed=8,
+        description="conv4-sized 7x7 DCNv2 forward bf16 (98 offset channels), B8 Cin=Cout=256 50x50 K7 s1 p3 G1"),
     "conv4_bwd": Workload(
         "conv4_bwd", LayerShape(B=8, Cin=256, H=50, W=50, Cout=256), "bf16", seed=5,
         offset_dist="normal1.5_edges", backward=True,

@@ -210,6 +210,9 @@ F32, BF16 = 0, 1
     (dict(B=1, H=16, W=16, Cin=16, Cout=64, G=1, dtype=F32), 0, "generic"),
     # bfloat16: the tcgen05 gather kernel for channel counts in multiples of 8
     (dict(B=8, H=50, W=50, Cin=256, Cout=256, G=1, dtype=BF16), 0, "tcgen05_gather_tmem"),
+    # 7x7: records held one kernel row (seven taps) at a time
+    (dict(B=1, H=11, W=9, Cin=16, Cout=24, K=7, pad=3, G=1, dtype=BF16), 0, "tcgen05_gather_tmem"),
+    (dict(B=1, H=11, W=9, Cin=16, Cout=264, K=7, pad=3, G=1, dtype=BF16), 0, "generic"),
     (dict(B=8, H=50, W=50, Cin=256, Cout=256, G=1, dtype=BF16), dcn.DCN_FLAG_GENERIC, "generic"),
     (dict(B=8, H=25, W=25, Cin=512, Cout=512, G=4, pad=2, dil=2, dtype=BF16), 0, "tcgen05_gather"),
     (dict(B=1, H=9, W=9, Cin=12, Cout=16, G=1, dtype=BF16), 0, "generic"),

@@ -215,7 +215,9 @@ def test_full_size_backward_sampled():
     (gen.LayerShape(B=1, Cin=16, H=11, W=9, Cout=24, K=7, pad=3), True),
     (gen.LayerShape(B=2, Cin=32, H=9, W=14, Cout=16, K=7, pad=3, dil=1, G=2), False),
     (gen.LayerShape(B=1, Cin=8, H=16, W=10, Cout=8, K=7, stride=2, pad=6, dil=2), True),
-], ids=["k7", "k7_g2_v1", "k7_s2_d2"])
+    # two 64-channel slices, six tiles split over many CTAs: stream-K segments start inside a tap row
+    (gen.LayerShape(B=2, Cin=128, H=20, W=18, Cout=64, K=7, pad=3), True),
+], ids=["k7", "k7_g2_v1", "k7_s2_d2", "k7_c128"])
 def test_seven_by_seven_layers(shape, mask, dtype):
     """K = 7 (49 taps, 98 offset channels per group), DCNv2 and DCNv1, forward and backward in full."""
     w = gen.Workload("k7", shape, dtype, seed=17, offset_dist="uniform2.5",
