@@ -424,6 +424,55 @@ __global__ void __launch_bounds__(B_THREADS, 1)
     const int rend = blockIdx.x + 1 == gridDim.x ? s.P : (int)(8 * (p8 * (blockIdx.x + 1) / gridDim.x));
     const int rounds = rend > rbeg ? (rend - rbeg + B_ROWS - 1) / B_ROWS : 0;
     const int plane = s.Ho * s.Wo;
+    const int nch = (a.mask ? 3 : 2) * s.K2;
+
+    // a round's rows, and the input rows its samples reach when no offset moves
+    // them by more than the margin (within one image; otherwise no band)
+    struct Round {
+        int r0, nr, nt, b_first, b_last, yb0, yb1, pix0;
+        bool use_band, od_bulk;
+    };
+    auto round_of = [&](int rd) {
+        Round R;
+        R.r0 = rbeg + rd * B_ROWS;
+        R.nr = min(B_ROWS, rend - R.r0);
+        R.nt = (R.nr + S_BM - 1) / S_BM;
+        R.b_first = R.r0 / plane;
+        R.b_last = (R.r0 + R.nr - 1) / plane;
+        R.yb0 = 0;
+        R.yb1 = -1;
+        if (ba.band_ok && R.b_first == R.b_last) {
+            const int ho0 = (R.r0 - R.b_first * plane) / s.Wo, ho1 = (R.r0 + R.nr - 1 - R.b_first * plane) / s.Wo;
+            R.yb0 = max(0, ho0 * s.stride - s.pad - B_BAND_MARGIN);
+            R.yb1 = min(s.H - 1, ho1 * s.stride - s.pad + (s.K - 1) * s.dil + 1 + B_BAND_MARGIN);
+            if ((long long)(R.yb1 - R.yb0 + 1) * s.W * CIN * 4 > (long long)B_BAND_MAX) R.yb1 = R.yb0 - 1;
+        }
+        R.use_band = R.yb1 >= R.yb0;
+        R.pix0 = R.r0 - R.b_first * plane;
+        R.od_bulk = ba.od_ok && R.b_first == R.b_last && (R.pix0 & 3) == 0;
+        return R;
+    };
+    // one thread: the band copy and the offset/mask boxes of a round
+    auto stage_copies = [&](const Round& R) {
+        if (R.use_band) {
+            const uint32_t bytes = (uint32_t)(R.yb1 - R.yb0 + 1) * s.W * CIN * 4;
+            const uint8_t* src = reinterpret_cast<const uint8_t*>(a.x + ((size_t)R.b_first * s.H + R.yb0) * s.W * CIN);
+            ptx::fence_proxy_async_smem();
+            ptx::mbar_arrive_expect_tx(ptx::smem_u32(band_bar), bytes);
+            ptx::bulk_load(ptx::smem_u32(smem + ba.band_off), src, bytes, ptx::smem_u32(band_bar));
+        }
+        if (R.od_bulk) {
+            ptx::fence_proxy_async_smem();
+            ptx::mbar_arrive_expect_tx(ptx::smem_u32(od_bar), (uint32_t)(R.nt * nch * S_BM * 4));
+            for (int tl = 0; tl < R.nt; ++tl) {
+                const uint32_t dst = ptx::smem_u32(s_od + tl * ts);
+                ptx::tma_load_2d(dst, &tmap_off, ptx::smem_u32(od_bar), R.pix0 + tl * S_BM, R.b_first * 2 * s.K2);
+                if (a.mask)
+                    ptx::tma_load_2d(dst + (uint32_t)(2 * s.K2 * S_BM * 4), &tmap_mask, ptx::smem_u32(od_bar),
+                                     R.pix0 + tl * S_BM, R.b_first * s.K2);
+            }
+        }
+    };
 
     if (tid == 0) {
         ptx::mbar_init(ptx::smem_u32(wbar), 1);
@@ -432,6 +481,8 @@ __global__ void __launch_bounds__(B_THREADS, 1)
         ptx::mbar_init(ptx::smem_u32(od_bar), 1);
         *s_abort = 0;
         ptx::fence_mbar_init();
+        // round 0's inputs first: nothing else of the kernel needs to be ready for them
+        if (rounds > 0) stage_copies(round_of(0));
         if (a.w_bulk) {
             ptx::mbar_arrive_expect_tx(ptx::smem_u32(wbar), wbytes);
             for (uint32_t o = 0; o < wbytes; o += 16384u)
@@ -454,53 +505,20 @@ __global__ void __launch_bounds__(B_THREADS, 1)
     bool ok = true;
     uint8_t* sB = smem + a.b_off;
     int band_uses = 0, od_uses = 0;
-    const int nch = (a.mask ? 3 : 2) * s.K2;
     int mma_iss[B_TILES] = {}, mma_wt[B_TILES] = {};  // per tile slot: MMA commits issued, and waited for
     const uint32_t abase = ptx::smem_u32(smem + a.a_off);
     for (int rd = 0; rd < rounds; ++rd) {
-        const int r0 = rbeg + rd * B_ROWS;
-        const int nr = min(B_ROWS, rend - r0);
-        const int nt = (nr + S_BM - 1) / S_BM;
-        // the input rows this round's samples reach when no offset moves them by
-        // more than the margin (within one image); neighbours outside are read globally
-        const int b_first = r0 / plane, b_last = (r0 + nr - 1) / plane;
-        int yb0 = 0, yb1 = -1;
-        if (ba.band_ok && b_first == b_last) {
-            const int ho0 = (r0 - b_first * plane) / s.Wo, ho1 = (r0 + nr - 1 - b_first * plane) / s.Wo;
-            yb0 = max(0, ho0 * s.stride - s.pad - B_BAND_MARGIN);
-            yb1 = min(s.H - 1, ho1 * s.stride - s.pad + (s.K - 1) * s.dil + 1 + B_BAND_MARGIN);
-            if ((long long)(yb1 - yb0 + 1) * s.W * CIN * 4 > (long long)B_BAND_MAX) yb1 = yb0 - 1;
-        }
-        const bool use_band = yb1 >= yb0;
+        const Round R = round_of(rd);
+        const int r0 = R.r0, nr = R.nr, nt = R.nt, yb0 = R.yb0, yb1 = R.yb1;
+        const bool use_band = R.use_band, od_bulk = R.od_bulk;
         // the previous round's stores have read the staging tiles (the A tiles' memory)
-        // and every thread is done with the band
+        // and every thread is done with the band and the offsets
         if (rd > 0) {
             if (tid == 0) ptx::bulk_wait_group_read0();
             __syncthreads();
+            if (tid == 0) stage_copies(R);
         }
-        if (tid == 0 && use_band) {
-            const uint32_t bytes = (uint32_t)(yb1 - yb0 + 1) * s.W * CIN * 4;
-            const uint8_t* src = reinterpret_cast<const uint8_t*>(a.x + ((size_t)b_first * s.H + yb0) * s.W * CIN);
-            ptx::fence_proxy_async_smem();
-            ptx::mbar_arrive_expect_tx(ptx::smem_u32(band_bar), bytes);
-            ptx::bulk_load(ptx::smem_u32(smem + ba.band_off), src, bytes, ptx::smem_u32(band_bar));
-        }
-        // offsets and mask of the round's rows into s_od
-        const int pix0 = r0 - b_first * plane;
-        const bool od_bulk = ba.od_ok && b_first == b_last && (pix0 & 3) == 0;
-        if (od_bulk) {
-            if (tid == 0) {
-                ptx::fence_proxy_async_smem();
-                ptx::mbar_arrive_expect_tx(ptx::smem_u32(od_bar), (uint32_t)(nt * nch * S_BM * 4));
-                for (int tl = 0; tl < nt; ++tl) {
-                    const uint32_t dst = ptx::smem_u32(s_od + tl * ts);
-                    ptx::tma_load_2d(dst, &tmap_off, ptx::smem_u32(od_bar), pix0 + tl * S_BM, b_first * 2 * s.K2);
-                    if (a.mask)
-                        ptx::tma_load_2d(dst + (uint32_t)(2 * s.K2 * S_BM * 4), &tmap_mask, ptx::smem_u32(od_bar),
-                                         pix0 + tl * S_BM, b_first * s.K2);
-                }
-            }
-        } else {
+        if (!od_bulk) {  // the threads load the offsets themselves
             for (int e = tid; e < nch * nr; e += B_THREADS) {
                 const int ch = e / nr, r = e - ch * nr;
                 const int p = r0 + r, bb = p / plane, pix = p - bb * plane;
