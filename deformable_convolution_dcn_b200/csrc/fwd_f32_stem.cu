@@ -577,7 +577,7 @@ __global__ void __launch_bounds__(B_THREADS, 1)
                     float ly, lx;
                     split_coord(oy + ti * s.dil, dy, y0, ly);
                     split_coord(ox + tj * s.dil, dx, x0, lx);
-                    const bool yin0 = y0 >= 0 && y0 < s.H, yin1 = y0 + 1 >= 0 && y0 + 1 < s.H;
+                    bool yin0 = y0 >= 0 && y0 < s.H, yin1 = y0 + 1 >= 0 && y0 + 1 < s.H;
                     const bool xin0 = x0 >= 0 && x0 < s.W, xin1 = x0 + 1 >= 0 && x0 + 1 < s.W;
                     const float w00 = (yin0 && xin0) ? (1.f - ly) * (1.f - lx) * mk : 0.f;
                     const float w01 = (yin0 && xin1) ? (1.f - ly) * lx * mk : 0.f;
@@ -585,10 +585,34 @@ __global__ void __launch_bounds__(B_THREADS, 1)
                     const float w11 = (yin1 && xin1) ? ly * lx * mk : 0.f;
                     // clamped neighbour coordinates: a neighbour outside the map reads a valid
                     // pixel and is zeroed by its weight and the select below
-                    const int yc0 = min(max(y0, 0), s.H - 1), yc1 = min(max(y0 + 1, 0), s.H - 1);
-                    const int xc0 = min(max(x0, 0), s.W - 1), xc1 = min(max(x0 + 1, 0), s.W - 1);
+                    int yc0 = min(max(y0, 0), s.H - 1), yc1 = min(max(y0 + 1, 0), s.H - 1);
+                    int xc0 = min(max(x0, 0), s.W - 1), xc1 = min(max(x0 + 1, 0), s.W - 1);
                     float v[4][CIN];
-                    if (use_band && yc0 >= yb0 && yc1 <= yb1) {
+                    bool in_band = use_band && yc0 >= yb0 && yc1 <= yb1;
+#ifdef DCN_CHECKED
+                    {  // range-checked build: the band rows read lie inside the staged band, and the
+                       // neighbours read from global memory inside x
+                        const size_t band_bytes = use_band ? (size_t)(yb1 - yb0 + 1) * s.W * CIN * 4 : 0;
+                        const float* bandp = reinterpret_cast<const float*>(smem + ba.band_off);
+                        const size_t xbytes = (size_t)s.B * s.H * s.W * CIN * 4;
+                        const int cy[4] = {yc0, yc0, yc1, yc1}, cx[4] = {xc0, xc1, xc0, xc1};
+                        bool ok_band = true, ok_glob = true;
+                        for (int q = 0; q < 4; ++q) {
+                            if (in_band)
+                                ok_band = ok_band && ptx::in_range(bandp + ((size_t)(cy[q] - yb0) * s.W + cx[q]) * CIN,
+                                                                   CIN * 4, bandp, band_bytes, a.status);
+                            else
+                                ok_glob = ok_glob && ptx::in_range(xb + ((size_t)cy[q] * s.W + cx[q]) * CIN, CIN * 4,
+                                                                   a.x, xbytes, a.status);
+                        }
+                        if (!ok_band || !ok_glob) {  // skip the sample's neighbours: read pixel 0, add nothing
+                            yin0 = yin1 = false;
+                            in_band = false;
+                            yc0 = yc1 = xc0 = xc1 = 0;
+                        }
+                    }
+#endif
+                    if (in_band) {
                         const uint32_t r0a = band_u + (uint32_t)(((yc0 - yb0) * s.W) * CIN) * 4;
                         const uint32_t r1a = band_u + (uint32_t)(((yc1 - yb0) * s.W) * CIN) * 4;
 #pragma unroll
