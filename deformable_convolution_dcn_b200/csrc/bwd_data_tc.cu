@@ -18,6 +18,17 @@
 // group-tap block) are split evenly over one CTA per SM; the TMEM accumulator
 // is double-buffered so the epilogue of one unit overlaps the MMAs of the next.
 // All waits are bounded.
+//
+// A second epilogue (EPI = 1, layers whose channels per group are a multiple of
+// 64) works per pixel instead of per channel: with
+//   S_n = sum_c G[c] * x_n[c]   (n = the four bilinear neighbours),
+// the mask gradient is sum_n w_n S_n and the offset gradients are m times the
+// differences of the S_n weighted by the other coordinate's fractions, so each
+// (pixel, channel) costs four multiply-adds. W^T's rows are permuted so that the
+// 16x256b TMEM load hands each thread 16 contiguous channels of two pixels,
+// which are also one 32-byte load of each neighbour; no shared-memory
+// transpose. grad_x is scattered from here only for the neighbours flagged in
+// `ovf` (or all of them when no flags are given).
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -52,16 +63,43 @@ struct BdArgs {
     float* gx;
     float* goff;
     float* gmask;
+    const uint8_t* ovf;  // EPI 1: [G*K2][Ppad] neighbours (bit n) whose grad_x share is scattered here; null: all
     unsigned* status;
     int nblk, units_per_tile, m_tiles, ppad, ctas, stages, kchunks;
     long long total_units;
 };
+
+// 32 zero bytes: the source of every neighbour load that is not made (EPI 1).
+__device__ __align__(32) uint32_t g_bd_zero[8];
+
+// 16 TMEM lanes x 64 f32 columns from lane base `taddr` (16x256b shape, 8
+// repetitions): for repetition m, registers 4m and 4m+1 hold lane t/4, columns
+// 8m + 2(t%4) and 8m + 2(t%4) + 1, registers 4m+2 and 4m+3 lane t/4 + 8, the
+// same columns (t: the thread's lane in the warp). Valid after tmem_wait_ld.
+__device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x8.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+
+// MMA column k (0..63) of a 64-channel block holds channel perm64(k): the
+// 16x256b load then gives thread t%4 = j the channels 16j .. 16j + 15 in
+// register-pair order (see tmem_ld_16x256b_x8). inv_perm64 is its inverse.
+__host__ __device__ __forceinline__ int perm64(int k) { return 16 * ((k >> 1) & 3) + 2 * (k >> 3) + (k & 1); }
+__host__ __device__ __forceinline__ int inv_perm64(int c) { return 8 * ((c >> 1) & 7) + 2 * (c >> 4) + (c & 1); }
 
 __device__ __forceinline__ long long unit_begin(int c, const BdArgs& a) { return a.total_units * c / a.ctas; }
 
 __device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
+template <int EPI>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     dcn_bwd_data_tc_kernel(const __grid_constant__ CUtensorMap tmap_dy, const __grid_constant__ CUtensorMap tmap_wt,
                            const BdArgs a) {
@@ -185,6 +223,156 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ptx::mbar_wait(ptx::smem_u32(drain), 0, &dummy, a.status, WAIT_LIMIT);
         }
         __syncwarp();
+    } else if constexpr (EPI == 1) {
+        // --------------------------------------------- per-pixel epilogue --
+        // Warp w reads TMEM lanes rb .. rb + 15 (rb = 32 (w % 4) + 16 (w / 4));
+        // thread t handles tile rows rb + t/4 and rb + t/4 + 8 and, in every
+        // 64-column block, channels 16 (t % 4) .. + 15 of both.
+        const int rbase = (warp & 3) * 32 + (warp >> 2) * 16;
+        const int j = lane & 3;
+        const int plane = s.Ho * s.Wo;
+        const uint8_t* zb = reinterpret_cast<const uint8_t*>(g_bd_zero);
+        const long long cin = s.Cin;
+#ifdef DCN_CHECKED
+        const size_t xbytes = (size_t)s.B * s.H * s.W * s.Cin * sizeof(bf16);  // range-checked build
+        const size_t gxbytes = (size_t)s.B * s.H * s.W * s.Cin * sizeof(float);
+#endif
+        int seg = 0;
+        bool ok = true;
+        for (long long u = ubeg; u < uend && ok; ++u, ++seg) {
+            const int abuf = seg & 1;
+            const uint32_t aphase = (seg >> 1) & 1;
+            const int mt = (int)(u / a.units_per_tile), r = (int)(u - (long long)mt * a.units_per_tile);
+            const int gtap = r / a.nblk, cb = r - gtap * a.nblk;
+            const int g = gtap / s.K2, tap = gtap - g * s.K2;
+            const int c0 = cb * NT;
+            const int nb64 = min(NT, s.Cg - c0) >> 6;  // 64-channel blocks of this unit (Cg % 64 == 0)
+            // the two pixels' samples: fractions, mask, neighbours inside the map
+            float4 rc[2];
+            uint32_t fl[2], sc[2];
+            long long q00[2];
+            int pp[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int p = mt * BM + rbase + (lane >> 2) + 8 * h;
+                pp[h] = p;
+                rc[h] = make_float4(0.f, 0.f, 0.f, __uint_as_float(0xFFFFFFFFu));
+                if (p < s.P) rc[h] = a.rec[(size_t)gtap * a.ppad + p];
+                const uint32_t yx = __float_as_uint(rc[h].w);
+                fl[h] = 0u;
+                q00[h] = 0;
+                if (p < s.P && yx != 0xFFFFFFFFu) {
+                    const int y0 = (int)(yx >> 16) - 1, x0 = (int)(yx & 0xFFFFu) - 1;
+                    fl[h] = (inside(s, y0, x0) ? 1u : 0u) | (inside(s, y0, x0 + 1) ? 2u : 0u) |
+                            (inside(s, y0 + 1, x0) ? 4u : 0u) | (inside(s, y0 + 1, x0 + 1) ? 8u : 0u);
+                    q00[h] = ((long long)(p / plane) * s.H + y0) * s.W + x0;
+                }
+                sc[h] = a.gx ? (a.ovf ? fl[h] & a.ovf[(size_t)gtap * a.ppad + min(p, a.ppad - 1)] : fl[h]) : 0u;
+            }
+            // neighbour n of pixel h: element offset (q00 + (n & 1) + (n >> 1) W) * Cin + this lane's channels
+            const long long xoff = (long long)g * s.Cg + c0 + 16 * j;
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(ptx::smem_u32(&acc_full[abuf]), aphase, s_abort, a.status,
+                                                        WAIT_LIMIT))) {
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after();
+            const uint32_t tacc = tmem_base + (uint32_t)(abuf * NT) + ((uint32_t)rbase << 16);
+            float S[2][4];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) S[h][0] = S[h][1] = S[h][2] = S[h][3] = 0.f;
+            for (int blk = 0; blk < nb64; ++blk) {
+                uint32_t G[32];
+                tmem_ld_16x256b_x8(tacc + (uint32_t)(blk * 64), G);
+                uint32_t v[2][4][8];
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int n = 0; n < 4; ++n) {
+                        const bf16* src = a.x + (q00[h] + (n & 1) + (n >> 1) * s.W) * cin + xoff + blk * 64;
+#ifdef DCN_CHECKED
+                        const bool rd = ((fl[h] >> n) & 1u) && ptx::in_range(src, 32, a.x, xbytes, a.status);
+#else
+                        const bool rd = (fl[h] >> n) & 1u;
+#endif
+                        ptx::ldg_v8(v[h][n], rd ? reinterpret_cast<const uint8_t*>(src) : zb);
+                    }
+                ptx::tmem_wait_ld(G);
+                if (blk == nb64 - 1) {
+                    // the accumulator is read: hand it to the MMAs of unit + 2
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&acc_empty[abuf]));
+                }
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int n = 0; n < 4; ++n)
+#pragma unroll
+                        for (int m = 0; m < 8; ++m) {
+                            S[h][n] = fmaf(__uint_as_float(G[4 * m + 2 * h]), bf_lo(v[h][n][m]), S[h][n]);
+                            S[h][n] = fmaf(__uint_as_float(G[4 * m + 2 * h + 1]), bf_hi(v[h][n][m]), S[h][n]);
+                        }
+                if (sc[0] | sc[1]) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const float ly = rc[h].x, lx = rc[h].y, mk = rc[h].z;
+#pragma unroll
+                        for (int n = 0; n < 4; ++n) {
+                            if (!((sc[h] >> n) & 1u)) continue;
+                            const float wy = (n >> 1) ? ly : 1.f - ly, wx = (n & 1) ? lx : 1.f - lx;
+                            const float wnn = wy * wx * mk;
+                            float* dst = a.gx + (q00[h] + (n & 1) + (n >> 1) * s.W) * cin + xoff + blk * 64;
+#ifdef DCN_CHECKED
+                            if (!ptx::in_range(dst, 64, a.gx, gxbytes, a.status)) continue;
+#endif
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                ptx::red_add_v4(dst + 4 * i, __uint_as_float(G[8 * i + 2 * h]) * wnn,
+                                                __uint_as_float(G[8 * i + 2 * h + 1]) * wnn,
+                                                __uint_as_float(G[8 * i + 4 + 2 * h]) * wnn,
+                                                __uint_as_float(G[8 * i + 5 + 2 * h]) * wnn);
+                        }
+                    }
+                }
+            }
+            // S_n over the unit's channels: sum the four lanes of each pixel
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int n = 0; n < 4; ++n) {
+                    S[h][n] += __shfl_xor_sync(0xffffffffu, S[h][n], 1);
+                    S[h][n] += __shfl_xor_sync(0xffffffffu, S[h][n], 2);
+                }
+            if (j == 0) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int p = pp[h];
+                    if (p >= s.P) continue;
+                    const float ly = rc[h].x, lx = rc[h].y, mk = rc[h].z;
+                    const float d_y = mk * ((1.f - lx) * (S[h][2] - S[h][0]) + lx * (S[h][3] - S[h][1]));
+                    const float d_x = mk * ((1.f - ly) * (S[h][1] - S[h][0]) + ly * (S[h][3] - S[h][2]));
+                    const float d_m = (1.f - ly) * ((1.f - lx) * S[h][0] + lx * S[h][1]) +
+                                      ly * ((1.f - lx) * S[h][2] + lx * S[h][3]);
+                    const int bb = p / plane, pix = p - bb * plane;
+                    const size_t ob = ((size_t)bb * 2 * s.G * s.K2 + (size_t)g * 2 * s.K2 + 2 * tap) * plane + pix;
+                    const size_t om = ((size_t)bb * s.G * s.K2 + (size_t)g * s.K2 + tap) * plane + pix;
+                    if (a.nblk == 1) {  // this unit holds all of the group's channels: plain stores
+                        if (a.goff) {
+                            a.goff[ob] = d_y;
+                            a.goff[ob + plane] = d_x;
+                        }
+                        if (a.gmask) a.gmask[om] = d_m;
+                    } else {
+                        if (a.goff) {
+                            atomicAdd(a.goff + ob, d_y);
+                            atomicAdd(a.goff + ob + plane, d_x);
+                        }
+                        if (a.gmask) atomicAdd(a.gmask + om, d_m);
+                    }
+                }
+            }
+        }
     } else {
         // ------------------------------------------------------ epilogue --
         // Thread = pixel row when reading TMEM; the 32x32 block of G is then
@@ -360,6 +548,9 @@ __global__ void __launch_bounds__(256) dcn_records_f32_kernel(Shape s, const bf1
 }
 
 // w [Cout, KC] -> wt [KC, Cout] (bf16), 32x32 tiles through shared memory.
+// PERM: row k of wt goes to row (k & ~63) | inv_perm64(k & 63) (KC and the
+// channel count a multiple of 64), the order the per-pixel epilogue reads.
+template <bool PERM>
 __global__ void __launch_bounds__(256) dcn_transpose_kernel(const bf16* __restrict__ w, bf16* __restrict__ wt,
                                                             int Cout, int KC) {
     __shared__ bf16 t[32][33];
@@ -371,19 +562,22 @@ __global__ void __launch_bounds__(256) dcn_transpose_kernel(const bf16* __restri
     __syncthreads();
     for (int i = threadIdx.y; i < 32; i += 8) {
         const int k = k0 + i, o = o0 + threadIdx.x;
-        if (o < Cout && k < KC) wt[(size_t)k * Cout + o] = t[threadIdx.x][i];
+        const int kd = PERM ? ((k & ~63) | inv_perm64(k & 63)) : k;
+        if (o < Cout && k < KC) wt[(size_t)kd * Cout + o] = t[threadIdx.x][i];
     }
 }
 
 struct BdPlan {
     bool ok;
+    int epi;  // 1: the per-pixel epilogue (channels per group a multiple of 64), else 0
     int nblk, units_per_tile, m_tiles, ppad, ctas, stages, kchunks;
     long long total_units;
     uint32_t smem_bytes;
     size_t rec_bytes, wt_off, ws_bytes;
 };
 
-BdPlan make_bd_plan(const Shape& s, int sms) {
+// x32: x is 32-byte aligned (the per-pixel epilogue loads 32-byte slices)
+BdPlan make_bd_plan(const Shape& s, int sms, bool x32 = true) {
     BdPlan pl{};
     if (s.Cin % 8 || s.Cg % 8 || s.Cout % 8 || s.H >= 65535 || s.W >= 65535) return pl;
     pl.nblk = (s.Cg + NT - 1) / NT;
@@ -393,10 +587,11 @@ BdPlan make_bd_plan(const Shape& s, int sms) {
     pl.kchunks = (s.Cout + BK - 1) / BK;
     pl.total_units = (long long)pl.m_tiles * pl.units_per_tile;
     pl.ctas = (int)std::min<long long>(sms, pl.total_units);
+    pl.epi = (x32 && s.Cg % 64 == 0 && s.Cin % 64 == 0) ? 1 : 0;
     const uint32_t budget = 227 * 1024;
-    const uint32_t tbytes = EPI_WARPS * 32 * TPITCH * 4;  // epilogue transpose buffers
+    const uint32_t tbytes = pl.epi ? 0u : (uint32_t)(EPI_WARPS * 32 * TPITCH * 4);  // epilogue transpose buffers
     int st = (int)((budget - 2048 - 1024 - tbytes) / (A_BYTES + B_BYTES));
-    pl.stages = std::min(st, 3);
+    pl.stages = std::min(st, pl.epi ? MAX_STAGES : 3);
     pl.smem_bytes = pl.stages * (A_BYTES + B_BYTES) + 1024 + tbytes + 1024;
     pl.rec_bytes = (size_t)s.G * s.K2 * pl.ppad * sizeof(float4);
     pl.wt_off = (pl.rec_bytes + 255) & ~(size_t)255;
@@ -442,7 +637,7 @@ size_t bwd_data_tc_workspace(const Shape& s) {
 cudaError_t bwd_data_tc(const Shape& s, const void* x, const void* off, const void* mask, const void* w,
                         const void* gy, float* gx, float* goff, float* gmask, void* ws, size_t ws_bytes,
                         unsigned* status, cudaStream_t st, int* launches) {
-    BdPlan pl = make_bd_plan(s, num_sms());
+    BdPlan pl = make_bd_plan(s, num_sms(), (reinterpret_cast<uintptr_t>(x) & 31) == 0);
     if (!pl.ok || !ws || ws_bytes < pl.ws_bytes) return cudaErrorInvalidValue;
     float4* rec = reinterpret_cast<float4*>(ws);
     bf16* wt = reinterpret_cast<bf16*>(static_cast<uint8_t*>(ws) + pl.wt_off);
@@ -450,12 +645,14 @@ cudaError_t bwd_data_tc(const Shape& s, const void* x, const void* off, const vo
     if (!encode_kmajor(&map_dy, gy, (uint64_t)s.Cout, (uint64_t)s.P, BM) ||
         !encode_kmajor(&map_wt, wt, (uint64_t)s.Cout, (uint64_t)s.KC, NT))
         return cudaErrorInvalidValue;
-    static DeviceFlags attr_set;
-    cudaError_t e = max_dynamic_smem_once((const void*)dcn_bwd_data_tc_kernel, 227 * 1024, attr_set);
+    auto kernel = pl.epi ? dcn_bwd_data_tc_kernel<1> : dcn_bwd_data_tc_kernel<0>;
+    static DeviceFlags attr_set[2];
+    cudaError_t e = max_dynamic_smem_once((const void*)kernel, 227 * 1024, attr_set[pl.epi]);
     if (e != cudaSuccess) return e;
     int n = 0;
     dim3 tg((s.KC + 31) / 32, (s.Cout + 31) / 32);
-    dcn_transpose_kernel<<<tg, dim3(32, 8), 0, st>>>((const bf16*)w, wt, s.Cout, s.KC);
+    if (pl.epi) dcn_transpose_kernel<true><<<tg, dim3(32, 8), 0, st>>>((const bf16*)w, wt, s.Cout, s.KC);
+    else dcn_transpose_kernel<false><<<tg, dim3(32, 8), 0, st>>>((const bf16*)w, wt, s.Cout, s.KC);
     ++n;
     dim3 rg((pl.ppad + 255) / 256, s.G * s.K2);
     dcn_records_f32_kernel<<<rg, 256, 0, st>>>(s, (const bf16*)off, (const bf16*)mask, rec, pl.ppad);
@@ -465,18 +662,20 @@ cudaError_t bwd_data_tc(const Shape& s, const void* x, const void* off, const vo
         if ((e = cudaMemsetAsync(gx, 0, sizeof(float) * (size_t)s.B * s.H * s.W * s.Cin, st)) != cudaSuccess) return e;
         ++n;
     }
-    if (goff) {
+    // the per-pixel epilogue stores grad_offset / grad_mask outright when one unit holds a group's channels
+    const bool zero_om = !(pl.epi && pl.nblk == 1);
+    if (goff && zero_om) {
         if ((e = cudaMemsetAsync(goff, 0, sizeof(float) * (size_t)s.P * 2 * s.G * s.K2, st)) != cudaSuccess) return e;
         ++n;
     }
-    if (gmask) {
+    if (gmask && zero_om) {
         if ((e = cudaMemsetAsync(gmask, 0, sizeof(float) * (size_t)s.P * s.G * s.K2, st)) != cudaSuccess) return e;
         ++n;
     }
     // grad_x through the shared-memory window kernel where it applies (and
     // DCN_BWD_GX_WINDOW is on); this file's kernel then computes only
     // grad_offset and grad_mask
-    if (DCN_BWD_GX_WINDOW && gx && bwd_gx_supported(s)) {
+    if (!pl.epi && DCN_BWD_GX_WINDOW && gx && bwd_gx_supported(s)) {
         e = bwd_gx_tc(s, gy, wt, rec, pl.ppad, gx, status, st, &n);
         if (e != cudaSuccess) return e;
         gx = nullptr;
@@ -492,6 +691,7 @@ cudaError_t bwd_data_tc(const Shape& s, const void* x, const void* off, const vo
     a.gx = gx;
     a.goff = goff;
     a.gmask = gmask;
+    a.ovf = nullptr;
     a.status = status;
     a.nblk = pl.nblk;
     a.units_per_tile = pl.units_per_tile;
@@ -501,7 +701,7 @@ cudaError_t bwd_data_tc(const Shape& s, const void* x, const void* off, const vo
     a.stages = pl.stages;
     a.kchunks = pl.kchunks;
     a.total_units = pl.total_units;
-    dcn_bwd_data_tc_kernel<<<pl.ctas, NUM_THREADS, pl.smem_bytes, st>>>(map_dy, map_wt, a);
+    kernel<<<pl.ctas, NUM_THREADS, pl.smem_bytes, st>>>(map_dy, map_wt, a);
     ++n;
     if (launches) *launches += n;
     return cudaGetLastError();
