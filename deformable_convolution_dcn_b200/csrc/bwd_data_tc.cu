@@ -55,6 +55,9 @@ constexpr int TPITCH = 36;                  // floats per row of an epilogue war
 #ifndef DCN_BWD_GX_WINDOW
 #define DCN_BWD_GX_WINDOW 0
 #endif
+#ifndef DCN_BD_EPI1_STAGES
+#define DCN_BD_EPI1_STAGES 2
+#endif
 
 struct BdArgs {
     Shape s;
@@ -574,6 +577,8 @@ struct BdPlan {
     long long total_units;
     uint32_t smem_bytes;
     size_t rec_bytes, wt_off, ws_bytes;
+    bool gxt;               // grad_x through the transposed gather-GEMM (per-pixel epilogue layers)
+    size_t ovf_off, gxt_off;
 };
 
 // x32: x is 32-byte aligned (the per-pixel epilogue loads 32-byte slices)
@@ -591,11 +596,20 @@ BdPlan make_bd_plan(const Shape& s, int sms, bool x32 = true) {
     const uint32_t budget = 227 * 1024;
     const uint32_t tbytes = pl.epi ? 0u : (uint32_t)(EPI_WARPS * 32 * TPITCH * 4);  // epilogue transpose buffers
     int st = (int)((budget - 2048 - 1024 - tbytes) / (A_BYTES + B_BYTES));
-    pl.stages = std::min(st, pl.epi ? MAX_STAGES : 3);
+    // the per-pixel epilogue's neighbour loads want L1 more than the MMAs want stages
+    pl.stages = std::min(st, pl.epi ? DCN_BD_EPI1_STAGES : 3);
     pl.smem_bytes = pl.stages * (A_BYTES + B_BYTES) + 1024 + tbytes + 1024;
     pl.rec_bytes = (size_t)s.G * s.K2 * pl.ppad * sizeof(float4);
     pl.wt_off = (pl.rec_bytes + 255) & ~(size_t)255;
     pl.ws_bytes = pl.wt_off + (size_t)s.KC * s.Cout * sizeof(bf16);
+    // grad_x without atomics where the transposed gather-GEMM takes the layer
+    pl.gxt = pl.epi && gxt_supported(s);
+    pl.ovf_off = pl.gxt_off = 0;
+    if (pl.gxt) {
+        pl.ovf_off = (pl.ws_bytes + 255) & ~(size_t)255;
+        pl.gxt_off = (pl.ovf_off + (size_t)s.G * s.K2 * pl.ppad + 255) & ~(size_t)255;
+        pl.ws_bytes = pl.gxt_off + gxt_workspace(s);
+    }
     pl.ok = (long long)s.B * s.H * s.W * s.Cin < (1LL << 31);
     return pl;
 }
@@ -647,7 +661,11 @@ cudaError_t bwd_data_tc(const Shape& s, const void* x, const void* off, const vo
         return cudaErrorInvalidValue;
     auto kernel = pl.epi ? dcn_bwd_data_tc_kernel<1> : dcn_bwd_data_tc_kernel<0>;
     static DeviceFlags attr_set[2];
+    static DeviceCarveout carve[2];
     cudaError_t e = max_dynamic_smem_once((const void*)kernel, 227 * 1024, attr_set[pl.epi]);
+    if (e != cudaSuccess) return e;
+    // the rest of the SM's 256 KB is L1 for the neighbour loads
+    e = smem_carveout_for((const void*)kernel, pl.smem_bytes, carve[pl.epi]);
     if (e != cudaSuccess) return e;
     int n = 0;
     dim3 tg((s.KC + 31) / 32, (s.Cout + 31) / 32);
@@ -658,7 +676,16 @@ cudaError_t bwd_data_tc(const Shape& s, const void* x, const void* off, const vo
     dcn_records_f32_kernel<<<rg, 256, 0, st>>>(s, (const bf16*)off, (const bf16*)mask, rec, pl.ppad);
     ++n;
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if (gx) {
+    // grad_x: the transposed gather-GEMM writes it (all but the flagged corners, which this
+    // file's kernel then adds with atomics); otherwise zeroed here and scattered in full
+    const uint8_t* ovf = nullptr;
+    if (gx && pl.gxt) {
+        uint8_t* ovf_w = static_cast<uint8_t*>(ws) + pl.ovf_off;
+        e = gxt(s, off, mask, w, gy, gx, ovf_w, pl.ppad, static_cast<uint8_t*>(ws) + pl.gxt_off,
+                ws_bytes - pl.gxt_off, status, st, &n);
+        if (e != cudaSuccess) return e;
+        ovf = ovf_w;
+    } else if (gx) {
         if ((e = cudaMemsetAsync(gx, 0, sizeof(float) * (size_t)s.B * s.H * s.W * s.Cin, st)) != cudaSuccess) return e;
         ++n;
     }
@@ -691,7 +718,7 @@ cudaError_t bwd_data_tc(const Shape& s, const void* x, const void* off, const vo
     a.gx = gx;
     a.goff = goff;
     a.gmask = gmask;
-    a.ovf = nullptr;
+    a.ovf = ovf;
     a.status = status;
     a.nblk = pl.nblk;
     a.units_per_tile = pl.units_per_tile;

@@ -16,6 +16,7 @@
 
 #include <algorithm>
 #include <mutex>
+#include <type_traits>
 
 #include "kernels.h"
 #include "tc_ptx.cuh"
@@ -253,6 +254,22 @@ __device__ __forceinline__ void store_row32(bf16* yrow, int cc, int ncols, uint3
     }
 }
 
+// As above for a float32 output row (no rounding): y[row, cc .. cc + 31] = r + bias.
+__device__ __forceinline__ void store_row32(float* yrow, int cc, int ncols, uint32_t (&r)[32], const float* sb) {
+    float v[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]) + (sb ? sb[cc + e] : 0.f);
+    if (cc + 32 <= ncols) {
+        float4* dst = reinterpret_cast<float4*>(yrow + cc);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+            if (cc + e < ncols) yrow[cc + e] = v[e];
+    }
+}
+
 // Walks this warp's 32 TMEM lanes over columns [0, ncols) in blocks of 32,
 // calling f(r, cc) on each block; PIPE: while the next block's load is in
 // flight (twice the registers). ncols is warp-uniform (the loads are
@@ -297,13 +314,14 @@ __device__ __forceinline__ void tmem_rows(uint32_t taddr, int ncols, F&& f) {
 // 128-byte row segments, eight lanes per row; otherwise each lane stores its row.
 // own_in_part: this CTA's own contribution is read back from part(cta) as
 // well (its accumulator has already been released).
-template <typename P>
+template <typename P, typename OutT>
 __device__ __forceinline__ void combine_rows(uint32_t taddr, int ncols, int c_lo, int c_hi, int cta, bool in_smem,
-                                             P&& part, const float* sb, uint32_t ybuf, bf16* ycol0, int pr,
+                                             P&& part, const float* sb, uint32_t ybuf, OutT* ycol0, int pr,
                                              int ldy, int cc_begin = 0, int cc_end = 1 << 30,
                                              bool own_in_part = false) {
     const int lane = threadIdx.x & 31;
-    const bool coalesce = ybuf != 0 && (ncols & 63) == 0;  // cc_begin must then be a multiple of 64
+    // staged, coalesced stores for bf16 outputs (cc_begin must then be a multiple of 64)
+    const bool coalesce = std::is_same<OutT, bf16>::value && ybuf != 0 && (ncols & 63) == 0;
     for (int cc = cc_begin; cc < min(ncols, cc_end); cc += 32) {
         uint32_t acc[32];
 #pragma unroll
@@ -329,36 +347,38 @@ __device__ __forceinline__ void combine_rows(uint32_t taddr, int ncols, int c_lo
             if (pr >= 0) store_row32(ycol0 + (size_t)pr * ldy, cc, ncols, acc, sb);
             continue;
         }
-        if (sb) {
+        if constexpr (std::is_same<OutT, bf16>::value) {
+            if (sb) {
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const float4 b = *reinterpret_cast<const float4*>(sb + cc + 4 * q);
-                acc[4 * q] = __float_as_uint(__uint_as_float(acc[4 * q]) + b.x);
-                acc[4 * q + 1] = __float_as_uint(__uint_as_float(acc[4 * q + 1]) + b.y);
-                acc[4 * q + 2] = __float_as_uint(__uint_as_float(acc[4 * q + 2]) + b.z);
-                acc[4 * q + 3] = __float_as_uint(__uint_as_float(acc[4 * q + 3]) + b.w);
+                for (int q = 0; q < 8; ++q) {
+                    const float4 b = *reinterpret_cast<const float4*>(sb + cc + 4 * q);
+                    acc[4 * q] = __float_as_uint(__uint_as_float(acc[4 * q]) + b.x);
+                    acc[4 * q + 1] = __float_as_uint(__uint_as_float(acc[4 * q + 1]) + b.y);
+                    acc[4 * q + 2] = __float_as_uint(__uint_as_float(acc[4 * q + 2]) + b.z);
+                    acc[4 * q + 3] = __float_as_uint(__uint_as_float(acc[4 * q + 3]) + b.w);
+                }
             }
-        }
-        const int h = (cc >> 5) & 1;  // which half of the 64-column group
+            const int h = (cc >> 5) & 1;  // which half of the 64-column group
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const uint32_t* w = acc + 8 * j;
-            ptx::sts_v4(ybuf + lane * 128 + (((4 * h + j) ^ (lane & 7)) << 4),
-                        make_uint4(pack_bf16(__uint_as_float(w[0]), __uint_as_float(w[1])),
-                                   pack_bf16(__uint_as_float(w[2]), __uint_as_float(w[3])),
-                                   pack_bf16(__uint_as_float(w[4]), __uint_as_float(w[5])),
-                                   pack_bf16(__uint_as_float(w[6]), __uint_as_float(w[7]))));
-        }
-        if (h == 1) {
-            __syncwarp();
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int rr = 4 * i + (lane >> 3), ch = lane & 7;
-                const uint4 v = ptx::lds_v4(ybuf + rr * 128 + ((ch ^ (rr & 7)) << 4));
-                const int prr = __shfl_sync(0xffffffffu, pr, rr);
-                if (prr >= 0) *reinterpret_cast<uint4*>(ycol0 + (size_t)prr * ldy + (cc - 32) + ch * 8) = v;
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t* w = acc + 8 * j;
+                ptx::sts_v4(ybuf + lane * 128 + (((4 * h + j) ^ (lane & 7)) << 4),
+                            make_uint4(pack_bf16(__uint_as_float(w[0]), __uint_as_float(w[1])),
+                                       pack_bf16(__uint_as_float(w[2]), __uint_as_float(w[3])),
+                                       pack_bf16(__uint_as_float(w[4]), __uint_as_float(w[5])),
+                                       pack_bf16(__uint_as_float(w[6]), __uint_as_float(w[7]))));
             }
-            __syncwarp();
+            if (h == 1) {
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int rr = 4 * i + (lane >> 3), ch = lane & 7;
+                    const uint4 v = ptx::lds_v4(ybuf + rr * 128 + ((ch ^ (rr & 7)) << 4));
+                    const int prr = __shfl_sync(0xffffffffu, pr, rr);
+                    if (prr >= 0) *reinterpret_cast<uint4*>(ycol0 + (size_t)prr * ldy + (cc - 32) + ch * 8) = v;
+                }
+                __syncwarp();
+            }
         }
     }
 }

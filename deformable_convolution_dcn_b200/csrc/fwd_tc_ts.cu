@@ -78,9 +78,24 @@ constexpr int ALL_TAPS = 25;
 constexpr int MAX_TAPS_TS = 49;
 constexpr int TAP_TABLE = 64;  // entries of the shared-memory tap table
 
+// Gather record of the transposed pass (MODE 1, the grad_x contraction): up
+// to LIST_E (dY row, weight) entries of one (input pixel, tap); entry e is
+// read when bit e of vmask is set. The weights pair up as in TapRec, so the
+// same packed blend sums them.
+constexpr int LIST_E = 4;
+struct __align__(16) ListRec {
+    int p[LIST_E];  // dY rows: output pixels (b*Ho + ho)*Wo + wo whose sample reaches this pixel
+    uint32_t w10;   // lo: entry 0's weight m * (corner weight), hi: entry 1's (bf16)
+    uint32_t w32;   // lo: entry 2's, hi: entry 3's
+    uint32_t vmask;
+    uint32_t pad;
+};
+
 struct TsArgs {
     FwdArgs f;
-    const TapRec* recs;   // [m tiles][G][K*K][BM] sampling records (workspace), tap-major
+    const uint8_t* recs;  // [m tiles][G][K*K][BM] records (workspace), tap-major: TapRec (MODE 0), ListRec (MODE 1)
+    float* yf;            // MODE 1: float32 output, row pitch ldy, first column col0
+    int ldy, col0;
     int ep_len, ep_taps;  // chunks per records epoch, taps held per record buffer
     int b_stages;
     uint32_t idle_bytes;  // shared memory free after the last MMA (the weight ring)
@@ -133,12 +148,27 @@ __global__ void __launch_bounds__(256) dcn_fwd_prepass_kernel(const bf16* __rest
     *reinterpret_cast<uint4*>(wp + ((size_t)o * U + u) * BK + 8 * k8) = make_uint4(v[0].x, v[0].y, v[1].x, v[1].y);
 }
 
+// Output column n0 of the tile's first row pointer, and the row pitch.
+template <int MODE>
+__device__ __forceinline__ auto out_col(const TsArgs& ta, int n0) {
+    if constexpr (MODE == 0) return ta.f.y + n0;
+    else return ta.yf + ta.col0 + n0;
+}
+template <int MODE>
+__device__ __forceinline__ int out_ld(const TsArgs& ta) {
+    return MODE == 0 ? ta.f.s.Cout : ta.ldy;
+}
+
 // --------------------------------------------------------------- kernel --
 // WIDE: x is 32-byte aligned and Cin, Cg are multiples of 16, so a lane's
 // 16-channel slice is one 32-byte load.
-template <bool WIDE>
+// MODE 0: the forward (Y = Col * W'^T, bf16 y + bias; bilinear TapRec records).
+// MODE 1: the transposed pass of the backward (rows = input pixels, the
+// gathered tensor is grad_y and the records are ListRec lists; float32 out).
+template <bool WIDE, int MODE>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     dcn_fwd_ts_kernel(const __grid_constant__ CUtensorMap tmap_w, const TsArgs ta) {
+    constexpr uint32_t REC_BYTES = MODE == 0 ? (uint32_t)sizeof(TapRec) : (uint32_t)sizeof(ListRec);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -146,7 +176,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const Shape& s = a.s;
 
     uint8_t* sB = smem;  // weight ring: b_stages x [N x 128 B], 128-byte swizzle
-    TapRec* s_rec = reinterpret_cast<TapRec*>(smem + a.info_off);  // two buffers of BM * K2 records
+    uint8_t* s_rec = smem + a.info_off;  // two buffers of BM * ep_taps records
     int2* s_tap = reinterpret_cast<int2*>(smem + a.row_off);        // per tap: (i*dil, j*dil)
     long long* s_starts = reinterpret_cast<long long*>(s_tap + TAP_TABLE);  // [ctas + 1] first unit of each CTA
     float* s_bias = reinterpret_cast<float*>(s_starts + MAX_CTAS + 2);  // [2][512] bias of a tile's columns
@@ -251,12 +281,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint32_t cmask = cg < s.Cg ? 0xFu : 0u;
             const bool hi_ok = cg + 8 < s.Cg;  // upper 8 channels present (narrow loads only)
             const uint8_t* xc = reinterpret_cast<const uint8_t*>(a.x + ich.g * s.Cg + cg);
-            const uint4 rc = ptx::lds_v4(irecs + (uint32_t)(((ich.tap - irb) * BM + row) * (int)sizeof(TapRec)));
-            w[0] = rc.x;  // TapRec::w01_00
-            w[1] = rc.y;  // TapRec::w11_10
-            const uint32_t vm = rc.w & cmask;  // TapRec::vmask
-            const uint8_t* p = xc + (long long)(int)rc.z * cin2;  // TapRec::base
-            const uint8_t* pc[4] = {p, p + cin2, p + rp2, p + rp2 + cin2};
+            const uint32_t ra = irecs + (uint32_t)((ich.tap - irb) * BM + row) * REC_BYTES;
+            const uint8_t* pc[4];
+            uint32_t vm;
+            if constexpr (MODE == 0) {
+                const uint4 rc = ptx::lds_v4(ra);
+                w[0] = rc.x;  // TapRec::w01_00
+                w[1] = rc.y;  // TapRec::w11_10
+                vm = rc.w & cmask;  // TapRec::vmask
+                const uint8_t* p = xc + (long long)(int)rc.z * cin2;  // TapRec::base
+                pc[0] = p;
+                pc[1] = p + cin2;
+                pc[2] = p + rp2;
+                pc[3] = p + rp2 + cin2;
+            } else {
+                const uint4 pe = ptx::lds_v4(ra);       // ListRec::p
+                const uint4 rw = ptx::lds_v4(ra + 16);  // ListRec::w10, w32, vmask
+                w[0] = rw.x;
+                w[1] = rw.y;
+                vm = rw.z & cmask;
+                pc[0] = xc + (long long)(int)pe.x * cin2;
+                pc[1] = xc + (long long)(int)pe.y * cin2;
+                pc[2] = xc + (long long)(int)pe.z * cin2;
+                pc[3] = xc + (long long)(int)pe.w * cin2;
+            }
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
 #ifdef DCN_CHECKED
@@ -299,7 +347,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 if (!__all_sync(0xffffffffu, ptx::mbar_wait(ptx::smem_u32(&rec_full[b]), par, s_abort, a.status,
                                                             WAIT_LIMIT)))
                     return false;
-                irecs = ptx::smem_u32(s_rec + b * BM * ta.ep_taps);
+                irecs = ptx::smem_u32(s_rec + (size_t)b * BM * ta.ep_taps * REC_BYTES);
             }
             return true;
         };
@@ -402,7 +450,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         if (staged)
                             return reinterpret_cast<const float*>(smem + (size_t)(c - c_lo - (c > cta)) * tile_bytes) + row * 4;
                         return partial_base(a, s_starts, c, tu0, row);
-                    }, sb, ybuf, a.y + n0, p, s.Cout, pr2 * 64, pr2 * 64 + 64);
+                    }, sb, ybuf, out_col<MODE>(ta, n0), p, out_ld<MODE>(ta), pr2 * 64, pr2 * 64 + 64);
             }
         }
     } else if (warp == TMA_WARP) {
@@ -521,11 +569,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         ok = false;
                     } else {
                         ptx::fence_proxy_async_smem();  // the producers' reads before the copy's writes
-                        const uint32_t bytes = (uint32_t)(BM * ta.ep_taps * sizeof(TapRec));
+                        const uint32_t bytes = (uint32_t)BM * ta.ep_taps * REC_BYTES;
                         const uint32_t fb = ptx::smem_u32(&rec_full[b]);
                         ptx::mbar_arrive_expect_tx(fb, bytes);
-                        ptx::bulk_load(ptx::smem_u32(s_rec + b * BM * ta.ep_taps),
-                                       ta.recs + (((size_t)(rs.t / a.n_tiles) * s.G + rg) * s.K2 + rt) * BM, bytes, fb);
+                        ptx::bulk_load(ptx::smem_u32(s_rec + (size_t)b * BM * ta.ep_taps * REC_BYTES),
+                                       ta.recs + (((size_t)(rs.t / a.n_tiles) * s.G + rg) * s.K2 + rt) * BM * REC_BYTES,
+                                       bytes, fb);
                     }
                 }
                 if (warp == 0) ok = __shfl_sync(0xffffffffu, ok, 0);  // warp 0 stays convergent
@@ -575,7 +624,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const float* sb = a.bias ? sbias : nullptr;
             const int p = strip_to_raster(mt * BM + row, a);
             const uint32_t taddr = tmem_base + (uint32_t)(abuf * a.acc_cols) + ((uint32_t)(quarter * 32) << 16);
-            bf16* ycol0 = a.y + n0;
+            auto* ycol0 = out_col<MODE>(ta, n0);
+            const int ldy = out_ld<MODE>(ta);
             if (s_last[seg & 1]) {
                 const uint32_t tile_bytes = (uint32_t)BM * a.bn_total * 4;
                 const bool staged = !full && last_proc && (uint32_t)(c_hi - c_lo) * tile_bytes <= ta.idle_bytes;
@@ -615,10 +665,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 };
                 if (help) {
                     for (int pr2 = 0; pr2 * 64 < ncols; pr2 += 3)
-                        combine_rows(taddr, ncols, c_lo, c_hi, cta, staged, part, sb, ybuf, ycol0, p, s.Cout, pr2 * 64,
+                        combine_rows(taddr, ncols, c_lo, c_hi, cta, staged, part, sb, ybuf, ycol0, p, ldy, pr2 * 64,
                                      pr2 * 64 + 64);
                 } else {
-                    combine_rows(taddr, ncols, c_lo, c_hi, cta, staged, part, sb, ybuf, ycol0, p, s.Cout);
+                    combine_rows(taddr, ncols, c_lo, c_hi, cta, staged, part, sb, ybuf, ycol0, p, ldy);
                 }
                 ptx::tc_fence_before();
                 __syncwarp();
@@ -655,7 +705,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     __threadfence();
                     combine_rows(taddr, ncols, c_lo, c_hi, cta, false, [&](int c) -> const float* {
                         return partial_base(a, s_starts, c, tu0, row);
-                    }, sb, 0u, ycol0, p, s.Cout, 0, 1 << 30, true);
+                    }, sb, 0u, ycol0, p, ldy, 0, 1 << 30, true);
                     if (threadIdx.x == 0) a.counters[t] = 0;
                 }
             }
@@ -682,9 +732,12 @@ struct TsPlan {
     long long nrec;
 };
 
-TsPlan make_ts_plan(const Shape& s, int sms) {
+// mode 0: the forward; mode 1: the transposed pass (ListRec records, kept
+// outside this workspace).
+TsPlan make_ts_plan(const Shape& s, int sms, int mode = 0) {
     TsPlan pl{};
     pl.ok = false;
+    const uint32_t rec_bytes = mode ? (uint32_t)sizeof(ListRec) : (uint32_t)sizeof(TapRec);
     if (s.Cin % 8 || s.Cg % 8 || s.Cout % 8 || s.K2 > MAX_TAPS_TS || s.Cout > 256) return pl;
     pl.bn_total = (s.Cout + 31) / 32 * 32;
     pl.k = plan_stream_k(s, pl.bn_total, sms);
@@ -693,9 +746,11 @@ TsPlan make_ts_plan(const Shape& s, int sms) {
     pl.b_stage_bytes = (uint32_t)pl.bn_total * 128;
     pl.b_stages = std::min(DCN_FWD_TS_B_STAGES, MAX_B_STAGES);
     const uint32_t ring = (uint32_t)pl.b_stages * pl.b_stage_bytes;
-    pl.ep_taps = s.K2 <= ALL_TAPS ? s.K2 : s.K;
-    pl.ep_len = s.K2 <= ALL_TAPS ? pl.k.nq * s.K2 : s.K;
-    const uint32_t info_bytes = (uint32_t)(2 * BM * pl.ep_taps * sizeof(TapRec));
+    // all taps of a (tile, group) per record buffer when they fit in 36 KB, else one kernel row
+    const bool all_taps = s.K2 <= ALL_TAPS && 2u * BM * s.K2 * rec_bytes <= 36u * 1024u;
+    pl.ep_taps = all_taps ? s.K2 : s.K;
+    pl.ep_len = all_taps ? pl.k.nq * s.K2 : s.K;
+    const uint32_t info_bytes = 2u * BM * (uint32_t)pl.ep_taps * rec_bytes;
     pl.info_off = ring;
     pl.row_off = pl.info_off + info_bytes;
     pl.bar_off = pl.row_off + (uint32_t)(TAP_TABLE * sizeof(int2) + (MAX_CTAS + 2) * sizeof(long long) +
@@ -708,56 +763,182 @@ TsPlan make_ts_plan(const Shape& s, int sms) {
     pl.ws_wperm_off = (pl.ws_counters_off + (size_t)pl.k.tiles * sizeof(int) + 255) & ~(size_t)255;
     pl.ws_recs_off = (pl.ws_wperm_off + (size_t)s.Cout * pl.k.U * BK * 2 + 255) & ~(size_t)255;
     pl.nrec = (long long)pl.k.m_tiles * s.G * s.K2 * BM;
-    pl.ws_bytes = pl.ws_recs_off + (size_t)pl.nrec * sizeof(TapRec);
+    pl.ws_bytes = pl.ws_recs_off + (mode ? (size_t)0 : (size_t)pl.nrec * sizeof(TapRec));
     pl.ok = true;
     return pl;
 }
 
-}  // namespace
 
-bool fwd_ts_supported(const Shape& s) { return make_ts_plan(s, num_sms()).ok; }
+// ------------------------------------------------- transposed pass (grad_x) --
+// grad_x[q, g*Cg + c] = sum_tap sum_o H_g[q, tap, o] * w[o, tap, g*Cg + c], with
+// H_g[q, tap, :] = the sum over the samples (p, corner n) of group g and tap
+// whose bilinear neighbour n is input pixel q of m * (corner weight) * grad_y[p, :]
+// (the transpose of the forward's sampling: the gradient equations of the
+// "Deformable ConvNets" notes summed per input pixel instead of scattered).
+// It runs as the main kernel above in MODE 1 on a virtual layer whose output
+// pixels are the input pixels, whose gathered tensor is grad_y and whose
+// output channels are one group's input channels.
 
-size_t fwd_ts_workspace(const Shape& s) {
-    const TsPlan pl = make_ts_plan(s, num_sms());
-    return pl.ok ? pl.ws_bytes : 0;
+// Row of input pixel q in the strip order of the virtual layer (the inverse of
+// strip_to_raster for Ho = H, Wo = W).
+__device__ __forceinline__ int raster_to_strip(int q, int H, int W, int sw, int nf, int wl) {
+    const int plane = H * W;
+    const int b = q / plane, rem = q - b * plane;
+    const int y = rem / W, xx = rem - y * W;
+    const int strip = xx / sw;
+    if (strip < nf) return b * plane + strip * (H * sw) + y * sw + (xx - strip * sw);
+    return b * plane + nf * H * sw + y * wl + (xx - nf * sw);
 }
 
-cudaError_t fwd_ts(const Shape& s, const void* x, const void* off, const void* mask, const void* w, const void* bias,
-                   void* y, void* ws, size_t ws_bytes, unsigned* status, cudaStream_t st, int* launches) {
-    const TsPlan pl = make_ts_plan(s, num_sms());
-    if (!pl.ok || ws_bytes < pl.ws_bytes || !ws) return cudaErrorInvalidValue;
-    auto encode = get_encode();
-    if (!encode) return cudaErrorNotSupported;
-    uint8_t* wsb = static_cast<uint8_t*>(ws);
-    int* counters = reinterpret_cast<int*>(wsb + pl.ws_counters_off);
-    bf16* wperm = reinterpret_cast<bf16*>(wsb + pl.ws_wperm_off);
-    CUtensorMap map;
-    cuuint64_t dims[2] = {(cuuint64_t)pl.k.U * BK, (cuuint64_t)s.Cout};
-    cuuint64_t strides[1] = {(cuuint64_t)pl.k.U * BK * 2};
-    cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)pl.bn_total};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, wperm, dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    const bool wide = s.Cin % 16 == 0 && s.Cg % 16 == 0 && (reinterpret_cast<uintptr_t>(x) & 31) == 0;
-    auto kernel = wide ? dcn_fwd_ts_kernel<true> : dcn_fwd_ts_kernel<false>;
-    static DeviceFlags attr_set[2];
-    static DeviceCarveout carve[2];
-    cudaError_t e = max_dynamic_smem_once((const void*)kernel, 227 * 1024, attr_set[wide]);
-    if (e != cudaSuccess) return e;
-    // the gather hits in L1: give it everything the kernel's shared memory does not need
-    e = smem_carveout_for((const void*)kernel, pl.smem_bytes, carve[wide]);
-    if (e != cudaSuccess) return e;
-    TsArgs ta;
+// One thread per (output pixel p, group-tap gt, corner n): the corner is
+// inserted into its input pixel's list, which keeps the LIST_E
+// smallest keys (p << 32 | n << 16 | bf16 weight) in ascending order: a key
+// goes down the slots with atomicMin, carrying on with whichever of it and
+// the slot's old key is larger, until it fills an empty slot (all bits set
+// on entry) or falls off the end. The lists and the set of corners that fall
+// off (flagged in ovf[gt * ovf_pitch + p'], bit n', zero on entry) therefore
+// do not depend on the order of the insertions. Corners outside the map or of
+// zero (bf16) weight add nothing and are skipped.
+constexpr unsigned long long EMPTY_KEY = ~0ull;
+__global__ void __launch_bounds__(256) dcn_gxt_fill_kernel(const Shape s, const bf16* __restrict__ off,
+                                                           const bf16* __restrict__ mask, ListRec* __restrict__ lrecs,
+                                                           uint8_t* __restrict__ ovf, int ovf_pitch, int mtiles_v,
+                                                           int sw, int nf, int wl) {
+    const int p = blockIdx.x * blockDim.x + threadIdx.x;
+    const int gt = blockIdx.y >> 2, n = blockIdx.y & 3;
+    if (p >= s.P) return;
+    const int g = gt / s.K2, tap = gt - g * s.K2;
+    const int plane = s.Ho * s.Wo;
+    const int b = p / plane, pix = p - b * plane;
+    const int ho = pix / s.Wo, wo = pix - ho * s.Wo;
+    const int i = tap / s.K, j = tap - i * s.K;
+    const bf16* offp = off + ((size_t)b * 2 * s.G * s.K2 + (size_t)g * 2 * s.K2 + 2 * tap) * plane + pix;
+    const float dy = __bfloat162float(offp[0]), dx = __bfloat162float(offp[plane]);
+    const float mk = mask ? __bfloat162float(mask[((size_t)b * s.G * s.K2 + (size_t)g * s.K2 + tap) * plane + pix])
+                          : 1.f;
+    int y0, x0;
+    float ly, lx;
+    split_coord(ho * s.stride - s.pad + i * s.dil, dy, y0, ly);
+    split_coord(wo * s.stride - s.pad + j * s.dil, dx, x0, lx);
+    {
+        const int yy = y0 + (n >> 1), xx = x0 + (n & 1);
+        if (!inside(s, yy, xx)) return;
+        const float wf = ((n >> 1) ? ly : 1.f - ly) * ((n & 1) ? lx : 1.f - lx) * mk;
+        const unsigned short wb = __bfloat16_as_ushort(__float2bfloat16_rn(wf));
+        if ((wb & 0x7FFFu) == 0) return;
+        const int sr = raster_to_strip((b * s.H + yy) * s.W + xx, s.H, s.W, sw, nf, wl);
+        unsigned long long* slot = reinterpret_cast<unsigned long long*>(
+            lrecs + ((size_t)(g * mtiles_v + sr / BM) * s.K2 + tap) * BM + (sr % BM));
+        unsigned long long key = ((unsigned long long)p << 32) | ((unsigned long long)n << 16) | wb;
+#pragma unroll 1
+        for (int e = 0; e < LIST_E && key != EMPTY_KEY; ++e) {
+            const unsigned long long old = atomicMin(slot + e, key);
+            key = old == EMPTY_KEY ? EMPTY_KEY : (old > key ? old : key);
+        }
+        if (key != EMPTY_KEY) {
+            const size_t at = (size_t)gt * ovf_pitch + (size_t)(key >> 32);
+            atomicOr(reinterpret_cast<unsigned*>(ovf + (at & ~(size_t)3)), (1u << ((key >> 16) & 3u)) << (8 * (at & 3)));
+        }
+    }
+}
+
+// Pre-pass of one group's launch. Blocks [0, wblocks): W' of the virtual layer,
+// W'[c][u*64 + k] = w[o][tap][g*Cg + c] for unit u = (q, tap) (taps innermost)
+// and o = 64 q + (16*((k >> 2) & 3) + 4*(k >> 4) + (k & 3)) (zero past Cout),
+// the order the producers store a chunk in; and the stream-K counters cleared.
+// The other blocks turn the group's key lists into ListRec records in place.
+__global__ void __launch_bounds__(256) dcn_gxt_prepass_kernel(const Shape s, const bf16* __restrict__ w,
+                                                              bf16* __restrict__ wp, ListRec* __restrict__ lrecs,
+                                                              const FwdArgs a, int g, int wblocks, long long nrec) {
+    asm volatile("griddepcontrol.launch_dependents;");
+    if ((int)blockIdx.x >= wblocks) {
+        const long long r = (long long)(blockIdx.x - wblocks) * blockDim.x + threadIdx.x;
+        if (r >= nrec) return;
+        const ulonglong4 k = *reinterpret_cast<const ulonglong4*>(lrecs + r);
+        const unsigned long long ks[4] = {k.x, k.y, k.z, k.w};
+        ListRec R;
+        uint32_t wv[4];
+        R.vmask = 0u;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const bool v = ks[e] != EMPTY_KEY;
+            R.p[e] = v ? (int)(ks[e] >> 32) : 0;
+            wv[e] = v ? (uint32_t)(ks[e] & 0xFFFFu) : 0u;
+            R.vmask |= v ? 1u << e : 0u;
+        }
+        R.w10 = wv[0] | (wv[1] << 16);
+        R.w32 = wv[2] | (wv[3] << 16);
+        R.pad = 0u;
+        lrecs[r] = R;
+        return;
+    }
+    const int U = a.U;
+    const long long n8 = (long long)s.Cg * U * 8;
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < a.tiles) a.counters[i] = 0;
+    if (i >= n8) return;
+    const int c = (int)(i % s.Cg);  // consecutive threads read consecutive channels of w
+    const long long uk = i / s.Cg;
+    const int k8 = (int)(uk & 7), u = (int)(uk >> 3);
+    const int q = u / s.K2, tap = u - q * s.K2;
+    uint32_t v[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        float e2[2];
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            const int k = 8 * k8 + 2 * h + t;
+            const int o = q * BK + 16 * ((k >> 2) & 3) + 4 * (k >> 4) + (k & 3);
+            e2[t] = o < s.Cout ? __bfloat162float(w[(size_t)o * s.KC + (size_t)tap * s.Cin + (size_t)g * s.Cg + c]) : 0.f;
+        }
+        v[h] = pack_bf16(e2[0], e2[1]);
+    }
+    *reinterpret_cast<uint4*>(wp + ((size_t)c * U + u) * BK + 8 * k8) = make_uint4(v[0], v[1], v[2], v[3]);
+}
+
+// The virtual layer of the transposed pass for one group of s.
+Shape gxt_shape(const Shape& s) {
+    Shape v = s;
+    v.H = s.Ho;  // the gathered tensor: grad_y [B, Ho, Wo, Cout]
+    v.W = s.Wo;
+    v.Ho = s.H;  // rows: the input pixels
+    v.Wo = s.W;
+    v.Cin = s.Cout;
+    v.Cg = s.Cout;
+    v.G = 1;
+    v.Cout = s.Cg;
+    v.P = s.B * s.H * s.W;
+    v.KC = s.K2 * s.Cout;
+    return v;
+}
+
+struct GxtPlan {
+    bool ok;
+    Shape v;
+    TsPlan ts;
+    size_t lrec_bytes, ts_off, ws_bytes;
+};
+
+GxtPlan make_gxt_plan(const Shape& s, int sms) {
+    GxtPlan gp{};
+    gp.ok = false;
+    if (s.Cg > 256 || s.Cg % 8 || s.Cout % 8 || (long long)s.B * s.H * s.W >= (1LL << 31) / 64) return gp;
+    gp.v = gxt_shape(s);
+    gp.ts = make_ts_plan(gp.v, sms, 1);
+    if (!gp.ts.ok) return gp;
+    gp.lrec_bytes = (size_t)s.G * gp.ts.k.m_tiles * s.K2 * BM * sizeof(ListRec);
+    gp.ts_off = (gp.lrec_bytes + 255) & ~(size_t)255;
+    gp.ws_bytes = gp.ts_off + gp.ts.ws_bytes;
+    gp.ok = true;
+    return gp;
+}
+
+// The kernel arguments a plan fixes (tensors and records are set by the caller).
+TsArgs make_ts_args(const TsPlan& pl, const Shape& s, void* ws, int* counters, unsigned* status) {
+    TsArgs ta{};
     FwdArgs& a = ta.f;
     a = FwdArgs{};
     a.s = s;
-    a.x = (const bf16*)x;
-    a.off = (const bf16*)off;
-    a.mask = (const bf16*)mask;
-    a.bias = (const bf16*)bias;
-    a.y = (bf16*)y;
     a.partials = reinterpret_cast<float*>(ws);
     a.counters = counters;
     a.status = status;
@@ -786,17 +967,33 @@ cudaError_t fwd_ts(const Shape& s, const void* x, const void* off, const void* m
     ta.idle_bytes = pl.idle_bytes;
     ta.ep_len = pl.ep_len;
     ta.ep_taps = pl.ep_taps;
-    TapRec* recs = reinterpret_cast<TapRec*>(wsb + pl.ws_recs_off);
-    ta.recs = recs;
-    {
-        const long long nw = std::max<long long>((long long)s.Cout * pl.k.U * 8, pl.k.tiles);
-        const int wblocks = (int)((nw + 255) / 256);
-        const long long rblocks = (pl.nrec + 255) / 256;
-        dcn_fwd_prepass_kernel<<<(unsigned)(wblocks + rblocks), 256, 0, st>>>((const bf16*)w, wperm, recs, a, wblocks,
-                                                                             pl.nrec);
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-    }
+    return ta;
+}
+
+// The weight tensor map of a plan: W' [Cout][U*64] bf16, boxes of 64 x bn_total, 128-byte swizzle.
+bool encode_wperm(CUtensorMap* map, const TsPlan& pl, const Shape& s, const void* wperm) {
+    auto encode = get_encode();
+    if (!encode) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)pl.k.U * BK, (cuuint64_t)s.Cout};
+    cuuint64_t strides[1] = {(cuuint64_t)pl.k.U * BK * 2};
+    cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)pl.bn_total};
+    cuuint32_t estr[2] = {1, 1};
+    return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(wperm), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Launches the main kernel as a programmatic dependent of the pre-pass just enqueued on st.
+template <int MODE>
+cudaError_t launch_ts(const TsPlan& pl, const CUtensorMap& map, const TsArgs& ta, bool wide, cudaStream_t st) {
+    auto kernel = wide ? dcn_fwd_ts_kernel<true, MODE> : dcn_fwd_ts_kernel<false, MODE>;
+    static DeviceFlags attr_set[2];
+    static DeviceCarveout carve[2];
+    cudaError_t e = max_dynamic_smem_once((const void*)kernel, 227 * 1024, attr_set[wide]);
+    if (e != cudaSuccess) return e;
+    // the gather hits in L1: give it everything the kernel's shared memory does not need
+    e = smem_carveout_for((const void*)kernel, pl.smem_bytes, carve[wide]);
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)pl.k.ctas);
     cfg.blockDim = dim3(NUM_THREADS);
@@ -809,8 +1006,100 @@ cudaError_t fwd_ts(const Shape& s, const void* x, const void* off, const void* m
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, kernel, map, ta);
     if (e != cudaSuccess) return e;
-    if (launches) *launches += 2;
     return cudaGetLastError();
+}
+}  // namespace
+
+bool fwd_ts_supported(const Shape& s) { return make_ts_plan(s, num_sms()).ok; }
+
+size_t fwd_ts_workspace(const Shape& s) {
+    const TsPlan pl = make_ts_plan(s, num_sms());
+    return pl.ok ? pl.ws_bytes : 0;
+}
+
+cudaError_t fwd_ts(const Shape& s, const void* x, const void* off, const void* mask, const void* w, const void* bias,
+                   void* y, void* ws, size_t ws_bytes, unsigned* status, cudaStream_t st, int* launches) {
+    const TsPlan pl = make_ts_plan(s, num_sms());
+    if (!pl.ok || ws_bytes < pl.ws_bytes || !ws) return cudaErrorInvalidValue;
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    int* counters = reinterpret_cast<int*>(wsb + pl.ws_counters_off);
+    bf16* wperm = reinterpret_cast<bf16*>(wsb + pl.ws_wperm_off);
+    CUtensorMap map;
+    if (!encode_wperm(&map, pl, s, wperm)) return cudaErrorInvalidValue;
+    const bool wide = s.Cin % 16 == 0 && s.Cg % 16 == 0 && (reinterpret_cast<uintptr_t>(x) & 31) == 0;
+    TsArgs ta = make_ts_args(pl, s, ws, counters, status);
+    FwdArgs& a = ta.f;
+    a.x = (const bf16*)x;
+    a.off = (const bf16*)off;
+    a.mask = (const bf16*)mask;
+    a.bias = (const bf16*)bias;
+    a.y = (bf16*)y;
+    TapRec* recs = reinterpret_cast<TapRec*>(wsb + pl.ws_recs_off);
+    ta.recs = reinterpret_cast<const uint8_t*>(recs);
+    ta.yf = nullptr;
+    ta.ldy = s.Cout;
+    ta.col0 = 0;
+    const long long nw = std::max<long long>((long long)s.Cout * pl.k.U * 8, pl.k.tiles);
+    const int wblocks = (int)((nw + 255) / 256);
+    const long long rblocks = (pl.nrec + 255) / 256;
+    dcn_fwd_prepass_kernel<<<(unsigned)(wblocks + rblocks), 256, 0, st>>>((const bf16*)w, wperm, recs, a, wblocks,
+                                                                         pl.nrec);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    e = launch_ts<0>(pl, map, ta, wide, st);
+    if (e != cudaSuccess) return e;
+    if (launches) *launches += 2;
+    return cudaSuccess;
+}
+
+bool gxt_supported(const Shape& s) { return make_gxt_plan(s, num_sms()).ok; }
+
+size_t gxt_workspace(const Shape& s) {
+    const GxtPlan gp = make_gxt_plan(s, num_sms());
+    return gp.ok ? gp.ws_bytes : 0;
+}
+
+cudaError_t gxt(const Shape& s, const void* off, const void* mask, const void* w, const void* gy, float* gx,
+                uint8_t* ovf, int ovf_pitch, void* ws, size_t ws_bytes, unsigned* status, cudaStream_t st,
+                int* launches) {
+    const GxtPlan gp = make_gxt_plan(s, num_sms());
+    if (!gp.ok || !ws || ws_bytes < gp.ws_bytes || ovf_pitch < s.P) return cudaErrorInvalidValue;
+    const TsPlan& pl = gp.ts;
+    const Shape& v = gp.v;
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    ListRec* lrecs = reinterpret_cast<ListRec*>(wsb);
+    uint8_t* tws = wsb + gp.ts_off;
+    int* counters = reinterpret_cast<int*>(tws + pl.ws_counters_off);
+    bf16* wperm = reinterpret_cast<bf16*>(tws + pl.ws_wperm_off);
+    CUtensorMap map;
+    if (!encode_wperm(&map, pl, v, wperm)) return cudaErrorInvalidValue;
+    cudaError_t e = cudaMemsetAsync(lrecs, 0xFF, gp.lrec_bytes, st);  // every slot empty
+    if (e != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(ovf, 0, (size_t)s.G * s.K2 * ovf_pitch, st)) != cudaSuccess) return e;
+    dcn_gxt_fill_kernel<<<dim3((unsigned)((s.P + 255) / 256), (unsigned)(s.G * s.K2 * 4)), 256, 0, st>>>(
+        s, (const bf16*)off, (const bf16*)mask, lrecs, ovf, ovf_pitch, pl.k.m_tiles, pl.k.sw, pl.k.nf, pl.k.wl);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const bool wide = v.Cin % 16 == 0 && (reinterpret_cast<uintptr_t>(gy) & 31) == 0;
+    const long long per_g = (long long)pl.k.m_tiles * s.K2 * BM;
+    const long long nw = std::max<long long>((long long)v.Cout * pl.k.U * 8, pl.k.tiles);
+    const int wblocks = (int)((nw + 255) / 256);
+    const long long rblocks = (per_g + 255) / 256;
+    int n = 3;
+    for (int g = 0; g < s.G; ++g) {
+        TsArgs ta = make_ts_args(pl, v, tws, counters, status);
+        ta.f.x = (const bf16*)gy;
+        ta.recs = reinterpret_cast<const uint8_t*>(lrecs + g * per_g);
+        ta.yf = gx;
+        ta.ldy = s.Cin;
+        ta.col0 = g * s.Cg;
+        dcn_gxt_prepass_kernel<<<(unsigned)(wblocks + rblocks), 256, 0, st>>>(
+            s, (const bf16*)w, wperm, lrecs + g * per_g, ta.f, g, wblocks, per_g);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if ((e = launch_ts<1>(pl, map, ta, wide, st)) != cudaSuccess) return e;
+        n += 2;
+    }
+    if (launches) *launches += n;
+    return cudaSuccess;
 }
 
 }  // namespace dcn

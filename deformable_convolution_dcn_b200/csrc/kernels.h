@@ -79,6 +79,16 @@ bool fwd_f32_small_supported(const Shape& s);
 cudaError_t fwd_f32_small(const Shape& s, const void* x, const void* off, const void* mask, const void* w,
                           const void* bias, void* y, cudaStream_t st);
 
+// fwd_tc_ts.cu, transposed pass — grad_x of a bfloat16 layer (channels per group
+// <= 256) as a gather-GEMM on tcgen05, written outright (no atomics, no zeroing).
+// Sample corners past a list's capacity are not included: they are flagged in
+// ovf[(g*K2 + tap) * ovf_pitch + p] (bit n = corner n) for the caller to add.
+bool gxt_supported(const Shape& s);
+size_t gxt_workspace(const Shape& s);
+cudaError_t gxt(const Shape& s, const void* off, const void* mask, const void* w, const void* gy, float* gx,
+                uint8_t* ovf, int ovf_pitch, void* ws, size_t ws_bytes, unsigned* status, cudaStream_t st,
+                int* launches);
+
 // bwd_weight_tc.cu — bfloat16 weight gradient on tcgen05 (workspace: sampling records).
 bool bwd_weight_tc_supported(const Shape& s);
 size_t bwd_weight_tc_workspace(const Shape& s);
