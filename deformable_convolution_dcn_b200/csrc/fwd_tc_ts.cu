@@ -79,17 +79,36 @@ constexpr int MAX_TAPS_TS = 49;
 constexpr int TAP_TABLE = 64;  // entries of the shared-memory tap table
 
 // Gather record of the transposed pass (MODE 1, the grad_x contraction): up
-// to LIST_E (dY row, weight) entries of one (input pixel, tap); entry e is
-// read when bit e of vmask is set. The weights pair up as in TapRec, so the
-// same packed blend sums them.
+// to LIST_E (dY row, weight) entries of one (input pixel, tap), gathered in
+// batches of four; entry e is read when bit e of vmask is set. The weights
+// pair up as in TapRec, so the same packed blend sums each batch. (Eight
+// entries in two batches halve the corners left to the atomic scatter but
+// expose the second batch's load latency: slower overall on conv4.)
 constexpr int LIST_E = 4;
 struct __align__(16) ListRec {
     int p[LIST_E];  // dY rows: output pixels (b*Ho + ho)*Wo + wo whose sample reaches this pixel
-    uint32_t w10;   // lo: entry 0's weight m * (corner weight), hi: entry 1's (bf16)
-    uint32_t w32;   // lo: entry 2's, hi: entry 3's
+    uint32_t w[LIST_E / 2];  // w[i]: lo = entry 2i's weight m * (corner weight), hi = entry 2i+1's (bf16)
     uint32_t vmask;
-    uint32_t pad;
+    uint32_t pad[LIST_E == 4 ? 1 : 3];
 };
+static_assert(sizeof(ListRec) == 8 * LIST_E, "ListRec: 16-byte multiple");
+
+// r += the blend of four neighbour slices (as blend16, accumulating).
+__device__ __forceinline__ void blend16_acc(uint32_t (&r)[8], const uint32_t (&v)[4][8], uint32_t w01_00,
+                                            uint32_t w11_10) {
+    const uint32_t w00 = __byte_perm(w01_00, 0, 0x1010), w01 = __byte_perm(w01_00, 0, 0x3232);
+    const uint32_t w10 = __byte_perm(w11_10, 0, 0x1010), w11 = __byte_perm(w11_10, 0, 0x3232);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        asm("{\n\t"
+            "fma.rn.bf16x2 %0, %1, %5, %0;\n\t"
+            "fma.rn.bf16x2 %0, %2, %6, %0;\n\t"
+            "fma.rn.bf16x2 %0, %3, %7, %0;\n\t"
+            "fma.rn.bf16x2 %0, %4, %8, %0;\n\t}"
+            : "+r"(r[q])
+            : "r"(v[0][q]), "r"(v[1][q]), "r"(v[2][q]), "r"(v[3][q]), "r"(w00), "r"(w01), "r"(w10), "r"(w11));
+    }
+}
 
 struct TsArgs {
     FwdArgs f;
@@ -276,7 +295,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             irb = ta.ep_taps == s.K2 ? 0 : ich.tap - ich.tap % s.K;
         }
         // loads of row `row` of the cursor chunk into v, its weights into w
-        auto issue = [&](uint32_t(&v)[4][8], uint32_t(&w)[2], int row) {
+        // batch: MODE 1's entries 4*batch .. 4*batch + 3
+        auto issue = [&](uint32_t(&v)[4][8], uint32_t(&w)[2], int row, int batch = 0) {
             const int cg = ich.q * BK + j4 * SLICE_CH;
             const uint32_t cmask = cg < s.Cg ? 0xFu : 0u;
             const bool hi_ok = cg + 8 < s.Cg;  // upper 8 channels present (narrow loads only)
@@ -295,11 +315,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 pc[2] = p + rp2;
                 pc[3] = p + rp2 + cin2;
             } else {
-                const uint4 pe = ptx::lds_v4(ra);       // ListRec::p
-                const uint4 rw = ptx::lds_v4(ra + 16);  // ListRec::w10, w32, vmask
-                w[0] = rw.x;
-                w[1] = rw.y;
-                vm = rw.z & cmask;
+                const uint4 pe = ptx::lds_v4(ra + 16 * batch);  // ListRec::p of the batch
+                if constexpr (LIST_E == 4) {
+                    const uint4 rw = ptx::lds_v4(ra + 16);  // ListRec::w, vmask
+                    w[0] = rw.x;
+                    w[1] = rw.y;
+                    vm = rw.z & cmask;
+                } else {
+                    const uint4 rw = ptx::lds_v4(ra + 4 * LIST_E);  // ListRec::w
+                    const uint32_t vall = ptx::lds_v4(ra + 6 * LIST_E).x;  // ListRec::vmask
+                    w[0] = batch ? rw.z : rw.x;
+                    w[1] = batch ? rw.w : rw.y;
+                    vm = (vall >> (4 * batch)) & cmask;
+                }
                 pc[0] = xc + (long long)(int)pe.x * cin2;
                 pc[1] = xc + (long long)(int)pe.y * cin2;
                 pc[2] = xc + (long long)(int)pe.z * cin2;
@@ -366,15 +394,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 break;
             }
             const bool more = n + 1 < total;
-            uint32_t r[16];
-            {
-                uint32_t t[8];
-                blend16(t, va, wa[0], wa[1]);
-#pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    r[4 * m] = t[2 * m];
-                    r[4 * m + 1] = t[2 * m + 1];
-                }
+            uint32_t ta8[8], tb8[8];
+            blend16(ta8, va, wa[0], wa[1]);
+            if constexpr (MODE == 1 && LIST_E > 4) {
+                // entries 4..7 of both rows of this chunk, then on to the next chunk
+                issue(va, wa, r0, 1);
+                blend16(tb8, vb, wb[0], wb[1]);
+                issue(vb, wb, r1, 1);
+                blend16_acc(ta8, va, wa[0], wa[1]);
             }
             if (more) {
                 if (!advance()) {
@@ -383,16 +410,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 }
                 issue(va, wa, r0);
             }
-            {
-                uint32_t t[8];
-                blend16(t, vb, wb[0], wb[1]);
-#pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    r[4 * m + 2] = t[2 * m];
-                    r[4 * m + 3] = t[2 * m + 1];
-                }
-            }
+            if constexpr (MODE == 1 && LIST_E > 4) blend16_acc(tb8, vb, wb[0], wb[1]);
+            else blend16(tb8, vb, wb[0], wb[1]);
             if (more) issue(vb, wb, r1);
+            uint32_t r[16];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                r[4 * m] = ta8[2 * m];
+                r[4 * m + 1] = ta8[2 * m + 1];
+                r[4 * m + 2] = tb8[2 * m];
+                r[4 * m + 3] = tb8[2 * m + 1];
+            }
             // the previous chunk's store has had this chunk's blend to land: publish it
             if (prev >= 0) {
                 tmem_wait_st();
@@ -746,8 +774,8 @@ TsPlan make_ts_plan(const Shape& s, int sms, int mode = 0) {
     pl.b_stage_bytes = (uint32_t)pl.bn_total * 128;
     pl.b_stages = std::min(DCN_FWD_TS_B_STAGES, MAX_B_STAGES);
     const uint32_t ring = (uint32_t)pl.b_stages * pl.b_stage_bytes;
-    // all taps of a (tile, group) per record buffer when they fit in 36 KB, else one kernel row
-    const bool all_taps = s.K2 <= ALL_TAPS && 2u * BM * s.K2 * rec_bytes <= 36u * 1024u;
+    // all taps of a (tile, group) per record buffer when both buffers fit in 80 KB, else one kernel row
+    const bool all_taps = s.K2 <= ALL_TAPS && 2u * BM * s.K2 * rec_bytes <= 80u * 1024u;
     pl.ep_taps = all_taps ? s.K2 : s.K;
     pl.ep_len = all_taps ? pl.k.nq * s.K2 : s.K;
     const uint32_t info_bytes = 2u * BM * (uint32_t)pl.ep_taps * rec_bytes;
@@ -790,18 +818,18 @@ __device__ __forceinline__ int raster_to_strip(int q, int H, int W, int sw, int 
     return b * plane + nf * H * sw + y * wl + (xx - nf * sw);
 }
 
-// One thread per (output pixel p, group-tap gt, corner n): the corner is
-// inserted into its input pixel's list, which keeps the LIST_E
-// smallest keys (p << 32 | n << 16 | bf16 weight) in ascending order: a key
-// goes down the slots with atomicMin, carrying on with whichever of it and
-// the slot's old key is larger, until it fills an empty slot (all bits set
-// on entry) or falls off the end. The lists and the set of corners that fall
-// off (flagged in ovf[gt * ovf_pitch + p'], bit n', zero on entry) therefore
-// do not depend on the order of the insertions. Corners outside the map or of
-// zero (bf16) weight add nothing and are skipped.
-constexpr unsigned long long EMPTY_KEY = ~0ull;
+// One thread per (output pixel p, group-tap gt, corner n): the corner's key
+// (p << 32 | n << 16 | bf16 weight) takes the next slot of its input pixel's
+// list (LIST_CAP slots; the count in cnt, zero on entry). A corner past the
+// last slot flags itself in ovf[gt * ovf_pitch + p] (bit n, zero on entry);
+// the pre-pass below sorts each list and keeps its LIST_E smallest keys, so
+// the lists and the flagged corners do not depend on the order of the
+// insertions. Corners outside the map or of zero (bf16) weight add nothing
+// and are skipped.
+constexpr int LIST_CAP = 2 * LIST_E;
 __global__ void __launch_bounds__(256) dcn_gxt_fill_kernel(const Shape s, const bf16* __restrict__ off,
-                                                           const bf16* __restrict__ mask, ListRec* __restrict__ lrecs,
+                                                           const bf16* __restrict__ mask, int* __restrict__ cnt,
+                                                           unsigned long long* __restrict__ keys,
                                                            uint8_t* __restrict__ ovf, int ovf_pitch, int mtiles_v,
                                                            int sw, int nf, int wl) {
     const int p = blockIdx.x * blockDim.x + threadIdx.x;
@@ -820,25 +848,19 @@ __global__ void __launch_bounds__(256) dcn_gxt_fill_kernel(const Shape s, const 
     float ly, lx;
     split_coord(ho * s.stride - s.pad + i * s.dil, dy, y0, ly);
     split_coord(wo * s.stride - s.pad + j * s.dil, dx, x0, lx);
-    {
-        const int yy = y0 + (n >> 1), xx = x0 + (n & 1);
-        if (!inside(s, yy, xx)) return;
-        const float wf = ((n >> 1) ? ly : 1.f - ly) * ((n & 1) ? lx : 1.f - lx) * mk;
-        const unsigned short wb = __bfloat16_as_ushort(__float2bfloat16_rn(wf));
-        if ((wb & 0x7FFFu) == 0) return;
-        const int sr = raster_to_strip((b * s.H + yy) * s.W + xx, s.H, s.W, sw, nf, wl);
-        unsigned long long* slot = reinterpret_cast<unsigned long long*>(
-            lrecs + ((size_t)(g * mtiles_v + sr / BM) * s.K2 + tap) * BM + (sr % BM));
-        unsigned long long key = ((unsigned long long)p << 32) | ((unsigned long long)n << 16) | wb;
-#pragma unroll 1
-        for (int e = 0; e < LIST_E && key != EMPTY_KEY; ++e) {
-            const unsigned long long old = atomicMin(slot + e, key);
-            key = old == EMPTY_KEY ? EMPTY_KEY : (old > key ? old : key);
-        }
-        if (key != EMPTY_KEY) {
-            const size_t at = (size_t)gt * ovf_pitch + (size_t)(key >> 32);
-            atomicOr(reinterpret_cast<unsigned*>(ovf + (at & ~(size_t)3)), (1u << ((key >> 16) & 3u)) << (8 * (at & 3)));
-        }
+    const int yy = y0 + (n >> 1), xx = x0 + (n & 1);
+    if (!inside(s, yy, xx)) return;
+    const float wf = ((n >> 1) ? ly : 1.f - ly) * ((n & 1) ? lx : 1.f - lx) * mk;
+    const unsigned short wb = __bfloat16_as_ushort(__float2bfloat16_rn(wf));
+    if ((wb & 0x7FFFu) == 0) return;
+    const int sr = raster_to_strip((b * s.H + yy) * s.W + xx, s.H, s.W, sw, nf, wl);
+    const size_t L = ((size_t)(g * mtiles_v + sr / BM) * s.K2 + tap) * BM + (sr % BM);
+    const int slot = atomicAdd(cnt + L, 1);
+    if (slot < LIST_CAP) {
+        keys[L * LIST_CAP + slot] = ((unsigned long long)p << 32) | ((unsigned long long)n << 16) | wb;
+    } else {
+        const size_t at = (size_t)gt * ovf_pitch + p;
+        atomicOr(reinterpret_cast<unsigned*>(ovf + (at & ~(size_t)3)), (1u << n) << (8 * (at & 3)));
     }
 }
 
@@ -846,29 +868,58 @@ __global__ void __launch_bounds__(256) dcn_gxt_fill_kernel(const Shape s, const 
 // W'[c][u*64 + k] = w[o][tap][g*Cg + c] for unit u = (q, tap) (taps innermost)
 // and o = 64 q + (16*((k >> 2) & 3) + 4*(k >> 4) + (k & 3)) (zero past Cout),
 // the order the producers store a chunk in; and the stream-K counters cleared.
-// The other blocks turn the group's key lists into ListRec records in place.
+// The other blocks turn the group's lists into ListRec records: a list of at
+// most LIST_CAP keys keeps its LIST_E smallest and flags the rest in ovf; a
+// longer one (some of its keys were never stored) flags all it holds and keeps
+// none, its other corners having flagged themselves.
 __global__ void __launch_bounds__(256) dcn_gxt_prepass_kernel(const Shape s, const bf16* __restrict__ w,
                                                               bf16* __restrict__ wp, ListRec* __restrict__ lrecs,
+                                                              const int* __restrict__ cnt,
+                                                              const unsigned long long* __restrict__ keys,
+                                                              uint8_t* __restrict__ ovf, int ovf_pitch,
                                                               const FwdArgs a, int g, int wblocks, long long nrec) {
     asm volatile("griddepcontrol.launch_dependents;");
     if ((int)blockIdx.x >= wblocks) {
         const long long r = (long long)(blockIdx.x - wblocks) * blockDim.x + threadIdx.x;
         if (r >= nrec) return;
-        const ulonglong4 k = *reinterpret_cast<const ulonglong4*>(lrecs + r);
-        const unsigned long long ks[4] = {k.x, k.y, k.z, k.w};
+        const int c = cnt[r];
+        const int tap = (int)((r / BM) % s.K2);
+        const size_t gt = (size_t)g * s.K2 + tap;
+        unsigned long long k[LIST_CAP];
+        const int m = c < LIST_CAP ? c : LIST_CAP;
+#pragma unroll
+        for (int e = 0; e < LIST_CAP; ++e) k[e] = e < m ? keys[r * LIST_CAP + e] : ~0ull;
+        // ascending order (insertion sort over the fixed-size array)
+#pragma unroll
+        for (int e = 1; e < LIST_CAP; ++e)
+#pragma unroll
+            for (int f = e; f > 0; --f) {
+                const unsigned long long lo = k[f - 1] < k[f] ? k[f - 1] : k[f];
+                const unsigned long long hi = k[f - 1] < k[f] ? k[f] : k[f - 1];
+                k[f - 1] = lo;
+                k[f] = hi;
+            }
+        const int keep = c > LIST_CAP ? 0 : (c < LIST_E ? c : LIST_E);
+#pragma unroll
+        for (int e = 0; e < LIST_CAP; ++e) {
+            if (e < keep || e >= m) continue;
+            const size_t at = gt * ovf_pitch + (size_t)(k[e] >> 32);
+            atomicOr(reinterpret_cast<unsigned*>(ovf + (at & ~(size_t)3)), (1u << ((k[e] >> 16) & 3u)) << (8 * (at & 3)));
+        }
         ListRec R;
-        uint32_t wv[4];
+        uint32_t wv[LIST_E];
         R.vmask = 0u;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const bool v = ks[e] != EMPTY_KEY;
-            R.p[e] = v ? (int)(ks[e] >> 32) : 0;
-            wv[e] = v ? (uint32_t)(ks[e] & 0xFFFFu) : 0u;
+        for (int e = 0; e < LIST_E; ++e) {
+            const bool v = e < keep;
+            R.p[e] = v ? (int)(k[e] >> 32) : 0;
+            wv[e] = v ? (uint32_t)(k[e] & 0xFFFFu) : 0u;
             R.vmask |= v ? 1u << e : 0u;
         }
-        R.w10 = wv[0] | (wv[1] << 16);
-        R.w32 = wv[2] | (wv[3] << 16);
-        R.pad = 0u;
+#pragma unroll
+        for (int e = 0; e < LIST_E / 2; ++e) R.w[e] = wv[2 * e] | (wv[2 * e + 1] << 16);
+#pragma unroll
+        for (int e = 0; e < (int)(sizeof(R.pad) / 4); ++e) R.pad[e] = 0u;
         lrecs[r] = R;
         return;
     }
@@ -916,7 +967,7 @@ struct GxtPlan {
     bool ok;
     Shape v;
     TsPlan ts;
-    size_t lrec_bytes, ts_off, ws_bytes;
+    size_t lists, lrec_bytes, cnt_off, keys_off, ts_off, ws_bytes;
 };
 
 GxtPlan make_gxt_plan(const Shape& s, int sms) {
@@ -926,8 +977,11 @@ GxtPlan make_gxt_plan(const Shape& s, int sms) {
     gp.v = gxt_shape(s);
     gp.ts = make_ts_plan(gp.v, sms, 1);
     if (!gp.ts.ok) return gp;
-    gp.lrec_bytes = (size_t)s.G * gp.ts.k.m_tiles * s.K2 * BM * sizeof(ListRec);
-    gp.ts_off = (gp.lrec_bytes + 255) & ~(size_t)255;
+    gp.lists = (size_t)s.G * gp.ts.k.m_tiles * s.K2 * BM;
+    gp.lrec_bytes = gp.lists * sizeof(ListRec);
+    gp.cnt_off = (gp.lrec_bytes + 255) & ~(size_t)255;
+    gp.keys_off = (gp.cnt_off + gp.lists * sizeof(int) + 255) & ~(size_t)255;
+    gp.ts_off = (gp.keys_off + gp.lists * LIST_CAP * sizeof(unsigned long long) + 255) & ~(size_t)255;
     gp.ws_bytes = gp.ts_off + gp.ts.ws_bytes;
     gp.ok = true;
     return gp;
@@ -1068,16 +1122,18 @@ cudaError_t gxt(const Shape& s, const void* off, const void* mask, const void* w
     const Shape& v = gp.v;
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     ListRec* lrecs = reinterpret_cast<ListRec*>(wsb);
+    int* cnt = reinterpret_cast<int*>(wsb + gp.cnt_off);
+    unsigned long long* keys = reinterpret_cast<unsigned long long*>(wsb + gp.keys_off);
     uint8_t* tws = wsb + gp.ts_off;
     int* counters = reinterpret_cast<int*>(tws + pl.ws_counters_off);
     bf16* wperm = reinterpret_cast<bf16*>(tws + pl.ws_wperm_off);
     CUtensorMap map;
     if (!encode_wperm(&map, pl, v, wperm)) return cudaErrorInvalidValue;
-    cudaError_t e = cudaMemsetAsync(lrecs, 0xFF, gp.lrec_bytes, st);  // every slot empty
+    cudaError_t e = cudaMemsetAsync(cnt, 0, gp.lists * sizeof(int), st);
     if (e != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(ovf, 0, (size_t)s.G * s.K2 * ovf_pitch, st)) != cudaSuccess) return e;
     dcn_gxt_fill_kernel<<<dim3((unsigned)((s.P + 255) / 256), (unsigned)(s.G * s.K2 * 4)), 256, 0, st>>>(
-        s, (const bf16*)off, (const bf16*)mask, lrecs, ovf, ovf_pitch, pl.k.m_tiles, pl.k.sw, pl.k.nf, pl.k.wl);
+        s, (const bf16*)off, (const bf16*)mask, cnt, keys, ovf, ovf_pitch, pl.k.m_tiles, pl.k.sw, pl.k.nf, pl.k.wl);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const bool wide = v.Cin % 16 == 0 && (reinterpret_cast<uintptr_t>(gy) & 31) == 0;
     const long long per_g = (long long)pl.k.m_tiles * s.K2 * BM;
@@ -1093,7 +1149,8 @@ cudaError_t gxt(const Shape& s, const void* off, const void* mask, const void* w
         ta.ldy = s.Cin;
         ta.col0 = g * s.Cg;
         dcn_gxt_prepass_kernel<<<(unsigned)(wblocks + rblocks), 256, 0, st>>>(
-            s, (const bf16*)w, wperm, lrecs + g * per_g, ta.f, g, wblocks, per_g);
+            s, (const bf16*)w, wperm, lrecs + g * per_g, cnt + g * per_g, keys + (size_t)g * per_g * LIST_CAP, ovf,
+            ovf_pitch, ta.f, g, wblocks, per_g);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         if ((e = launch_ts<1>(pl, map, ta, wide, st)) != cudaSuccess) return e;
         n += 2;
