@@ -105,6 +105,31 @@ def test_samples_all_outside_give_bias(dtype):
     assert float(g["grad_weight"].abs().max()) == 0.0
 
 
+@pytest.mark.parametrize("spread", [0.3, 2.5], ids=["converging", "crowded"])
+def test_backward_converging_samples(spread):
+    """Offsets that pull every sample of a tap towards one point of the map: the
+    input pixels there receive far more bilinear corners than the per-pixel
+    lists of the transposed grad_x pass hold (spread 0.3: hundreds each, all
+    left to the atomic scatter; 2.5: tens, partly kept). Full backward against
+    the oracle, element by element."""
+    s, d = gen.random_case(21, "bf16", B=2, Cin=64, Cout=64, H=11, W=13, K=3, stride=1, pad=1, dil=1, G=1)
+    g = torch.Generator().manual_seed(22)
+    ho = torch.arange(s.Ho, dtype=torch.float32).view(1, 1, s.Ho, 1)
+    wo = torch.arange(s.Wo, dtype=torch.float32).view(1, 1, 1, s.Wo)
+    off = torch.empty((s.B, 2 * s.K * s.K, s.Ho, s.Wo))
+    for tap in range(s.K * s.K):
+        i, j = divmod(tap, s.K)
+        # sample row = ho - pad + i + dy lands near row 5.3, column near 6.6
+        off[:, 2 * tap] = (5.3 - (ho - s.pad + i) + spread * torch.randn((s.B, 1, s.Ho, s.Wo), generator=g))[:, 0]
+        off[:, 2 * tap + 1] = (6.6 - (wo - s.pad + j) + spread * torch.randn((s.B, 1, s.Ho, s.Wo), generator=g))[:, 0]
+    d["offset"] = off.to(d["offset"].dtype)
+    a = f64(d)
+    g_ = run_backward(s, to_dev(d))
+    ref = _oracle_backward(s, a)
+    for k in ("grad_x", "grad_offset", "grad_mask", "grad_weight", "grad_bias"):
+        assert_close(_cpu(g_[k]), ref[k], "bf16", k)
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_mask_zero_gives_bias(dtype):
     s, d = gen.random_case(4, dtype, Cin=32, Cout=16, H=8, W=10)
