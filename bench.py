@@ -393,14 +393,20 @@ def load_traffic(workload, kernel, path=None):
     """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
     committed ncu summary profiles/traffic.json, or None: None as well when the
     kernel's source file has changed since the counters were taken (each entry
-    records the source file and its digest at capture time)."""
+    records the source file and its digest at capture time; a pass of several
+    kernels, their sum and a list of files and digests)."""
     path = path or os.path.join(ROOT, "profiles", "traffic.json")
     try:
         e = json.load(open(path))[workload][kernel]
     except Exception:
         return None
     if isinstance(e, dict):
-        if e.get("sha") != _source_digest(e.get("source", "")):
+        # a pass of several kernels lists every source file and its digest
+        srcs, shas = e.get("source", ""), e.get("sha")
+        if isinstance(srcs, str):
+            srcs, shas = [srcs], [shas]
+        if not isinstance(shas, list) or len(shas) != len(srcs) or \
+                any(h != _source_digest(f) for f, h in zip(srcs, shas)):
             return None
         return e.get("bytes")
     return None

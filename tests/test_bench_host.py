@@ -64,10 +64,14 @@ def test_committed_traffic_figures_are_read():
             continue
         for k, v in kernels.items():
             assert v["bytes"] > 0
-            src = os.path.join(ROOT, "deformable_convolution_dcn_b200", "csrc", v["source"])
-            assert os.path.exists(src)
-            # a figure is reported only while its kernel's source is the one it was taken on
-            fresh = v["sha"] == bench._source_digest(v["source"])
+            srcs = v["source"] if isinstance(v["source"], list) else [v["source"]]
+            shas = v["sha"] if isinstance(v["sha"], list) else [v["sha"]]
+            for f in srcs:
+                assert os.path.exists(os.path.join(ROOT, "deformable_convolution_dcn_b200", "csrc", f))
+            if "kernels" in v:  # a pass of several kernels: their sum
+                assert sum(v["kernels"].values()) == v["bytes"]
+            # a figure is reported only while its kernels' sources are the ones it was taken on
+            fresh = all(h == bench._source_digest(f) for f, h in zip(srcs, shas))
             assert bench.load_traffic(wl, k) == (v["bytes"] if fresh else None)
     assert bench.load_traffic("conv4", "no_such_kernel") is None
 
@@ -79,6 +83,13 @@ def test_traffic_of_a_changed_kernel_is_dropped(tmp_path):
                                        "backward_data": {"bytes": 456, "source": "fwd_tc.cu", "sha": "0" * 16}}}))
     assert bench.load_traffic("conv4", "forward", path=str(p)) == 123
     assert bench.load_traffic("conv4", "backward_data", path=str(p)) is None
+    # a pass of several kernels: every listed source must be unchanged
+    other = bench._source_digest("bwd_data_tc.cu")
+    p.write_text(json.dumps({"conv4": {
+        "backward_data": {"bytes": 7, "source": ["fwd_tc.cu", "bwd_data_tc.cu"], "sha": [good, other]},
+        "backward_weight": {"bytes": 8, "source": ["fwd_tc.cu", "bwd_data_tc.cu"], "sha": [good, "0" * 16]}}}))
+    assert bench.load_traffic("conv4", "backward_data", path=str(p)) == 7
+    assert bench.load_traffic("conv4", "backward_weight", path=str(p)) is None
 
 
 def test_arguments_are_checked():
