@@ -672,16 +672,19 @@ cudaError_t bwd_data_tc(const Shape& s, const void* x, const void* off, const vo
     if (pl.epi) dcn_transpose_kernel<true><<<tg, dim3(32, 8), 0, st>>>((const bf16*)w, wt, s.Cout, s.KC);
     else dcn_transpose_kernel<false><<<tg, dim3(32, 8), 0, st>>>((const bf16*)w, wt, s.Cout, s.KC);
     ++n;
-    dim3 rg((pl.ppad + 255) / 256, s.G * s.K2);
-    dcn_records_f32_kernel<<<rg, 256, 0, st>>>(s, (const bf16*)off, (const bf16*)mask, rec, pl.ppad);
-    ++n;
+    // the sampling records: written by the transposed pass's fill kernel when it runs, else here
+    if (!(gx && pl.gxt)) {
+        dim3 rg((pl.ppad + 255) / 256, s.G * s.K2);
+        dcn_records_f32_kernel<<<rg, 256, 0, st>>>(s, (const bf16*)off, (const bf16*)mask, rec, pl.ppad);
+        ++n;
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // grad_x: the transposed gather-GEMM writes it (all but the flagged corners, which this
     // file's kernel then adds with atomics); otherwise zeroed here and scattered in full
     const uint8_t* ovf = nullptr;
     if (gx && pl.gxt) {
         uint8_t* ovf_w = static_cast<uint8_t*>(ws) + pl.ovf_off;
-        e = gxt(s, off, mask, w, gy, gx, ovf_w, pl.ppad, static_cast<uint8_t*>(ws) + pl.gxt_off,
+        e = gxt(s, off, mask, w, gy, gx, ovf_w, rec, pl.ppad, static_cast<uint8_t*>(ws) + pl.gxt_off,
                 ws_bytes - pl.gxt_off, status, st, &n);
         if (e != cudaSuccess) return e;
         ovf = ovf_w;

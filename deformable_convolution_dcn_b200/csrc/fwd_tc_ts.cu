@@ -825,13 +825,17 @@ __device__ __forceinline__ int raster_to_strip(int q, int H, int W, int sw, int 
 // the pre-pass below sorts each list and keeps its LIST_E smallest keys, so
 // the lists and the flagged corners do not depend on the order of the
 // insertions. Corners outside the map or of zero (bf16) weight add nothing
-// and are skipped.
+// and are skipped. The corner-0 thread also writes the sample's float32
+// record for the backward-data kernel (rec[gt * ovf_pitch + p]: fractions,
+// mask, (y0 + 1) << 16 | (x0 + 1), or all bits set when no corner is inside).
 constexpr int LIST_CAP = 2 * LIST_E;
 __global__ void __launch_bounds__(256) dcn_gxt_fill_kernel(const Shape s, const bf16* __restrict__ off,
                                                            const bf16* __restrict__ mask, int* __restrict__ cnt,
                                                            unsigned long long* __restrict__ keys,
-                                                           uint8_t* __restrict__ ovf, int ovf_pitch, int mtiles_v,
-                                                           int sw, int nf, int wl) {
+                                                           uint8_t* __restrict__ ovf, float4* __restrict__ rec,
+                                                           int ovf_pitch, int mtiles_v, int sw, int nf, int wl) {
+    // the pre-pass may start: its weight blocks do not read what this grid writes
+    asm volatile("griddepcontrol.launch_dependents;");
     const int p = blockIdx.x * blockDim.x + threadIdx.x;
     const int gt = blockIdx.y >> 2, n = blockIdx.y & 3;
     if (p >= s.P) return;
@@ -848,6 +852,11 @@ __global__ void __launch_bounds__(256) dcn_gxt_fill_kernel(const Shape s, const 
     float ly, lx;
     split_coord(ho * s.stride - s.pad + i * s.dil, dy, y0, ly);
     split_coord(wo * s.stride - s.pad + j * s.dil, dx, x0, lx);
+    if (n == 0 && rec) {
+        const bool any = inside(s, y0, x0) || inside(s, y0, x0 + 1) || inside(s, y0 + 1, x0) || inside(s, y0 + 1, x0 + 1);
+        rec[(size_t)gt * ovf_pitch + p] =
+            make_float4(ly, lx, mk, __uint_as_float(any ? (((uint32_t)(y0 + 1) << 16) | (uint32_t)(x0 + 1)) : 0xFFFFFFFFu));
+    }
     const int yy = y0 + (n >> 1), xx = x0 + (n & 1);
     if (!inside(s, yy, xx)) return;
     const float wf = ((n >> 1) ? ly : 1.f - ly) * ((n & 1) ? lx : 1.f - lx) * mk;
@@ -880,6 +889,8 @@ __global__ void __launch_bounds__(256) dcn_gxt_prepass_kernel(const Shape s, con
                                                               const FwdArgs a, int g, int wblocks, long long nrec) {
     asm volatile("griddepcontrol.launch_dependents;");
     if ((int)blockIdx.x >= wblocks) {
+        // the lists are complete once the fill grid is (launched as its programmatic dependent)
+        asm volatile("griddepcontrol.wait;" ::: "memory");
         const long long r = (long long)(blockIdx.x - wblocks) * blockDim.x + threadIdx.x;
         if (r >= nrec) return;
         const int c = cnt[r];
@@ -1114,7 +1125,7 @@ size_t gxt_workspace(const Shape& s) {
 }
 
 cudaError_t gxt(const Shape& s, const void* off, const void* mask, const void* w, const void* gy, float* gx,
-                uint8_t* ovf, int ovf_pitch, void* ws, size_t ws_bytes, unsigned* status, cudaStream_t st,
+                uint8_t* ovf, void* rec, int ovf_pitch, void* ws, size_t ws_bytes, unsigned* status, cudaStream_t st,
                 int* launches) {
     const GxtPlan gp = make_gxt_plan(s, num_sms());
     if (!gp.ok || !ws || ws_bytes < gp.ws_bytes || ovf_pitch < s.P) return cudaErrorInvalidValue;
@@ -1133,7 +1144,8 @@ cudaError_t gxt(const Shape& s, const void* off, const void* mask, const void* w
     if (e != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(ovf, 0, (size_t)s.G * s.K2 * ovf_pitch, st)) != cudaSuccess) return e;
     dcn_gxt_fill_kernel<<<dim3((unsigned)((s.P + 255) / 256), (unsigned)(s.G * s.K2 * 4)), 256, 0, st>>>(
-        s, (const bf16*)off, (const bf16*)mask, cnt, keys, ovf, ovf_pitch, pl.k.m_tiles, pl.k.sw, pl.k.nf, pl.k.wl);
+        s, (const bf16*)off, (const bf16*)mask, cnt, keys, ovf, static_cast<float4*>(rec), ovf_pitch, pl.k.m_tiles,
+        pl.k.sw, pl.k.nf, pl.k.wl);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const bool wide = v.Cin % 16 == 0 && (reinterpret_cast<uintptr_t>(gy) & 31) == 0;
     const long long per_g = (long long)pl.k.m_tiles * s.K2 * BM;
@@ -1148,9 +1160,23 @@ cudaError_t gxt(const Shape& s, const void* off, const void* mask, const void* w
         ta.yf = gx;
         ta.ldy = s.Cin;
         ta.col0 = g * s.Cg;
-        dcn_gxt_prepass_kernel<<<(unsigned)(wblocks + rblocks), 256, 0, st>>>(
-            s, (const bf16*)w, wperm, lrecs + g * per_g, cnt + g * per_g, keys + (size_t)g * per_g * LIST_CAP, ovf,
-            ovf_pitch, ta.f, g, wblocks, per_g);
+        {
+            // a programmatic dependent of the fill (group 0; later groups follow the previous main kernel,
+            // which lets no dependent start early)
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3((unsigned)(wblocks + rblocks));
+            cfg.blockDim = dim3(256);
+            cfg.stream = st;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr[0].val.programmaticStreamSerializationAllowed = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            e = cudaLaunchKernelEx(&cfg, dcn_gxt_prepass_kernel, s, (const bf16*)w, wperm, lrecs + g * per_g,
+                                   (const int*)(cnt + g * per_g), (const unsigned long long*)(keys + (size_t)g * per_g * LIST_CAP),
+                                   ovf, ovf_pitch, ta.f, g, wblocks, per_g);
+            if (e != cudaSuccess) return e;
+        }
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         if ((e = launch_ts<1>(pl, map, ta, wide, st)) != cudaSuccess) return e;
         n += 2;

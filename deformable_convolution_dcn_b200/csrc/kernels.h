@@ -83,11 +83,13 @@ cudaError_t fwd_f32_small(const Shape& s, const void* x, const void* off, const 
 // <= 256) as a gather-GEMM on tcgen05, written outright (no atomics, no zeroing).
 // Sample corners past a list's capacity are not included: they are flagged in
 // ovf[(g*K2 + tap) * ovf_pitch + p] (bit n = corner n) for the caller to add.
+// rec (optional): the float32 sampling records of bwd_data_tc.cu, written at
+// the same index.
 bool gxt_supported(const Shape& s);
 size_t gxt_workspace(const Shape& s);
 cudaError_t gxt(const Shape& s, const void* off, const void* mask, const void* w, const void* gy, float* gx,
-                uint8_t* ovf, int ovf_pitch, void* ws, size_t ws_bytes, unsigned* status, cudaStream_t st,
-                int* launches);
+                uint8_t* ovf, void* rec, int ovf_pitch, void* ws, size_t ws_bytes, unsigned* status,
+                cudaStream_t st, int* launches);
 
 // bwd_weight_tc.cu — bfloat16 weight gradient on tcgen05 (workspace: sampling records).
 bool bwd_weight_tc_supported(const Shape& s);
