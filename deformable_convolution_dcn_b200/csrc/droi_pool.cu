@@ -22,6 +22,7 @@
 // order in shared memory (no atomics).
 #include "common.cuh"
 #include "kernels.h"
+#include "tc_ptx.cuh"
 
 namespace dcn {
 namespace {
@@ -83,6 +84,34 @@ template <typename T>
 __device__ __forceinline__ float px_or_zero(const T* xb, const RoiArgs& a, int r, int q, int c) {
     if (r < 0 || r >= a.H || q < 0 || q >= a.W) return 0.f;
     return ldf(xb + ((size_t)r * a.W + q) * a.C + c);
+}
+
+// A bin's samples sit on a unit grid (rows y1 + dy + u, columns x1 + dx + v):
+// all share the fractions (ly, lx), and sample u's bilinear rows are
+// fy + u and fy + u + 1. Summed over the bin, the pixel rows fy + u_lo + a,
+// a = 0 .. nu (nu = the number of sample rows), weigh wy(a) = 1 - ly for the
+// first, ly for the last, 1 in between (and likewise the columns), so the bin
+// reads each of its (nu + 1) x (nv + 1) pixels once instead of four times per
+// sample. Sample positions are taken from the bin's first row and column.
+struct BinBox {
+    int y0, x0;   // top-left pixel of the box (may lie outside the map)
+    int nu, nv;   // sample rows and columns (the box is (nu + 1) x (nv + 1) pixels)
+    float ly, lx;
+};
+__device__ __forceinline__ BinBox bin_box(const BinGeom& g) {
+    BinBox bx;
+    const Corner q = corner(g.y1 + g.u_lo + g.dy, g.x1 + g.v_lo + g.dx);
+    bx.y0 = q.y0;
+    bx.x0 = q.x0;
+    bx.ly = q.ly;
+    bx.lx = q.lx;
+    bx.nu = max(g.u_hi - g.u_lo, 0);
+    bx.nv = max(g.v_hi - g.v_lo, 0);
+    return bx;
+}
+// the box weight of pixel row a (0 .. n) for n sample rows with fraction l
+__device__ __forceinline__ float box_w(int a, int n, float l) {
+    return (a < n ? 1.f - l : 0.f) + (a > 0 ? l : 0.f);
 }
 
 template <typename T>
@@ -169,19 +198,21 @@ __global__ void __launch_bounds__(256) droi_fwd_vec_kernel(RoiArgs a, const T* _
         return;
     }
     const T* xb = x + (size_t)g.b * a.H * a.W * a.C;
+    const BinBox bx = bin_box(g);
     for (int cv = threadIdx.x; cv < nv; cv += blockDim.x) {
         const int c = cv * N;
         float acc[N];
 #pragma unroll
         for (int e = 0; e < N; ++e) acc[e] = 0.f;
-        for (int u = g.u_lo; u < g.u_hi; ++u)
-            for (int v = g.v_lo; v < g.v_hi; ++v) {
-                const Corner q = corner(g.y1 + u + g.dy, g.x1 + v + g.dx);
-#pragma unroll
-                for (int nb = 0; nb < 4; ++nb) {
-                    const int rr = q.y0 + (nb >> 1), cc = q.x0 + (nb & 1);
-                    if (rr < 0 || rr >= a.H || cc < 0 || cc >= a.W) continue;
-                    const float wt = ((nb >> 1) ? q.ly : 1.f - q.ly) * ((nb & 1) ? q.lx : 1.f - q.lx);
+        if (bx.nu > 0 && bx.nv > 0)
+            for (int ra = 0; ra <= bx.nu; ++ra) {
+                const int rr = bx.y0 + ra;
+                if (rr < 0 || rr >= a.H) continue;
+                const float wy = box_w(ra, bx.nu, bx.ly);
+                for (int cb = 0; cb <= bx.nv; ++cb) {
+                    const int cc = bx.x0 + cb;
+                    if (cc < 0 || cc >= a.W) continue;
+                    const float wt = wy * box_w(cb, bx.nv, bx.lx);
                     float vv[N];
                     load16(xb + ((size_t)rr * a.W + cc) * a.C + c, vv);
 #pragma unroll
@@ -257,6 +288,94 @@ __global__ void __launch_bounds__(256) droi_bwd_kernel(RoiArgs a, const T* __res
     }
 }
 
+// As droi_bwd_kernel, 16 bytes of channels per thread over the bin's pixel box
+// (BinBox): grad_x gets each box pixel's share m/n * grad_y * wy * wx once, by
+// 16-byte vector atomics; the offset gradients telescope over the sample rows
+// (columns) to the box's last minus its first pixel row (column), and the mask
+// gradient is the box sum. C a multiple of 16 bytes; x, grad_y and grad_x
+// 16-byte aligned.
+template <typename T>
+__global__ void __launch_bounds__(256) droi_bwd_vec_kernel(RoiArgs a, const T* __restrict__ x,
+                                                           const T* __restrict__ off, const T* __restrict__ mask,
+                                                           const T* __restrict__ gy, float* __restrict__ gx,
+                                                           float* __restrict__ goff, float* __restrict__ gmask) {
+    constexpr int N = Vec16<T>::N;
+    __shared__ float red[3][256];
+    const int bin = blockIdx.x, kk = a.k * a.k;
+    const int r = bin / kk, t = bin - r * kk;
+    const BinGeom g = bin_geom(a, off, mask, r, t);
+    float s_dy = 0.f, s_dx = 0.f, s_m = 0.f;
+    const BinBox bx = bin_box(g);
+    if (g.b >= 0 && bx.nu > 0 && bx.nv > 0) {
+        const T* xb = x + (size_t)g.b * a.H * a.W * a.C;
+        float* gxb = gx + (size_t)g.b * a.H * a.W * a.C;
+        const T* gyb = gy + (size_t)bin * a.C;
+        for (int cv = threadIdx.x; cv < a.C / N; cv += blockDim.x) {
+            const int c = cv * N;
+            float gc[N], gm[N], dyv[N], dxv[N], mv[N];
+            load16(gyb + c, gc);
+#pragma unroll
+            for (int e = 0; e < N; ++e) {
+                gc[e] /= g.n;
+                gm[e] = gc[e] * g.m;
+                dyv[e] = dxv[e] = mv[e] = 0.f;
+            }
+            for (int ra = 0; ra <= bx.nu; ++ra) {
+                const int rr = bx.y0 + ra;
+                if (rr < 0 || rr >= a.H) continue;
+                const float wy = box_w(ra, bx.nu, bx.ly);
+                const float sy = ra == bx.nu ? 1.f : (ra == 0 ? -1.f : 0.f);
+                for (int cb = 0; cb <= bx.nv; ++cb) {
+                    const int cc = bx.x0 + cb;
+                    if (cc < 0 || cc >= a.W) continue;
+                    const float wx = box_w(cb, bx.nv, bx.lx), wt = wy * wx;
+                    const float sx = cb == bx.nv ? 1.f : (cb == 0 ? -1.f : 0.f);
+                    const size_t o = ((size_t)rr * a.W + cc) * a.C + c;
+                    float vv[N];
+                    load16(xb + o, vv);
+                    if (wt != 0.f)  // a box edge of zero weight (a fraction of exactly 0) adds nothing
+#pragma unroll
+                        for (int q = 0; q < N; q += 4)
+                            ptx::red_add_v4(gxb + o + q, gm[q] * wt, gm[q + 1] * wt, gm[q + 2] * wt, gm[q + 3] * wt);
+#pragma unroll
+                    for (int e = 0; e < N; ++e) {
+                        mv[e] += wt * vv[e];
+                        dyv[e] += (sy * wx) * vv[e];
+                        dxv[e] += (sx * wy) * vv[e];
+                    }
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < N; ++e) {
+                s_dy += gm[e] * dyv[e];
+                s_dx += gm[e] * dxv[e];
+                s_m += gc[e] * mv[e];
+            }
+        }
+    }
+    if (goff == nullptr && gmask == nullptr) return;
+    red[0][threadIdx.x] = s_dy;
+    red[1][threadIdx.x] = s_dx;
+    red[2][threadIdx.x] = s_m;
+    __syncthreads();
+    for (int st = blockDim.x / 2; st > 0; st >>= 1) {
+        if ((int)threadIdx.x < st) {
+            red[0][threadIdx.x] += red[0][threadIdx.x + st];
+            red[1][threadIdx.x] += red[1][threadIdx.x + st];
+            red[2][threadIdx.x] += red[2][threadIdx.x + st];
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        const bool live = g.b >= 0;
+        if (goff) {
+            goff[(size_t)r * 2 * kk + 2 * t] = live ? red[0][0] * a.gamma * g.h : 0.f;
+            goff[(size_t)r * 2 * kk + 2 * t + 1] = live ? red[1][0] * a.gamma * g.w : 0.f;
+        }
+        if (gmask) gmask[(size_t)r * kk + t] = live ? red[2][0] : 0.f;
+    }
+}
+
 // a power of two from 32 to 256 covering the channels (the reduction halves it)
 int block_for(int C) {
     int t = 32;
@@ -292,7 +411,16 @@ cudaError_t droi_backward(const RoiArgs& a, int dtype_bf16, const void* x, const
                           const void* gy, float* gx, float* goff, float* gmask, cudaStream_t st) {
     const long long bins = (long long)a.R * a.k * a.k;
     if (bins == 0) return cudaSuccess;
-    if (dtype_bf16)
+    const int es = dtype_bf16 ? 2 : 4, n = 16 / es;
+    const bool vec = a.C % n == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0 &&
+                     (reinterpret_cast<uintptr_t>(gy) & 15) == 0 && (reinterpret_cast<uintptr_t>(gx) & 15) == 0;
+    if (vec && dtype_bf16)
+        droi_bwd_vec_kernel<bf16><<<(unsigned)bins, block_for(a.C / n), 0, st>>>(
+            a, (const bf16*)x, (const bf16*)off, (const bf16*)mask, (const bf16*)gy, gx, goff, gmask);
+    else if (vec)
+        droi_bwd_vec_kernel<float><<<(unsigned)bins, block_for(a.C / n), 0, st>>>(
+            a, (const float*)x, (const float*)off, (const float*)mask, (const float*)gy, gx, goff, gmask);
+    else if (dtype_bf16)
         droi_bwd_kernel<bf16><<<(unsigned)bins, block_for(a.C), 0, st>>>(
             a, (const bf16*)x, (const bf16*)off, (const bf16*)mask, (const bf16*)gy, gx, goff, gmask);
     else
