@@ -317,6 +317,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                             S[h][n] = fmaf(__uint_as_float(G[4 * m + 2 * h + 1]), bf_hi(v[h][n][m]), S[h][n]);
                         }
                 if (sc[0] | sc[1]) {
+                    // after the transposed pass has stored grad_x (a no-op unless launched as its dependent)
+                    asm volatile("griddepcontrol.wait;" ::: "memory");
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const float ly = rc[h].x, lx = rc[h].y, mk = rc[h].z;
@@ -731,7 +733,24 @@ cudaError_t bwd_data_tc(const Shape& s, const void* x, const void* off, const vo
     a.stages = pl.stages;
     a.kchunks = pl.kchunks;
     a.total_units = pl.total_units;
-    kernel<<<pl.ctas, NUM_THREADS, pl.smem_bytes, st>>>(map_dy, map_wt, a);
+    if (ovf) {
+        // after the transposed pass: a programmatic dependent, whose CTAs start on the SMs that pass
+        // frees and wait for it before their first grad_x atomic
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)pl.ctas);
+        cfg.blockDim = dim3(NUM_THREADS);
+        cfg.dynamicSmemBytes = pl.smem_bytes;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, kernel, map_dy, map_wt, a);
+        if (e != cudaSuccess) return e;
+    } else {
+        kernel<<<pl.ctas, NUM_THREADS, pl.smem_bytes, st>>>(map_dy, map_wt, a);
+    }
     ++n;
     if (launches) *launches += n;
     return cudaGetLastError();

@@ -261,6 +261,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // (barriers, TMEM, the stream-K plan) overlapped its tail; the records, W'
     // and the tile counters it writes are read only after this point.
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    // MODE 1: the backward-data kernel that follows may start on the SMs this
+    // grid leaves; it waits for this grid before it adds into grad_x, and what
+    // it reads was complete before this point
+    if constexpr (MODE == 1) asm volatile("griddepcontrol.launch_dependents;");
 
     const int cta = blockIdx.x;
     const long long ubeg = s_starts[cta], uend = s_starts[cta + 1];
