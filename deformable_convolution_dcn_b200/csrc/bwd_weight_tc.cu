@@ -133,6 +133,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::tc_fence_after();
     const uint32_t tmem_base = *s_tmem;
     const long long ubeg = unit_begin(blockIdx.x, a), uend = unit_begin(blockIdx.x + 1, a);
+    // launched as a programmatic dependent of the records kernel (which the weight warp
+    // waits for below); a bias-gradient kernel after this one may start alongside
+    asm volatile("griddepcontrol.launch_dependents;");
 
     if (warp >= PROD_WARP0) {
         // ------------------------------------------------------ producers --
@@ -205,6 +208,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
     } else if (warp == TMA_WARP) {
         // ------------------------------------------ grad_y tiles + records --
+        asm volatile("griddepcontrol.wait;" ::: "memory");  // the records are written
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0, issued = 0, issued_par = 0;
@@ -350,6 +354,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 __global__ void __launch_bounds__(256) dcn_records_kernel(Shape s, const bf16* __restrict__ off,
                                                           const bf16* __restrict__ mask, uint4* __restrict__ rec,
                                                           int ppad) {
+    // the main kernel may start: it reads the records only after a griddepcontrol.wait
+    asm volatile("griddepcontrol.launch_dependents;");
     const int p = blockIdx.x * blockDim.x + threadIdx.x;
     const int gt = blockIdx.y;
     if (p >= ppad) return;
@@ -444,11 +450,11 @@ cudaError_t bwd_weight_tc(const Shape& s, const void* x, const void* off, const 
     cudaError_t e = max_dynamic_smem_once((const void*)dcn_bwd_weight_tc_kernel, 227 * 1024, attr_set);
     if (e != cudaSuccess) return e;
     uint4* rec = reinterpret_cast<uint4*>(ws);
+    e = cudaMemsetAsync(gw, 0, sizeof(float) * (size_t)s.Cout * s.KC, st);
+    if (e != cudaSuccess) return e;
     dim3 rg((pl.ppad + 255) / 256, s.G * s.K2);
     dcn_records_kernel<<<rg, 256, 0, st>>>(s, (const bf16*)off, (const bf16*)mask, rec, pl.ppad);
     e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    e = cudaMemsetAsync(gw, 0, sizeof(float) * (size_t)s.Cout * s.KC, st);
     if (e != cudaSuccess) return e;
     BwArgs a;
     a.s = s;
@@ -467,7 +473,18 @@ cudaError_t bwd_weight_tc(const Shape& s, const void* x, const void* off, const 
     a.a_bytes = pl.a_bytes;
     a.stage_bytes = pl.stage_bytes;
     a.bar_off = pl.bar_off;
-    dcn_bwd_weight_tc_kernel<<<pl.ctas, NUM_THREADS, pl.smem_bytes, st>>>(map, a);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)pl.ctas);
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = pl.smem_bytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, dcn_bwd_weight_tc_kernel, map, a);
+    if (e != cudaSuccess) return e;
     if (launches) *launches += 3;
     return cudaGetLastError();
 }

@@ -343,7 +343,14 @@ int dcn_backward_weight(const dcn_params_t* params, const void* x, const void* o
     TRY(check_ptr(grad_bias, "grad_bias", 4, false));
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e;
+    if (grad_bias) {  // zeroed first, so that its kernel can follow the weight kernel's launch directly
+        e = cudaMemsetAsync(grad_bias, 0, sizeof(float) * (size_t)s.Cout, st);
+        g_launches += 1;
+        if (e != cudaSuccess) return cuda_fail(e, "zeroing grad_bias");
+    }
+    bool tc = false;
     if (use_bwd_weight_tc(params, s) && aligned16(x) && aligned16(grad_y) && aligned16(grad_weight)) {
+        tc = true;
         const size_t need = dcn::bwd_weight_tc_workspace(s);
         if (!workspace || workspace_bytes < need)
             return fail(DCN_ERR_WORKSPACE, "backward-weight needs %zu bytes of workspace, got %zu", need,
@@ -364,10 +371,8 @@ int dcn_backward_weight(const dcn_params_t* params, const void* x, const void* o
         if (e != cudaSuccess) return cuda_fail(e, "backward-weight launch");
     }
     if (grad_bias) {
-        e = cudaMemsetAsync(grad_bias, 0, sizeof(float) * (size_t)s.Cout, st);
-        g_launches += 1;
-        if (e != cudaSuccess) return cuda_fail(e, "zeroing grad_bias");
-        e = dcn::bias_grad(s, params->dtype, grad_y, grad_bias, st);
+        // after the tensor-core weight kernel: a programmatic dependent that runs alongside it
+        e = dcn::bias_grad(s, params->dtype, grad_y, grad_bias, st, tc);
         g_launches += 1;
         if (e != cudaSuccess) return cuda_fail(e, "bias-gradient launch");
     }

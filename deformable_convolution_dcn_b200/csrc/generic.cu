@@ -389,17 +389,25 @@ cudaError_t generic_backward_weight(const Shape& s, int dtype, const void* x, co
                       : launch_generic_backward_weight<bf16>(s, x, off, mask, gy, gw, st);
 }
 
-cudaError_t bias_grad(const Shape& s, int dtype, const void* gy, float* gb, cudaStream_t st) {
+cudaError_t bias_grad(const Shape& s, int dtype, const void* gy, float* gb, cudaStream_t st, bool pdl) {
     const int esz = dtype == 0 ? 4 : 2, V = 16 / esz;
     if ((reinterpret_cast<uintptr_t>(gy) & 15) == 0 && s.Cout % V == 0 && s.Cout / V <= 256 && s.P > 0) {
         const int blocks = std::min<long long>(2 * 148, s.P);
         const int per_block = (int)((s.P + blocks - 1) / blocks);
         const int nb = (int)((s.P + per_block - 1) / per_block);
-        if (dtype == 0)
-            bias_grad_vec_kernel<float><<<nb, 256, 0, st>>>(s, (const float*)gy, gb, per_block);
-        else
-            bias_grad_vec_kernel<bf16><<<nb, 256, 0, st>>>(s, (const bf16*)gy, gb, per_block);
-        return cudaGetLastError();
+        // pdl: a programmatic dependent of the kernel before it, which neither writes
+        // grad_y nor reads grad_bias (the weight kernel): it may run alongside it
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)nb);
+        cfg.blockDim = dim3(256);
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = pdl ? 1 : 0;
+        if (dtype == 0) return cudaLaunchKernelEx(&cfg, bias_grad_vec_kernel<float>, s, (const float*)gy, gb, per_block);
+        return cudaLaunchKernelEx(&cfg, bias_grad_vec_kernel<bf16>, s, (const bf16*)gy, gb, per_block);
     }
     const int per = 64;
     dim3 g2((s.Cout + 255) / 256, (s.P + per - 1) / per);

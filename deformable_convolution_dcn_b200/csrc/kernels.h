@@ -18,7 +18,7 @@ cudaError_t generic_backward_data(const Shape& s, int dtype, const void* x, cons
                                   cudaStream_t st);
 cudaError_t generic_backward_weight(const Shape& s, int dtype, const void* x, const void* off, const void* mask,
                                     const void* gy, float* gw, cudaStream_t st);
-cudaError_t bias_grad(const Shape& s, int dtype, const void* gy, float* gb, cudaStream_t st);
+cudaError_t bias_grad(const Shape& s, int dtype, const void* gy, float* gb, cudaStream_t st, bool pdl = false);
 
 // fwd_tc.cu — bfloat16 forward on tcgen05 tensor cores with the fused deformable gather.
 bool fwd_tc_supported(const Shape& s);
