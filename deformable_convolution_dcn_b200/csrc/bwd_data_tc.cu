@@ -558,6 +558,8 @@ __global__ void __launch_bounds__(256) dcn_records_f32_kernel(Shape s, const bf1
 template <bool PERM>
 __global__ void __launch_bounds__(256) dcn_transpose_kernel(const bf16* __restrict__ w, bf16* __restrict__ wt,
                                                             int Cout, int KC) {
+    // the transposed pass's fill may run alongside (it waits for this grid before it completes)
+    asm volatile("griddepcontrol.launch_dependents;");
     __shared__ bf16 t[32][33];
     const int k0 = blockIdx.x * 32, o0 = blockIdx.y * 32;
     for (int i = threadIdx.y; i < 32; i += 8) {
@@ -670,6 +672,11 @@ cudaError_t bwd_data_tc(const Shape& s, const void* x, const void* off, const vo
     e = smem_carveout_for((const void*)kernel, pl.smem_bytes, carve[pl.epi]);
     if (e != cudaSuccess) return e;
     int n = 0;
+    if (gx && pl.gxt) {
+        e = gxt_prepare(s, static_cast<uint8_t*>(ws) + pl.ovf_off, pl.ppad, static_cast<uint8_t*>(ws) + pl.gxt_off,
+                        ws_bytes - pl.gxt_off, st, &n);
+        if (e != cudaSuccess) return e;
+    }
     dim3 tg((s.KC + 31) / 32, (s.Cout + 31) / 32);
     if (pl.epi) dcn_transpose_kernel<true><<<tg, dim3(32, 8), 0, st>>>((const bf16*)w, wt, s.Cout, s.KC);
     else dcn_transpose_kernel<false><<<tg, dim3(32, 8), 0, st>>>((const bf16*)w, wt, s.Cout, s.KC);

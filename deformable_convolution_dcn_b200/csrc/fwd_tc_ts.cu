@@ -833,13 +833,10 @@ __device__ __forceinline__ int raster_to_strip(int q, int H, int W, int sw, int 
 // record for the backward-data kernel (rec[gt * ovf_pitch + p]: fractions,
 // mask, (y0 + 1) << 16 | (x0 + 1), or all bits set when no corner is inside).
 constexpr int LIST_CAP = 2 * LIST_E;
-__global__ void __launch_bounds__(256) dcn_gxt_fill_kernel(const Shape s, const bf16* __restrict__ off,
-                                                           const bf16* __restrict__ mask, int* __restrict__ cnt,
-                                                           unsigned long long* __restrict__ keys,
-                                                           uint8_t* __restrict__ ovf, float4* __restrict__ rec,
-                                                           int ovf_pitch, int mtiles_v, int sw, int nf, int wl) {
-    // the pre-pass may start: its weight blocks do not read what this grid writes
-    asm volatile("griddepcontrol.launch_dependents;");
+__device__ __forceinline__ void gxt_fill(const Shape& s, const bf16* __restrict__ off, const bf16* __restrict__ mask,
+                                         int* __restrict__ cnt, unsigned long long* __restrict__ keys,
+                                         uint8_t* __restrict__ ovf, float4* __restrict__ rec, int ovf_pitch,
+                                         int mtiles_v, int sw, int nf, int wl) {
     const int p = blockIdx.x * blockDim.x + threadIdx.x;
     const int gt = blockIdx.y >> 2, n = blockIdx.y & 3;
     if (p >= s.P) return;
@@ -875,6 +872,19 @@ __global__ void __launch_bounds__(256) dcn_gxt_fill_kernel(const Shape s, const 
         const size_t at = (size_t)gt * ovf_pitch + p;
         atomicOr(reinterpret_cast<unsigned*>(ovf + (at & ~(size_t)3)), (1u << n) << (8 * (at & 3)));
     }
+}
+__global__ void __launch_bounds__(256) dcn_gxt_fill_kernel(const Shape s, const bf16* __restrict__ off,
+                                                           const bf16* __restrict__ mask, int* __restrict__ cnt,
+                                                           unsigned long long* __restrict__ keys,
+                                                           uint8_t* __restrict__ ovf, float4* __restrict__ rec,
+                                                           int ovf_pitch, int mtiles_v, int sw, int nf, int wl) {
+    // the pre-pass may start: its weight blocks do not read what this grid writes
+    asm volatile("griddepcontrol.launch_dependents;");
+    gxt_fill(s, off, mask, cnt, keys, ovf, rec, ovf_pitch, mtiles_v, sw, nf, wl);
+    // launched as a programmatic dependent of the backward-data transpose (which writes nothing
+    // this grid touches): this grid completes only after it, so that everything after the
+    // pre-pass may take both as done
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // Pre-pass of one group's launch. Blocks [0, wblocks): W' of the virtual layer,
@@ -1123,6 +1133,17 @@ cudaError_t fwd_ts(const Shape& s, const void* x, const void* off, const void* m
 
 bool gxt_supported(const Shape& s) { return make_gxt_plan(s, num_sms()).ok; }
 
+cudaError_t gxt_prepare(const Shape& s, uint8_t* ovf, int ovf_pitch, void* ws, size_t ws_bytes, cudaStream_t st,
+                        int* launches) {
+    const GxtPlan gp = make_gxt_plan(s, num_sms());
+    if (!gp.ok || !ws || ws_bytes < gp.ws_bytes || ovf_pitch < s.P) return cudaErrorInvalidValue;
+    cudaError_t e = cudaMemsetAsync(static_cast<uint8_t*>(ws) + gp.cnt_off, 0, gp.lists * sizeof(int), st);
+    if (e != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(ovf, 0, (size_t)s.G * s.K2 * ovf_pitch, st)) != cudaSuccess) return e;
+    if (launches) *launches += 2;
+    return cudaSuccess;
+}
+
 size_t gxt_workspace(const Shape& s) {
     const GxtPlan gp = make_gxt_plan(s, num_sms());
     return gp.ok ? gp.ws_bytes : 0;
@@ -1144,19 +1165,29 @@ cudaError_t gxt(const Shape& s, const void* off, const void* mask, const void* w
     bf16* wperm = reinterpret_cast<bf16*>(tws + pl.ws_wperm_off);
     CUtensorMap map;
     if (!encode_wperm(&map, pl, v, wperm)) return cudaErrorInvalidValue;
-    cudaError_t e = cudaMemsetAsync(cnt, 0, gp.lists * sizeof(int), st);
-    if (e != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(ovf, 0, (size_t)s.G * s.K2 * ovf_pitch, st)) != cudaSuccess) return e;
-    dcn_gxt_fill_kernel<<<dim3((unsigned)((s.P + 255) / 256), (unsigned)(s.G * s.K2 * 4)), 256, 0, st>>>(
-        s, (const bf16*)off, (const bf16*)mask, cnt, keys, ovf, static_cast<float4*>(rec), ovf_pitch, pl.k.m_tiles,
-        pl.k.sw, pl.k.nf, pl.k.wl);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    cudaError_t e;
+    {
+        // a programmatic dependent of the kernel before it (the caller's transpose of W, which
+        // neither reads nor writes what the fill does); the counts and flags were zeroed by gxt_prepare
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)((s.P + 255) / 256), (unsigned)(s.G * s.K2 * 4));
+        cfg.blockDim = dim3(256);
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, dcn_gxt_fill_kernel, s, (const bf16*)off, (const bf16*)mask, cnt, keys, ovf,
+                               static_cast<float4*>(rec), ovf_pitch, pl.k.m_tiles, pl.k.sw, pl.k.nf, pl.k.wl);
+        if (e != cudaSuccess) return e;
+    }
     const bool wide = v.Cin % 16 == 0 && (reinterpret_cast<uintptr_t>(gy) & 31) == 0;
     const long long per_g = (long long)pl.k.m_tiles * s.K2 * BM;
     const long long nw = std::max<long long>((long long)v.Cout * pl.k.U * 8, pl.k.tiles);
     const int wblocks = (int)((nw + 255) / 256);
     const long long rblocks = (per_g + 255) / 256;
-    int n = 3;
+    int n = 1;
     for (int g = 0; g < s.G; ++g) {
         TsArgs ta = make_ts_args(pl, v, tws, counters, status);
         ta.f.x = (const bf16*)gy;

@@ -87,6 +87,10 @@ cudaError_t fwd_f32_small(const Shape& s, const void* x, const void* off, const 
 // the same index.
 bool gxt_supported(const Shape& s);
 size_t gxt_workspace(const Shape& s);
+// zeroes the lists' counts and the flags; enqueue it before the kernel that gxt's
+// first kernel follows (gxt launches it as that kernel's programmatic dependent)
+cudaError_t gxt_prepare(const Shape& s, uint8_t* ovf, int ovf_pitch, void* ws, size_t ws_bytes, cudaStream_t st,
+                        int* launches);
 cudaError_t gxt(const Shape& s, const void* off, const void* mask, const void* w, const void* gy, float* gx,
                 uint8_t* ovf, void* rec, int ovf_pitch, void* ws, size_t ws_bytes, unsigned* status,
                 cudaStream_t st, int* launches);
