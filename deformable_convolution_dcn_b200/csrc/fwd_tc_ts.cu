@@ -117,6 +117,7 @@ struct TsArgs {
     int ldy, col0;
     int ep_len, ep_taps;  // chunks per records epoch, taps held per record buffer
     int b_stages;
+    int band_pf;          // MODE 0: prefetch each next tile's input rows into L2 (inputs that do not stay in L2)
     uint32_t idle_bytes;  // shared memory free after the last MMA (the weight ring)
 };
 
@@ -165,6 +166,46 @@ __global__ void __launch_bounds__(256) dcn_fwd_prepass_kernel(const bf16* __rest
             v[h] = *reinterpret_cast<const uint2*>(w + (size_t)o * s.KC + (size_t)tap * s.Cin + (size_t)g * s.Cg + cg);
     }
     *reinterpret_cast<uint4*>(wp + ((size_t)o * U + u) * BK + 8 * k8) = make_uint4(v[0].x, v[0].y, v[1].x, v[1].y);
+}
+
+// The input rows a tile's samples can reach (its output rows' taps plus a
+// margin of BAND_MARGIN pixels for the offsets) into L2, one bulk prefetch per
+// input row, so that the gather of a tile whose input has left L2 meets L2
+// latency rather than DRAM latency. Issued for the next tile while the current
+// one is gathered; samples beyond the margin are simply fetched when needed.
+constexpr int BAND_MARGIN = 4;
+__device__ __forceinline__ void prefetch_strip_part(const FwdArgs& a, int b, int ho_lo, int ho_hi, int wo_lo,
+                                                    int wo_hi) {
+    const Shape& s = a.s;
+    const int reach = (s.K - 1) * s.dil + 1;
+    const int y_lo = max(0, ho_lo * s.stride - s.pad - BAND_MARGIN);
+    const int y_hi = min(s.H - 1, ho_hi * s.stride - s.pad + reach + BAND_MARGIN);
+    const int x_lo = max(0, wo_lo * s.stride - s.pad - BAND_MARGIN);
+    const int x_hi = min(s.W - 1, wo_hi * s.stride - s.pad + reach + BAND_MARGIN);
+    if (y_lo > y_hi || x_lo > x_hi) return;
+    const uint32_t bytes = (uint32_t)(x_hi - x_lo + 1) * (uint32_t)s.Cin * 2u;
+    for (int y = y_lo; y <= y_hi; ++y)
+        ptx::bulk_prefetch_l2(a.x + (((size_t)b * s.H + y) * s.W + x_lo) * s.Cin, bytes);
+}
+__device__ __forceinline__ void prefetch_tile_band(const FwdArgs& a, int t) {
+    const Shape& s = a.s;
+    const int mt = t / a.n_tiles;
+    const int r0 = mt * BM, r1 = min(r0 + BM, s.P) - 1;
+    const int p0 = strip_to_raster(r0, a), p1 = strip_to_raster(r1, a);
+    if (p0 < 0 || p1 < 0) return;
+    const int plane = s.Ho * s.Wo;
+    const int b0 = p0 / plane, b1 = p1 / plane;
+    const int ho0 = (p0 - b0 * plane) / s.Wo, wo0 = (p0 - b0 * plane) % s.Wo;
+    const int ho1 = (p1 - b1 * plane) / s.Wo, wo1 = (p1 - b1 * plane) % s.Wo;
+    const int st0 = min(wo0 / a.sw, a.nf), st1 = min(wo1 / a.sw, a.nf);  // strip index (nf: the narrow last one)
+    auto strip_lo = [&](int st) { return st * a.sw; };
+    auto strip_hi = [&](int st) { return st < a.nf ? st * a.sw + a.sw - 1 : s.Wo - 1; };
+    if (b0 == b1 && st0 == st1) {
+        prefetch_strip_part(a, b0, ho0, ho1, strip_lo(st0), strip_hi(st0));
+    } else {  // the tile ends one strip (or image) and begins the next
+        prefetch_strip_part(a, b0, ho0, s.Ho - 1, strip_lo(st0), strip_hi(st0));
+        prefetch_strip_part(a, b1, 0, ho1, strip_lo(st1), strip_hi(st1));
+    }
 }
 
 // Output column n0 of the tile's first row pointer, and the row pitch.
@@ -589,6 +630,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int seg = 0; seg < L.ns && ok; ++seg) {
             const Seg sg = seg_at(L, seg);
             const int t = sg.t;
+            if constexpr (MODE == 0) {
+                if (ta.band_pf && threadIdx.x == 0 && seg + 1 < L.ns) prefetch_tile_band(a, seg_at(L, seg + 1).t);
+            }
             while (rseg < L.ns && (rseg <= seg || (rseg == seg + 1 && rk == seg_at(L, rseg).k0))) {
                 const Seg rs = seg_at(L, rseg);
                 const int b = rec_epoch & 1;
@@ -1118,6 +1162,8 @@ cudaError_t fwd_ts(const Shape& s, const void* x, const void* off, const void* m
     ta.yf = nullptr;
     ta.ldy = s.Cout;
     ta.col0 = 0;
+    // an input of 64 MB or more does not stay in the 126 MB L2 between its tiles' gathers
+    ta.band_pf = (size_t)s.B * s.H * s.W * s.Cin * sizeof(bf16) >= ((size_t)64 << 20) ? 1 : 0;
     const long long nw = std::max<long long>((long long)s.Cout * pl.k.U * 8, pl.k.tiles);
     const int wblocks = (int)((nw + 255) / 256);
     const long long rblocks = (pl.nrec + 255) / 256;

@@ -137,6 +137,13 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
         : "memory");
 }
 
+// Asynchronous prefetch of `bytes` bytes from global memory into L2 (p 16-byte
+// aligned, bytes a multiple of 16); nothing waits for it.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+                 : "memory");
+}
+
 // Hint to bring the line holding p into this SM's L1 (no register result; an
 // address must still be a valid global address).
 __device__ __forceinline__ void prefetch_l1(const void* p) {
