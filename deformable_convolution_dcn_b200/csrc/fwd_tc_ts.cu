@@ -135,6 +135,9 @@ __global__ void __launch_bounds__(256) dcn_fwd_prepass_kernel(const bf16* __rest
     const Shape& s = a.s;
     // the main kernel may be scheduled now; it waits for this grid's completion before reading its outputs
     asm volatile("griddepcontrol.launch_dependents;");
+    // launched as a programmatic dependent of whatever the stream ran before (so that this grid's
+    // launch overlaps its tail): nothing is read or written before that work is complete
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     if ((int)blockIdx.x >= wblocks) {
         const long long r = (long long)(blockIdx.x - wblocks) * blockDim.x + threadIdx.x;
         if (r >= nrec) return;
@@ -1167,10 +1170,21 @@ cudaError_t fwd_ts(const Shape& s, const void* x, const void* off, const void* m
     const long long nw = std::max<long long>((long long)s.Cout * pl.k.U * 8, pl.k.tiles);
     const int wblocks = (int)((nw + 255) / 256);
     const long long rblocks = (pl.nrec + 255) / 256;
-    dcn_fwd_prepass_kernel<<<(unsigned)(wblocks + rblocks), 256, 0, st>>>((const bf16*)w, wperm, recs, a, wblocks,
-                                                                         pl.nrec);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    cudaError_t e;
+    {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(wblocks + rblocks));
+        cfg.blockDim = dim3(256);
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, dcn_fwd_prepass_kernel, (const bf16*)w, wperm, recs, (const FwdArgs)a, wblocks,
+                               pl.nrec);
+        if (e != cudaSuccess) return e;
+    }
     e = launch_ts<0>(pl, map, ta, wide, st);
     if (e != cudaSuccess) return e;
     if (launches) *launches += 2;
