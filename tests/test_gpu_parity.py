@@ -306,8 +306,9 @@ def _tf32_split_applies(s):
     # input rows staged in shared memory (a map row a whole number of 16 bytes), CTAs spanning two images
     (gen.LayerShape(B=2, Cin=3, H=40, W=32, Cout=64, K=3, stride=1, pad=1), True),
     (gen.LayerShape(B=1, Cin=3, H=12, W=16, Cout=64, K=3, stride=2, pad=1), True),
-    # more than three 128-row tiles per CTA: several rounds
+    # more than three 128-row tiles per CTA: several rounds (waves), one of them spanning two images
     (gen.LayerShape(B=1, Cin=1, H=250, W=240, Cout=32, K=3, stride=1, pad=1), True),
+    (gen.LayerShape(B=2, Cin=3, H=160, W=180, Cout=64, K=3, stride=1, pad=1), True),
 ], ids=lambda v: v if isinstance(v, bool) else "C%dx%dK%ds%dd%dG%d" % (v.Cin, v.Cout, v.K, v.stride, v.dil, v.G))
 def test_small_channel_f32_layers(shape, mask, kernel):
     """Float32 layers with few input channels, compared in full: the split-tf32
