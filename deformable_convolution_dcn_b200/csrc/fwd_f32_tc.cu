@@ -346,7 +346,7 @@ bool fwd_f32_tc_supported(const Shape& s) {
 
 cudaError_t fwd_f32_tc(const Shape& s, const void* x, const void* off, const void* mask, const void* w,
                        const void* bias, void* y, unsigned* status, cudaStream_t st) {
-    // up to 128 output channels: the persistent kernel of fwd_f32_stem.cu
+    // up to 128 output channels: the kernels of fwd_f32_stem.cu
     if (fwd_f32_stem_supported(s)) return fwd_f32_stem(s, x, off, mask, w, bias, y, status, st);
     const float *xf = (const float*)x, *of = (const float*)off, *mf = (const float*)mask, *wf = (const float*)w,
                 *bf = (const float*)bias;

@@ -68,8 +68,9 @@ bool fwd_f32_tc_supported(const Shape& s);
 cudaError_t fwd_f32_tc(const Shape& s, const void* x, const void* off, const void* mask, const void* w,
                        const void* bias, void* y, unsigned* status, cudaStream_t st);
 
-// fwd_f32_stem.cu — the same float32 layers with Cout <= 128 on a persistent, double-buffered
-// kernel (one CTA per SM over the 128-pixel tiles); fwd_f32_tc() dispatches to it where it applies.
+// fwd_f32_stem.cu — the same float32 layers with Cout <= 128, one CTA per SM over an equal share
+// of the output rows (a row-per-thread kernel for Cout 32 or 64, a persistent double-buffered one
+// above); fwd_f32_tc() dispatches to it where it applies.
 bool fwd_f32_stem_supported(const Shape& s);
 cudaError_t fwd_f32_stem(const Shape& s, const void* x, const void* off, const void* mask, const void* w,
                          const void* bias, void* y, unsigned* status, cudaStream_t st);
