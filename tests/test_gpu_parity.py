@@ -309,6 +309,8 @@ def _tf32_split_applies(s):
     # more than three 128-row tiles per CTA: several rounds (waves), one of them spanning two images
     (gen.LayerShape(B=1, Cin=1, H=250, W=240, Cout=32, K=3, stride=1, pad=1), True),
     (gen.LayerShape(B=2, Cin=3, H=160, W=180, Cout=64, K=3, stride=1, pad=1), True),
+    # no mask on the row-per-thread kernel (Cout <= 64)
+    (gen.LayerShape(B=2, Cin=2, H=15, W=21, Cout=64, K=3, stride=1, pad=1), False),
 ], ids=lambda v: v if isinstance(v, bool) else "C%dx%dK%ds%dd%dG%d" % (v.Cin, v.Cout, v.K, v.stride, v.dil, v.G))
 def test_small_channel_f32_layers(shape, mask, kernel):
     """Float32 layers with few input channels, compared in full: the split-tf32
@@ -327,4 +329,25 @@ def test_small_channel_f32_layers(shape, mask, kernel):
                     flags=flags)
     torch.cuda.synchronize()
     dcn.check_status()
+    assert_close(_cpu(y), _oracle_forward(shape, f64(d)), "f32", "y")
+
+
+@pytest.mark.parametrize("far", [100.0, -3.0e6])
+def test_stem_kernel_samples_off_the_band(far):
+    """The float32 stem kernel (Cin 3, Cout 64) when every sample misses its
+    staged band and the map (offsets of `far`, beyond the clamping bound in one
+    case): y equals the bias, which this kernel adds as a contraction column of
+    split tf32 parts, so to float32 rounding rather than bit for bit."""
+    shape = gen.LayerShape(B=2, Cin=3, H=14, W=20, Cout=64, K=3, stride=1, pad=1)
+    w = gen.Workload("smallc", shape, "f32", seed=5, offset_dist="normal1.5_edges", bias=True)
+    d = gen.make_inputs(w)
+    d["offset"] = torch.full_like(d["offset"], far)
+    p = dcn._params(d["x"], d["weight"], d["offset"], shape.stride, shape.pad, shape.dil, False)
+    assert dcn.forward_path(p) == "tcgen05_tf32_split"
+    dd = to_dev(d)
+    y = dcn.forward(dd["x"], dd["offset"], dd["mask"], dd["weight"], dd["bias"], shape.stride, shape.pad, shape.dil)
+    torch.cuda.synchronize()
+    dcn.check_status()
+    expect = np.broadcast_to(d["bias"].double().numpy(), y.shape)
+    assert_close(_cpu(y), expect, "f32", "y")
     assert_close(_cpu(y), _oracle_forward(shape, f64(d)), "f32", "y")
