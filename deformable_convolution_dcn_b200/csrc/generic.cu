@@ -301,20 +301,32 @@ __global__ void __launch_bounds__(256) bias_grad_vec_kernel(Shape s, const T* __
 #pragma unroll
     for (int v = 0; v < V; ++v) acc[v] = 0.f;
     if (pr < rows) {
-        for (int p = pbeg + pr; p < pend; p += rows) {
-            const uint4 q = __ldg(reinterpret_cast<const uint4*>(gy + (size_t)p * s.Cout) + g);
-            if constexpr (sizeof(T) == 2) {
-                const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+        // eight pixels' loads in flight before any is summed (a missing pixel reads as zero)
+        constexpr int BATCH = 8;
+        for (int p0 = pbeg + pr; p0 < pend; p0 += BATCH * rows) {
+            uint4 qs[BATCH];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    acc[2 * i] += __uint_as_float(w[i] << 16);
-                    acc[2 * i + 1] += __uint_as_float(w[i] & 0xFFFF0000u);
+            for (int u = 0; u < BATCH; ++u) {
+                const int p = p0 + u * rows;
+                qs[u] = p < pend ? __ldg(reinterpret_cast<const uint4*>(gy + (size_t)p * s.Cout) + g)
+                                 : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int u = 0; u < BATCH; ++u) {
+                const uint4 q = qs[u];
+                if constexpr (sizeof(T) == 2) {
+                    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        acc[2 * i] += __uint_as_float(w[i] << 16);
+                        acc[2 * i + 1] += __uint_as_float(w[i] & 0xFFFF0000u);
+                    }
+                } else {
+                    acc[0] += __uint_as_float(q.x);
+                    acc[1] += __uint_as_float(q.y);
+                    acc[2] += __uint_as_float(q.z);
+                    acc[3] += __uint_as_float(q.w);
                 }
-            } else {
-                acc[0] += __uint_as_float(q.x);
-                acc[1] += __uint_as_float(q.y);
-                acc[2] += __uint_as_float(q.z);
-                acc[3] += __uint_as_float(q.w);
             }
         }
 #pragma unroll
