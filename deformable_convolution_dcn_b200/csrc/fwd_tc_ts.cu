@@ -869,23 +869,24 @@ __device__ __forceinline__ int raster_to_strip(int q, int H, int W, int sw, int 
     return b * plane + nf * H * sw + y * wl + (xx - nf * sw);
 }
 
-// One thread per (output pixel p, group-tap gt, corner n): the corner's key
-// (p << 32 | n << 16 | bf16 weight) takes the next slot of its input pixel's
-// list (LIST_CAP slots; the count in cnt, zero on entry). A corner past the
-// last slot flags itself in ovf[gt * ovf_pitch + p] (bit n, zero on entry);
-// the pre-pass below sorts each list and keeps its LIST_E smallest keys, so
-// the lists and the flagged corners do not depend on the order of the
-// insertions. Corners outside the map or of zero (bf16) weight add nothing
-// and are skipped. The corner-0 thread also writes the sample's float32
-// record for the backward-data kernel (rec[gt * ovf_pitch + p]: fractions,
-// mask, (y0 + 1) << 16 | (x0 + 1), or all bits set when no corner is inside).
+// One thread per (output pixel p, group-tap gt), for the sample's four corners
+// n (their slot claims in flight together): a corner's key (p << 32 | n << 16
+// | bf16 weight) takes the next slot of its input pixel's list (LIST_CAP
+// slots; the count in cnt, zero on entry). A corner past the last slot is
+// flagged in ovf[gt * ovf_pitch + p] (bit n, zero on entry); the pre-pass
+// below sorts each list and keeps its LIST_E smallest keys, so the lists and
+// the flagged corners do not depend on the order of the insertions. Corners
+// outside the map or of zero (bf16) weight add nothing and are skipped. The
+// thread also writes the sample's float32 record for the backward-data kernel
+// (rec[gt * ovf_pitch + p]: fractions, mask, (y0 + 1) << 16 | (x0 + 1), or all
+// bits set when no corner is inside).
 constexpr int LIST_CAP = 2 * LIST_E;
 __device__ __forceinline__ void gxt_fill(const Shape& s, const bf16* __restrict__ off, const bf16* __restrict__ mask,
                                          int* __restrict__ cnt, unsigned long long* __restrict__ keys,
                                          uint8_t* __restrict__ ovf, float4* __restrict__ rec, int ovf_pitch,
                                          int mtiles_v, int sw, int nf, int wl) {
     const int p = blockIdx.x * blockDim.x + threadIdx.x;
-    const int gt = blockIdx.y >> 2, n = blockIdx.y & 3;
+    const int gt = blockIdx.y;
     if (p >= s.P) return;
     const int g = gt / s.K2, tap = gt - g * s.K2;
     const int plane = s.Ho * s.Wo;
@@ -900,24 +901,41 @@ __device__ __forceinline__ void gxt_fill(const Shape& s, const bf16* __restrict_
     float ly, lx;
     split_coord(ho * s.stride - s.pad + i * s.dil, dy, y0, ly);
     split_coord(wo * s.stride - s.pad + j * s.dil, dx, x0, lx);
-    if (n == 0 && rec) {
+    if (rec) {
         const bool any = inside(s, y0, x0) || inside(s, y0, x0 + 1) || inside(s, y0 + 1, x0) || inside(s, y0 + 1, x0 + 1);
         rec[(size_t)gt * ovf_pitch + p] =
             make_float4(ly, lx, mk, __uint_as_float(any ? (((uint32_t)(y0 + 1) << 16) | (uint32_t)(x0 + 1)) : 0xFFFFFFFFu));
     }
-    const int yy = y0 + (n >> 1), xx = x0 + (n & 1);
-    if (!inside(s, yy, xx)) return;
-    const float wf = ((n >> 1) ? ly : 1.f - ly) * ((n & 1) ? lx : 1.f - lx) * mk;
-    const unsigned short wb = __bfloat16_as_ushort(__float2bfloat16_rn(wf));
-    if ((wb & 0x7FFFu) == 0) return;
-    const int sr = raster_to_strip((b * s.H + yy) * s.W + xx, s.H, s.W, sw, nf, wl);
-    const size_t L = ((size_t)(g * mtiles_v + sr / BM) * s.K2 + tap) * BM + (sr % BM);
-    const int slot = atomicAdd(cnt + L, 1);
-    if (slot < LIST_CAP) {
-        keys[L * LIST_CAP + slot] = ((unsigned long long)p << 32) | ((unsigned long long)n << 16) | wb;
-    } else {
+    size_t L[4];
+    int slot[4];
+    unsigned short wbs[4];
+#pragma unroll
+    for (int n = 0; n < 4; ++n) {
+        slot[n] = -1;
+        L[n] = 0;
+        wbs[n] = 0;
+        const int yy = y0 + (n >> 1), xx = x0 + (n & 1);
+        if (!inside(s, yy, xx)) continue;
+        const float wf = ((n >> 1) ? ly : 1.f - ly) * ((n & 1) ? lx : 1.f - lx) * mk;
+        const unsigned short wb = __bfloat16_as_ushort(__float2bfloat16_rn(wf));
+        if ((wb & 0x7FFFu) == 0) continue;
+        const int sr = raster_to_strip((b * s.H + yy) * s.W + xx, s.H, s.W, sw, nf, wl);
+        L[n] = ((size_t)(g * mtiles_v + sr / BM) * s.K2 + tap) * BM + (sr % BM);
+        wbs[n] = wb;
+        slot[n] = atomicAdd(cnt + L[n], 1);
+    }
+    unsigned flags = 0;
+#pragma unroll
+    for (int n = 0; n < 4; ++n) {
+        if (slot[n] < 0) continue;
+        if (slot[n] < LIST_CAP)
+            keys[L[n] * LIST_CAP + slot[n]] = ((unsigned long long)p << 32) | ((unsigned long long)n << 16) | wbs[n];
+        else
+            flags |= 1u << n;
+    }
+    if (flags) {
         const size_t at = (size_t)gt * ovf_pitch + p;
-        atomicOr(reinterpret_cast<unsigned*>(ovf + (at & ~(size_t)3)), (1u << n) << (8 * (at & 3)));
+        atomicOr(reinterpret_cast<unsigned*>(ovf + (at & ~(size_t)3)), flags << (8 * (at & 3)));
     }
 }
 __global__ void __launch_bounds__(256) dcn_gxt_fill_kernel(const Shape s, const bf16* __restrict__ off,
@@ -1230,7 +1248,7 @@ cudaError_t gxt(const Shape& s, const void* off, const void* mask, const void* w
         // a programmatic dependent of the kernel before it (the caller's transpose of W, which
         // neither reads nor writes what the fill does); the counts and flags were zeroed by gxt_prepare
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)((s.P + 255) / 256), (unsigned)(s.G * s.K2 * 4));
+        cfg.gridDim = dim3((unsigned)((s.P + 255) / 256), (unsigned)(s.G * s.K2));
         cfg.blockDim = dim3(256);
         cfg.stream = st;
         cudaLaunchAttribute attr[1];
