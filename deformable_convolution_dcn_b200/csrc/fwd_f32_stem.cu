@@ -614,8 +614,9 @@ __global__ void __launch_bounds__(R_THREADS, 1)
         ptx::tmem_alloc(ptx::smem_u32(s_tmem), (uint32_t)a.tmem_cols);
         ptx::tmem_relinquish();
     }
-    bool ok = true;
-    int band_uses = 0, od_uses = 0;  // phases of band_bar, and of this thread's tile's od_bar, waited for
+    // phases of band_bar, and of this thread's tile's od_bar, waited for (a wait that gives up
+    // records the timeout in the status word and raises the abort flag, read at the next wave)
+    int band_uses = 0, od_uses = 0;
     if (waves > 0) {
         if (!(V.one_image && a.od_tma)) od_load(V);
         if (V.band && !a.band_bulk) band_load(V);
@@ -640,7 +641,7 @@ __global__ void __launch_bounds__(R_THREADS, 1)
     __syncthreads();  // barriers initialised before any thread waits on them
     if (waves > 0 && V.band) {
         if (a.band_bulk) {
-            ok = ptx::mbar_wait(ptx::smem_u32(band_bar), band_uses & 1, s_abort, a.status, WAIT_LIMIT) && ok;
+            ptx::mbar_wait(ptx::smem_u32(band_bar), band_uses & 1, s_abort, a.status, WAIT_LIMIT);
             ++band_uses;
             band_repack(V);
         } else {
@@ -670,7 +671,7 @@ __global__ void __launch_bounds__(R_THREADS, 1)
             if (!(V.one_image && a.od_tma)) od_load(V);
             if (V.band) {
                 if (a.band_bulk) {
-                    ok = ptx::mbar_wait(ptx::smem_u32(band_bar), band_uses & 1, s_abort, a.status, WAIT_LIMIT) && ok;
+                    ptx::mbar_wait(ptx::smem_u32(band_bar), band_uses & 1, s_abort, a.status, WAIT_LIMIT);
                     ++band_uses;
                     band_repack(V);
                 } else {
@@ -683,7 +684,7 @@ __global__ void __launch_bounds__(R_THREADS, 1)
         }
         const int trows = rows_of(V, tile);
         if (trows > 0 && V.one_image && a.od_tma) {
-            ok = ptx::mbar_wait(ptx::smem_u32(&od_bar[tile]), od_uses & 1, s_abort, a.status, WAIT_LIMIT) && ok;
+            ptx::mbar_wait(ptx::smem_u32(&od_bar[tile]), od_uses & 1, s_abort, a.status, WAIT_LIMIT);
             ++od_uses;
         }
         if (tid < V.nr) {
