@@ -244,10 +244,14 @@ def test_full_size_backward_sampled():
     (gen.LayerShape(B=2, Cin=128, H=20, W=18, Cout=64, K=7, pad=3), True),
 ], ids=["k7", "k7_g2_v1", "k7_s2_d2", "k7_c128"])
 def test_seven_by_seven_layers(shape, mask, dtype):
-    """K = 7 (49 taps, 98 offset channels per group), DCNv2 and DCNv1, forward and backward in full."""
+    """K = 7 (49 taps, 98 offset channels per group), DCNv2 and DCNv1, forward and backward in full;
+    the bf16 forward runs on the TMEM-operand tensor-core kernel."""
     w = gen.Workload("k7", shape, dtype, seed=17, offset_dist="uniform2.5",
                      mask_dist="uniform" if mask else "none", bias=True, backward=True)
     d = gen.make_inputs(w)
+    if dtype == "bf16":
+        p = dcn._params(d["x"], d["weight"], d["offset"], shape.stride, shape.pad, shape.dil, False)
+        assert dcn.forward_path(p) == "tcgen05_gather_tmem"
     a = f64(d)
     dd = to_dev(d)
     assert_close(_cpu(run_forward(shape, dd)), _oracle_forward(shape, a), dtype, "y")
