@@ -317,6 +317,9 @@ def _tf32_split_applies(s):
     (gen.LayerShape(B=2, Cin=2, H=15, W=21, Cout=64, K=3, stride=1, pad=1), False),
     # map rows too wide for the kernel's shared-memory band: every sample read from global memory
     (gen.LayerShape(B=1, Cin=3, H=6, W=1000, Cout=32, K=3, stride=1, pad=1), True),
+    # 1x1 and 2x2 kernels on the row-per-thread kernel
+    (gen.LayerShape(B=1, Cin=3, H=10, W=17, Cout=32, K=1, stride=1, pad=0), True),
+    (gen.LayerShape(B=2, Cin=2, H=11, W=13, Cout=64, K=2, stride=1, pad=0), True),
 ], ids=lambda v: v if isinstance(v, bool) else "C%dx%dK%ds%dd%dG%d" % (v.Cin, v.Cout, v.K, v.stride, v.dil, v.G))
 def test_small_channel_f32_layers(shape, mask, kernel):
     """Float32 layers with few input channels, compared in full: the split-tf32
